@@ -1,0 +1,25 @@
+"""Oracle package: TEST INFRASTRUCTURE ONLY (see ``oracle.paged_kv``).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` import this package.  The CUDA library and its Python binding do
+not, and this package imports nothing from them.
+"""
+
+from .paged_kv import (  # noqa: F401
+    BF16,
+    F16,
+    append_token,
+    attend,
+    copy_blocks,
+    decode_bits,
+    decode_sequence,
+    encode_bits,
+    free_request,
+    kv_head_of,
+    lse_combine,
+    materialize,
+    paged_attention_decode,
+    partial_state,
+    reshape_and_cache,
+    slot_location,
+)

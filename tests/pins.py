@@ -1,0 +1,384 @@
+"""Pins of the oracle to facts outside itself.
+
+Each ``check_*`` raises AssertionError when the oracle disagrees with what the
+pages, the mathematics or an independent computation fix.  They call the oracle
+through the module attribute (``O.name``) at call time, so a test can plant a
+mistake in the oracle with ``monkeypatch`` and confirm some check catches it.
+"""
+
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+import oracle.paged_kv as O
+import workloads as W
+from conftest import read_fixture
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rand_bits(rng, shape, dtype):
+    return W.to_bits(rng.standard_normal(shape, dtype=np.float32), dtype)
+
+
+# ---------------------------------------------------------------------------
+# Paging: block table, append rule, gather
+# ---------------------------------------------------------------------------
+
+def check_block_table_example():
+    """The page's Block Tables A = [3, 7, 12] and B = [1, 5, 9, 14]: tag every
+    (block, position) of a 16-block pool with a unique code and read the
+    requests back through their tables.  The expected sequences are written
+    block by block from the tables (16 tokens per block, in table order)."""
+    fx = read_fixture(os.path.join(GOLDEN, "block_table_example.txt"))
+    B = fx["block_size"][0]
+    pool = np.zeros((16, 1, B, 1), dtype=np.uint16)
+    for b in range(16):
+        for o in range(B):
+            pool[b, 0, o, 0] = b * 100 + o
+    exp_a = [300 + o for o in range(16)] + [700 + o for o in range(16)] + [1200 + o for o in range(16)]
+    exp_b = ([100 + o for o in range(16)] + [500 + o for o in range(16)]
+             + [900 + o for o in range(16)] + [1400 + o for o in range(16)])
+    for name, expected in (("table_A", exp_a), ("table_B", exp_b)):
+        table = np.array(fx[name], dtype=np.int32)
+        for length in (1, 15, 16, 17, 20, len(expected)):
+            got = O.materialize(pool, table, length, B)[0, :, 0].tolist()
+            assert got == expected[:length], (name, length)
+    # token 20 of request A sits in its second block (Block7) at position 4
+    assert O.materialize(pool, np.array(fx["table_A"]), 21, B)[0, 20, 0] == 704
+
+
+def check_append_rule_example():
+    fx = read_fixture(os.path.join(GOLDEN, "append_rule_example.txt"))
+    B = fx["block_size"][0]
+    free = list(fx["free_pool"])
+    table, slots = [], []
+    for t in range(fx["tokens"][0]):
+        slots.append(O.append_token(table, t, free, B))
+    assert table == fx["expect_table"]
+    for t in (0, 15, 16, 31, 32):
+        assert slots[t] == fx[f"expect_slot_token_{t}"][0], t
+    assert free == [8]
+    O.free_request(table, free)
+    assert free == fx["expect_free_after_finish"] and table == []
+
+
+def check_generator_follows_append_rule():
+    """Replaying the append rule token by token, with each sequence's blocks
+    as the free pool in table order, rebuilds the generated Block Tables and
+    the slot of every sequence's new token."""
+    batch = W.small_case(11, num_seqs=6, num_q_heads=4, num_kv_heads=2, head_dim=8,
+                         block_size=8, dtype=W.F16, max_len=40)
+    B = batch.block_size
+    for s in range(batch.num_seqs):
+        L = int(batch.context_lens[s])
+        nb = -(-L // B)
+        free = batch.block_tables[s, :nb].tolist()
+        table, slot = [], None
+        for t in range(L):
+            slot = O.append_token(table, t, free, B)
+        assert table == batch.block_tables[s, :nb].tolist()
+        assert slot == int(batch.slot_mapping[s])
+
+
+def check_materialize_roundtrip():
+    """Scatter a contiguous sequence into a shuffled pool one block slice at a
+    time; reading it back through the table returns it bit for bit."""
+    rng = np.random.default_rng(7)
+    for B, L in ((8, 1), (8, 8), (16, 37), (32, 100), (64, 64)):
+        Hkv, D = 3, 16
+        nb = -(-L // B)
+        N = nb + 5
+        table = rng.permutation(N)[:nb].astype(np.int32)
+        seq = rng.integers(0, 2 ** 16, size=(Hkv, L, D)).astype(np.uint16)
+        pool = rng.integers(0, 2 ** 16, size=(N, Hkv, B, D)).astype(np.uint16)
+        start = 0
+        for blk in table:
+            stop = min(start + B, L)
+            pool[blk, :, : stop - start, :] = seq[:, start:stop, :]
+            start = stop
+        assert np.array_equal(O.materialize(pool, table, L, B), seq), (B, L)
+
+
+# ---------------------------------------------------------------------------
+# Attention core: closed forms and special cases
+# ---------------------------------------------------------------------------
+
+def check_single_token_returns_value():
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((3, 16))
+    K = rng.standard_normal((1, 16)) * 10
+    V = rng.standard_normal((1, 16))
+    out = O.attend(q, K, V, 0.37)
+    assert np.array_equal(out, np.repeat(V, 3, axis=0))
+
+
+def check_two_token_sigmoid():
+    """With two keys the softmax weight of key 1 is the logistic function of
+    the score difference: out = s(D) v1 + (1 - s(D)) v0, D = scale q.(k1 - k0)."""
+    rng = np.random.default_rng(2)
+    for _ in range(20):
+        D = 8
+        q = rng.standard_normal(D)
+        K = rng.standard_normal((2, D)) * 2
+        V = rng.standard_normal((2, D))
+        scale = float(rng.uniform(0.05, 1.5))
+        delta = scale * sum(q[i] * (K[1, i] - K[0, i]) for i in range(D))
+        w1 = 1.0 / (1.0 + math.exp(-delta))
+        expected = [w1 * V[1, i] + (1.0 - w1) * V[0, i] for i in range(D)]
+        got = O.attend(q[None, :], K, V, scale)[0]
+        assert np.allclose(got, expected, rtol=0, atol=1e-13)
+
+
+def check_uniform_weights_give_mean():
+    """Equal keys, or scale 0, make every weight 1/L: the output is the mean of V."""
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((2, 12))
+    V = rng.standard_normal((9, 12))
+    K_equal = np.repeat(rng.standard_normal((1, 12)), 9, axis=0)
+    mean = V.sum(axis=0) / 9
+    assert np.allclose(O.attend(q, K_equal, V, 0.8), mean[None, :], rtol=0, atol=1e-14)
+    K = rng.standard_normal((9, 12))
+    assert np.allclose(O.attend(q, K, V, 0.0), mean[None, :], rtol=0, atol=1e-14)
+
+
+def check_dominant_key():
+    """A key aligned with the query and far larger than the others takes all
+    the weight: the output is that key's value (to within e^-gap)."""
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal(16)
+    K = rng.standard_normal((30, 16))
+    K[17] = 40.0 * q / np.linalg.norm(q)
+    V = rng.standard_normal((30, 16))
+    out = O.attend(q[None, :], K, V, 1.0)[0]
+    assert np.allclose(out, V[17], rtol=0, atol=1e-9)
+
+
+def check_against_torch_sdpa():
+    """Library special case: on the materialised sequences, decode attention
+    equals torch's scaled_dot_product_attention in float64 on the CPU (grouped
+    query heads expanded with ``repeat_interleave``)."""
+    import torch
+
+    for dtype in (W.F16, W.BF16):
+        batch = W.small_case(21, num_seqs=5, num_q_heads=8, num_kv_heads=2, head_dim=32,
+                             block_size=16, dtype=dtype, max_len=70, write_new_token=False)
+        out = O.paged_attention_decode(batch.q, batch.k_cache, batch.v_cache, batch.block_tables,
+                                       batch.context_lens, batch.block_size, batch.scale, dtype)
+        G = batch.num_q_heads // batch.num_kv_heads
+        for s in range(batch.num_seqs):
+            L = int(batch.context_lens[s])
+            K = O.decode_bits(O.materialize(batch.k_cache, batch.block_tables[s], L, 16), dtype)
+            V = O.decode_bits(O.materialize(batch.v_cache, batch.block_tables[s], L, 16), dtype)
+            q = torch.from_numpy(O.decode_bits(batch.q[s], dtype))[:, None, :]  # [Hq, 1, D]
+            Kt = torch.from_numpy(K).repeat_interleave(G, dim=0)  # [Hq, L, D]
+            Vt = torch.from_numpy(V).repeat_interleave(G, dim=0)
+            ref = torch.nn.functional.scaled_dot_product_attention(q, Kt, Vt, scale=batch.scale)
+            assert np.allclose(out[s], ref[:, 0, :].numpy(), rtol=0, atol=1e-12), (dtype, s)
+
+
+def check_gqa_grouping():
+    """Query head h reads kv head h // G: with V constant per kv head (value
+    g+1), every output element of head h equals h // G + 1."""
+    rng = np.random.default_rng(5)
+    Hq, Hkv, D, B, L = 8, 2, 8, 8, 11
+    N = 4
+    table = np.array([2, 0], dtype=np.int32)
+    k_cache = _rand_bits(rng, (N, Hkv, B, D), W.BF16)
+    v_cache = np.zeros((N, Hkv, B, D), dtype=np.uint16)
+    for g in range(Hkv):
+        v_cache[:, g] = W.to_bits(np.full((N, B, D), g + 1, np.float32), W.BF16)
+    q = _rand_bits(rng, (Hq, D), W.BF16)
+    out = O.decode_sequence(q, k_cache, v_cache, table, L, B, 0.3, W.BF16)
+    for h in range(Hq):
+        assert np.allclose(out[h], h // (Hq // Hkv) + 1, rtol=0, atol=1e-14), h
+
+
+def check_brute_force_tiny():
+    """An independent pure-Python evaluation on a tiny batch: every key and
+    value fetched token by token with its own table lookup, scores, softmax
+    and weighted sum written as loops."""
+    batch = W.small_case(31, num_seqs=3, num_q_heads=4, num_kv_heads=2, head_dim=4,
+                         block_size=4, dtype=W.F16, max_len=11, write_new_token=False)
+    out = O.paged_attention_decode(batch.q, batch.k_cache, batch.v_cache, batch.block_tables,
+                                   batch.context_lens, batch.block_size, batch.scale, W.F16)
+    Bs = batch.block_size
+    f16 = lambda b: float(np.uint16(b).view(np.float16))  # noqa: E731
+    for s in range(batch.num_seqs):
+        L = int(batch.context_lens[s])
+        for h in range(4):
+            g = h // 2
+            keys, vals = [], []
+            for i in range(L):
+                blk = int(batch.block_tables[s][i // Bs])
+                keys.append([f16(batch.k_cache[blk, g, i % Bs, d]) for d in range(4)])
+                vals.append([f16(batch.v_cache[blk, g, i % Bs, d]) for d in range(4)])
+            qv = [f16(batch.q[s, h, d]) for d in range(4)]
+            scores = [batch.scale * sum(qv[d] * k[d] for d in range(4)) for k in keys]
+            top = max(scores)
+            ws = [math.exp(z - top) for z in scores]
+            tot = sum(ws)
+            for d in range(4):
+                ref = sum(ws[i] * vals[i][d] for i in range(L)) / tot
+                assert abs(out[s, h, d] - ref) <= 1e-13, (s, h, d)
+
+
+def check_empty_sequence_is_zero():
+    rng = np.random.default_rng(6)
+    out = O.attend(rng.standard_normal((2, 8)), np.zeros((0, 8)), np.zeros((0, 8)), 1.0)
+    assert np.array_equal(out, np.zeros((2, 8)))
+
+
+# ---------------------------------------------------------------------------
+# Paging invariants
+# ---------------------------------------------------------------------------
+
+def _decode(batch, tables=None, k_cache=None, v_cache=None):
+    return O.paged_attention_decode(
+        batch.q, batch.k_cache if k_cache is None else k_cache,
+        batch.v_cache if v_cache is None else v_cache,
+        batch.block_tables if tables is None else tables, batch.context_lens,
+        batch.block_size, batch.scale, batch.dtype)
+
+
+def check_placement_invariance():
+    """Physical storage is decoupled from the logical view: moving every block
+    to another physical slot (and rewriting the tables) changes nothing."""
+    batch = W.small_case(41, num_seqs=4, num_q_heads=4, num_kv_heads=4, head_dim=16,
+                         block_size=8, dtype=W.BF16, max_len=60, write_new_token=False)
+    base = _decode(batch)
+    rng = np.random.default_rng(42)
+    N = batch.num_blocks
+    perm = rng.permutation(N)  # new home of block b is perm[b]
+    k2 = np.empty_like(batch.k_cache)
+    v2 = np.empty_like(batch.v_cache)
+    k2[perm] = batch.k_cache
+    v2[perm] = batch.v_cache
+    t2 = np.where(batch.block_tables >= 0, perm[np.maximum(batch.block_tables, 0)], -1).astype(np.int32)
+    assert np.array_equal(_decode(batch, t2, k2, v2), base)
+
+
+def check_table_padding_ignored():
+    """Table entries past a sequence's last block are never read: pointing them
+    at other sequences' blocks changes nothing."""
+    batch = W.small_case(43, num_seqs=5, num_q_heads=2, num_kv_heads=1, head_dim=8,
+                         block_size=8, dtype=W.F16, max_len=50, write_new_token=False)
+    base = _decode(batch)
+    rng = np.random.default_rng(44)
+    t2 = batch.block_tables.copy()
+    pad = t2 < 0
+    t2[pad] = rng.integers(0, batch.num_blocks, size=int(pad.sum()))
+    assert np.array_equal(_decode(batch, t2), base)
+
+
+def check_shared_prefix_equals_private_copy():
+    """Sequences reading a shared prefix block give the same output as after
+    copy-on-write gave each of them a private copy ([LSHU] 内存共享)."""
+    batch = W.prefix_share(45, num_seqs=6, prefix_tokens=40, suffix_range=(3, 20), num_q_heads=4,
+                           num_kv_heads=2, head_dim=16, block_size=16, dtype=W.F16)
+    # Block-aligned?  40 % 16 = 8: the copied block also receives new tokens,
+    # so compare on the pool state where no new token is written yet.
+    kc, vc = O.copy_blocks(batch.k_cache, batch.v_cache, batch.cow_pairs)
+    lens = batch.context_lens
+    # Attend over the prefix plus the suffix tokens stored before this step,
+    # i.e. up to the first position that is written in this step.
+    first_new = np.array([40] * batch.num_seqs, dtype=np.int32)
+    shared = O.paged_attention_decode(batch.q, kc, vc, batch.block_tables_before_cow, first_new,
+                                      16, batch.scale, batch.dtype)
+    private = O.paged_attention_decode(batch.q, kc, vc, batch.block_tables, first_new,
+                                       16, batch.scale, batch.dtype)
+    assert np.array_equal(shared, private)
+    assert np.all(np.isfinite(shared))
+    del lens
+
+
+def check_split_lse_combine():
+    """Merging the partial states of any partition of [0, L) reproduces the
+    unsplit softmax attention."""
+    rng = np.random.default_rng(8)
+    for trial in range(30):
+        L = int(rng.integers(1, 300))
+        G, D = 4, 16
+        q = rng.standard_normal((G, D))
+        K = rng.standard_normal((L, D)) * (1 + 4 * (trial % 3 == 0))
+        V = rng.standard_normal((L, D))
+        cuts = sorted(set(rng.integers(0, L + 1, size=int(rng.integers(0, 6))).tolist()) | {0, L})
+        parts = [O.partial_state(q, K[a:b], V[a:b], 0.2) for a, b in zip(cuts[:-1], cuts[1:])]
+        parts.append(O.partial_state(q, K[:0], V[:0], 0.2))  # an empty partition
+        ms = np.stack([p[0] for p in parts])
+        ls = np.stack([p[1] for p in parts])
+        os_ = np.stack([p[2] for p in parts])
+        assert np.allclose(O.lse_combine(ms, ls, os_), O.attend(q, K, V, 0.2), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Cache write, block copy, storage formats
+# ---------------------------------------------------------------------------
+
+def check_reshape_and_cache_example():
+    """Three new tokens with slots [5, -1, 18] in a pool of 8-token blocks:
+    token 0 lands in block 0 position 5, token 1 is padding, token 2 lands in
+    block 2 position 2; nothing else changes."""
+    N, Hkv, B, D = 4, 2, 8, 4
+    kc = np.full((N, Hkv, B, D), 0xAAAA, np.uint16)
+    vc = np.full((N, Hkv, B, D), 0x5555, np.uint16)
+    key = np.arange(3 * Hkv * D, dtype=np.uint16).reshape(3, Hkv, D) + 1
+    value = key + 1000
+    k2, v2 = O.reshape_and_cache(kc, vc, key, value, np.array([5, -1, 18]), B)
+    ek, ev = kc.copy(), vc.copy()
+    ek[0, :, 5, :] = key[0]
+    ev[0, :, 5, :] = value[0]
+    ek[2, :, 2, :] = key[2]
+    ev[2, :, 2, :] = value[2]
+    assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
+    assert np.all(kc == 0xAAAA)  # inputs untouched
+
+
+def check_copy_blocks_example():
+    N, Hkv, B, D = 6, 2, 4, 4
+    kc = np.arange(N * Hkv * B * D, dtype=np.uint16).reshape(N, Hkv, B, D)
+    vc = kc + 7
+    k2, v2 = O.copy_blocks(kc, vc, np.array([[1, 4], [3, 0]]))
+    ek, ev = kc.copy(), vc.copy()
+    ek[4], ev[4] = kc[1], vc[1]
+    ek[0], ev[0] = kc[3], vc[3]
+    assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
+
+
+def check_storage_formats():
+    """Known encodings: bf16 1.0 = 0x3F80, -2.0 = 0xC000, 0.1 = 0x3DCD (rounded
+    up from 0x3DCCCCCD), 1 + 2^-8 ties to even 0x3F80, 1 + 3*2^-8 ties to
+    0x3F82; fp16 1.0 = 0x3C00, 65504 = 0x7BFF, 2^-24 = 0x0001."""
+    b = O.encode_bits(np.array([1.0, -2.0, 0.1, 1 + 2 ** -8, 1 + 3 * 2 ** -8]), O.BF16)
+    assert b.tolist() == [0x3F80, 0xC000, 0x3DCD, 0x3F80, 0x3F82]
+    assert O.decode_bits(np.array([0x3F80, 0xC000, 0x3DCD], np.uint16), O.BF16).tolist() == \
+        [1.0, -2.0, 0.10009765625]
+    h = O.encode_bits(np.array([1.0, 65504.0, 2.0 ** -24]), O.F16)
+    assert h.tolist() == [0x3C00, 0x7BFF, 0x0001]
+    assert O.decode_bits(h, O.F16).tolist() == [1.0, 65504.0, 2.0 ** -24]
+
+
+ALL_CHECKS = [
+    check_block_table_example,
+    check_append_rule_example,
+    check_generator_follows_append_rule,
+    check_materialize_roundtrip,
+    check_single_token_returns_value,
+    check_two_token_sigmoid,
+    check_uniform_weights_give_mean,
+    check_dominant_key,
+    check_against_torch_sdpa,
+    check_gqa_grouping,
+    check_brute_force_tiny,
+    check_empty_sequence_is_zero,
+    check_placement_invariance,
+    check_table_padding_ignored,
+    check_shared_prefix_equals_private_copy,
+    check_split_lse_combine,
+    check_reshape_and_cache_example,
+    check_copy_blocks_example,
+    check_storage_formats,
+]

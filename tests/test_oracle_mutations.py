@@ -1,0 +1,111 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and confirm that at
+least one pin catches each of them."""
+
+import numpy as np
+import pytest
+
+import oracle.paged_kv as O
+from pins import ALL_CHECKS
+
+_orig_attend = O.attend
+_orig_materialize = O.materialize
+_orig_lse = O.lse_combine
+
+
+def _attend_no_scale(q, K, V, scale):
+    return _orig_attend(q, K, V, 1.0)
+
+
+def _attend_values_from_keys(q, K, V, scale):
+    return _orig_attend(q, K, K, scale)
+
+
+def _attend_softmax_wrong_axis(q, K, V, scale):
+    q = np.asarray(q, dtype=np.float64)
+    if K.shape[0] == 0:
+        return np.zeros((q.shape[0], V.shape[1]))
+    z = scale * (q @ K.T)
+    e = np.exp(z - z.max(axis=0, keepdims=True))
+    return (e / e.sum(axis=0, keepdims=True)) @ V
+
+
+def _attend_drop_last_token(q, K, V, scale):
+    return _orig_attend(q, K[:-1] if K.shape[0] > 1 else K, V[:-1] if V.shape[0] > 1 else V, scale)
+
+
+def _materialize_offset_shift(cache, table_row, length, block_size):
+    pos = np.arange(length)
+    blocks = np.asarray(table_row)[pos // block_size].astype(np.int64)
+    offs = (pos + 1) % block_size
+    return np.ascontiguousarray(cache[blocks, :, offs, :].transpose(1, 0, 2))
+
+
+def _materialize_heads_swapped(cache, table_row, length, block_size):
+    return _orig_materialize(cache, table_row, length, block_size)[::-1].copy()
+
+
+def _kv_head_modulo(h, num_q_heads, num_kv_heads):
+    return h % num_kv_heads
+
+
+def _slot_location_swapped(slot, block_size):
+    return int(slot) % block_size, int(slot) // block_size
+
+
+def _copy_blocks_reversed(k_cache, v_cache, block_pairs):
+    pairs = np.asarray(block_pairs).reshape(-1, 2)[:, ::-1]
+    k0, v0 = np.array(k_cache), np.array(v_cache)
+    kc, vc = k0.copy(), v0.copy()
+    for src, dst in pairs.tolist():
+        kc[dst], vc[dst] = k0[src], v0[src]
+    return kc, vc
+
+
+def _lse_unweighted_l(ms, ls, os):
+    M = ms.max(axis=0)
+    w = np.exp(ms - M)
+    w = np.where(np.isfinite(w), w, 0.0)
+    return (w[:, :, None] * os).sum(axis=0) / ls.sum(axis=0)[:, None]
+
+
+def _append_always_new_block(table, length, free_pool, block_size):
+    table.append(free_pool.pop(0))
+    return table[-1] * block_size
+
+
+def _encode_truncate(x, dtype):
+    x = np.asarray(x, dtype=np.float64)
+    if dtype == O.BF16:
+        return (x.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    return x.astype(np.float16).view(np.uint16)
+
+
+MUTANTS = {
+    "attend_drops_scale": ("attend", _attend_no_scale),
+    "attend_uses_keys_as_values": ("attend", _attend_values_from_keys),
+    "softmax_over_wrong_axis": ("attend", _attend_softmax_wrong_axis),
+    "attend_drops_last_token": ("attend", _attend_drop_last_token),
+    "gather_offset_off_by_one": ("materialize", _materialize_offset_shift),
+    "gather_heads_reversed": ("materialize", _materialize_heads_swapped),
+    "gqa_modulo_grouping": ("kv_head_of", _kv_head_modulo),
+    "slot_block_offset_swapped": ("slot_location", _slot_location_swapped),
+    "copy_blocks_direction_reversed": ("copy_blocks", _copy_blocks_reversed),
+    "lse_combine_unweighted_sum": ("lse_combine", _lse_unweighted_l),
+    "append_without_filling_block": ("append_token", _append_always_new_block),
+    "bf16_truncates_instead_of_rounding": ("encode_bits", _encode_truncate),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            check()
+        except AssertionError:
+            caught.append(check.__name__)
+        except (IndexError, ValueError):
+            caught.append(check.__name__ + " (raised)")
+    assert caught, f"no pin catches the planted mistake {name}"
