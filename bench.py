@@ -1,0 +1,485 @@
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of one attention layer over a seeded synthetic
+batch resident in HBM: ``copy_blocks`` for the batch's copy-on-write pairs
+(none in the default workload), ``reshape_and_cache`` of every sequence's new
+token, then ``paged_attention_decode`` (split-K attention kernel plus, when a
+sequence spans several partitions, the log-sum-exp merge kernel).
+
+Default workload: Llama-7B-shaped multi-head decode layer (64 sequences,
+32 q = 32 kv heads, head_dim 128, 16-token blocks, fp16, context lengths
+uniform on [128, 2048], pool = needed blocks + 10 %, shuffled).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Under torchrun every rank runs its own batch (weak scaling, seed + rank);
+ranks share no data and the only collectives are the barrier and the max of
+the timings.  Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s and tokens/s on 1 B200; % of HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/paged_attention.cu",
+                  "paged_kv_cache_407_b200/csrc/pkv_device.cuh"]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="llama7b_mha")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return p.parse_args(argv)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(PROFILE_DIR, f"paged_decode_kernel_{workload}.txt")
+    try:
+        kv = {}
+        with open(path, encoding="utf-8") as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(kv["dram_bytes_per_launch_full_workload"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ["timestamp", "uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+        self.window = None  # wall-clock (start, end) of the timed region
+
+    def mark(self, start: float, end: float):
+        self.window = (start, end)
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="pkv_clocks_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+        return False
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                if self.uuid and self.uuid not in parts[1]:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                except (ValueError, IndexError):
+                    ts = None
+                rows.append((ts, parts))
+        os.unlink(self.path)
+        if self.window is not None:
+            lo, hi = self.window
+            inside = [r for ts, r in rows if ts is not None and lo - 0.06 <= ts <= hi + 0.06]
+        else:
+            inside = []
+        used = inside if inside else [r for _, r in rows]
+        if not used:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [v for v in (num(r[2]) for r in used) if v is not None]
+        mx = [v for v in (num(r[3]) for r in used) if v is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in used for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(used),
+                "samples_in_timed_window": len(inside)}
+
+
+# ----------------------------------------------------------------- helpers
+def step_bytes(batch):
+    from paged_kv_cache_407_b200 import accounting as A
+
+    att = A.decode_bytes(batch.context_lens, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                         batch.block_size)
+    write = A.reshape_and_cache_bytes(batch.num_tokens, batch.num_kv_heads, batch.head_dim)
+    copy = A.copy_blocks_bytes(batch.cow_pairs.shape[0], batch.num_kv_heads, batch.block_size, batch.head_dim)
+    return att, write, copy
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_sample_rate(batch, seconds: float):
+    """Time the oracle's decode over whole sequences of the batch until about
+    ``seconds`` of CPU work; returns (GB/s, description, cores)."""
+    import oracle as O
+    from paged_kv_cache_407_b200 import accounting as A
+
+    order = np.random.default_rng(12345).permutation(batch.num_seqs)
+    done, t0 = [], time.perf_counter()
+    while len(done) < len(order) and time.perf_counter() - t0 < seconds:
+        s = int(order[len(done)])
+        O.decode_sequence(batch.q[s], batch.k_cache, batch.v_cache, batch.block_tables[s],
+                          int(batch.context_lens[s]), batch.block_size, batch.scale, batch.dtype)
+        done.append(s)
+    dt = time.perf_counter() - t0
+    b = A.decode_bytes(batch.context_lens[done], batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                       batch.block_size)["total"]
+    desc = (f"oracle decode (fp64 NumPy) of {len(done)} of {batch.num_seqs} sequences of the "
+            f"{batch.name} batch ({int(batch.context_lens[done].sum())} tokens), {dt:.1f} s")
+    return b / dt / 1e9, desc, blas_threads(), dt
+
+
+def build_workload(name: str, rank: int):
+    import workloads as W
+
+    fn = W.WORKLOADS[name]
+    base = {"tiny": 1, "llama7b_mha": 2, "gqa_write": 3, "prefix_share": 4, "long_context": 5}[name]
+    return fn(seed=base + 1000 * rank)
+
+
+def workload_config(batch, args, n_gpus):
+    lens = batch.context_lens
+    return {
+        "workload": batch.name,
+        "num_seqs_per_gpu": batch.num_seqs,
+        "global_batch": batch.num_seqs * n_gpus,
+        "num_q_heads": batch.num_q_heads,
+        "num_kv_heads": batch.num_kv_heads,
+        "head_dim": batch.head_dim,
+        "block_size": batch.block_size,
+        "context_len_mean": float(lens.mean()),
+        "context_len_max": int(lens.max()),
+        "pool_blocks": batch.num_blocks,
+        "pool_bytes": int(batch.k_cache.nbytes * 2),
+        "new_tokens_per_step": batch.num_tokens,
+        "cow_pairs_per_step": int(batch.cow_pairs.shape[0]),
+        "parallelism": f"dp{n_gpus} (independent sequences per GPU)",
+        "l2": "inputs larger than L2: the KV pool is re-read every step",
+    }
+
+
+def reduce_across_ranks(maxima, sums, device):
+    """Max of the timings and sum of the byte/sequence counts over all ranks
+    (identity on one process).  Every rank calls it once, in the same order."""
+    import torch
+    import torch.distributed as dist
+
+    t_max = torch.tensor(list(maxima), dtype=torch.float64, device=device)
+    t_sum = torch.tensor(list(sums), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+        dist.all_reduce(t_sum, op=dist.ReduceOp.SUM)
+    return t_max.tolist(), t_sum.tolist()
+
+
+# --------------------------------------------------------------- reference
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0  # the reference arm runs on rank 0 only
+    batch = build_workload(args.workload, 0)
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample_rate(batch, per_step)
+    rates, secs = [], 0.0
+    desc = ""
+    cores = 1
+    for _ in range(args.steps):
+        r, desc, cores, dt = oracle_sample_rate(batch, per_step)
+        rates.append(r)
+        secs += dt
+    value = float(statistics.median(rates))
+    att, _, _ = step_bytes(batch)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": workload_config(batch, args, 1),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": desc + "; each step a bounded sample of this workload"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "decode_tokens_per_s": round(value * 1e9 / att["total"] * batch.num_seqs, 2),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_407_b200 as pkv
+    from paged_kv_cache_407_b200.build import build
+    from workloads.device import upload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    pkv.library()
+
+    batch = build_workload(args.workload, rank)
+    db = upload(batch, dev)
+    ws_bytes = pkv.workspace_size(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                                  batch.block_size, batch.max_context_len, batch.partition_size)
+    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    P = pkv.partition_size(batch.num_seqs, batch.num_kv_heads, batch.block_size, batch.max_context_len,
+                           batch.partition_size)
+    split = batch.max_context_len > P
+    has_cow = batch.cow_pairs.shape[0] > 0
+    launches_per_step = 1 + 1 + (1 if split else 0) + (1 if has_cow else 0)
+
+    def step(q=db.q, out=db.out, key=db.key, value=db.value, slots=db.slot_mapping, tables=db.block_tables,
+             lens=db.context_lens, ev=None):
+        if has_cow:
+            pkv.copy_blocks(db.k_cache, db.v_cache, db.cow_pairs, d_status=status, stream=stream)
+        pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=status, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, batch.max_context_len,
+                                   batch.scale, partition_size=batch.partition_size, workspace=workspace,
+                                   d_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        pass
+    K = args.steps
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        wall0 = time.time()
+        t_start.record(stream)
+        for i in range(K):
+            step(ev=att_ev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks.mark(wall0, time.time())
+        if world > 1:
+            dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    att_ms = [a.elapsed_time(b) for a, b in att_ev]
+    clock = clocks.summary()
+
+    # -------- end to end through the public API, host buffers -----------
+    e2e = None
+    if not args.no_e2e:
+        h_in = {n: t.detach().cpu().pin_memory() for n, t in
+                (("q", db.q), ("key", db.key), ("value", db.value), ("slots", db.slot_mapping),
+                 ("tables", db.block_tables), ("lens", db.context_lens))}
+        d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
+        h_out = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            for n in h_in:
+                d_in[n].copy_(h_in[n], non_blocking=True)
+            step(q=d_in["q"], out=db.out, key=d_in["key"], value=d_in["value"], slots=d_in["slots"],
+                 tables=d_in["tables"], lens=d_in["lens"])
+            h_out.copy_(db.out, non_blocking=True)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = {"ms": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h}
+
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+    att_bytes, write_bytes, copy_bytes = step_bytes(batch)
+    att_ms_mean = float(np.mean(att_ms))
+    (ms_total, att_ms_max, e2e_ms), (bytes_all, seqs_all) = reduce_across_ranks(
+        [ms_total, att_ms_mean, e2e["ms"] if e2e else 0.0], [att_bytes["total"], batch.num_seqs], dev)
+    ms_step = ms_total / K
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, cores, _ = oracle_sample_rate(batch, args.cpu_seconds)
+        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_kind = measured_peak()
+    total_att_bytes = bytes_all  # every rank's own batch, summed
+    value = total_att_bytes / (ms_step * 1e-3) / 1e9
+    achieved = att_bytes["total"] / (att_ms_max * 1e-3) / 1e9
+    traffic = profiled_traffic(batch.name)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": batch.dtype,
+        "data": "synthetic (seeded generator, inputs resident in HBM)",
+        "config": workload_config(batch, args, world),
+        "decode_tokens_per_s": round(seqs_all / (ms_step * 1e-3), 1),
+        "decode_tokens_per_s_32_layer_attention_only": round(seqs_all / (ms_step * 1e-3) / 32, 1),
+        "bytes_per_step": {"attention": att_bytes["total"], "attention_kv": att_bytes["kv"],
+                           "cache_write": write_bytes, "block_copy": copy_bytes},
+        "attention_ms_per_call": round(att_ms_max, 5),
+        "split_k": {"partition_tokens": P, "split": bool(split)},
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "paged_attention_decode (attention kernel + log-sum-exp merge, timed together)",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+        },
+        "clocks": clock,
+        "gpu_launches": launches_per_step * K,
+    }
+    if e2e:
+        line["e2e"] = {"value": round(total_att_bytes / (e2e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_ms / K, 5)}
+    if cpu:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

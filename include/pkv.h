@@ -1,0 +1,204 @@
+/*
+ * pkv.h - C ABI of libpkv: the decode hot path of a paged KV cache on B200 (sm_100a).
+ *
+ * The KV cache of every attention layer is a pool of fixed-size physical
+ * blocks; each sequence reaches its tokens through its own Block Table, which
+ * maps logical block j (tokens j*B .. j*B+B-1) to a physical block id.  Sources:
+ *   lshu.cn/news/11644 (vLLM architecture analysis), section
+ *   "核心创新：PagedAttention 的设计逻辑": sub-section "方案：页式内存管理"
+ *   (blocks of 16 tokens, Block Table per request, append rule, the attention
+ *   kernel reading the scattered blocks through the table as one logical K/V
+ *   sequence) and "内存共享" (prefix blocks shared read-only, copy-on-write on
+ *   divergence); zzmblog.top "vLLM使用指南", section "核心原理 / Transformer推理
+ *   与KV缓存" (a decode step computes only the current token's K and V, appends
+ *   them to the cache, then computes attention).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named d_* or described as device memory are device pointers
+ *     owned by the caller.  The library allocates nothing and frees nothing.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) and returns once its kernels are queued.
+ *   - Host-detectable errors return a non-zero pkv_status before anything is
+ *     queued; outputs are then untouched.
+ *   - Errors that only the device can see (a block id outside the pool, a slot
+ *     outside the pool, a context length the call's bounds cannot hold, a wait
+ *     that ran out) are OR-ed as PKV_DEV_* bits into *d_status when d_status is
+ *     not NULL (an int32 in device memory, to be read after the stream
+ *     synchronises; the library never clears it).  Kernels never trap: an
+ *     offending element is skipped or masked and the flag is raised.
+ *   - The library keeps no mutable global state apart from a once-only lookup
+ *     of the driver's tensor-map encoder; calls are thread-safe.
+ *
+ * Cache layout ("HND"): k_cache and v_cache are separate pools, each
+ *   [num_blocks][num_kv_heads][block_size][head_dim] row-major, element type
+ *   fp16 or bf16.  Slot s names block s / block_size, position s % block_size.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pkv_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_NULL_POINTER = 1,   /* a required pointer is NULL */
+  PKV_ERR_BAD_DTYPE = 2,      /* dtype is not PKV_F16 / PKV_BF16 */
+  PKV_ERR_BAD_SHAPE = 3,      /* unsupported head_dim / block_size / head counts / negative size */
+  PKV_ERR_MISALIGNED = 4,     /* a pointer or stride breaks the stated alignment */
+  PKV_ERR_WORKSPACE = 5,      /* workspace NULL or smaller than pkv_paged_attention_workspace_size */
+  PKV_ERR_BAD_PARTITION = 6,  /* partition_size not a positive multiple of block_size */
+  PKV_ERR_TOO_LARGE = 7,      /* a size exceeds what the kernels index (see each call) */
+  PKV_ERR_CUDA = 8,           /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
+  PKV_ERR_DEVICE = 9          /* current device is not compute capability 10.0 (B200 / sm_100a) */
+} pkv_status;
+
+/* Device-side error bits OR-ed into *d_status. */
+#define PKV_DEV_BAD_BLOCK 0x1  /* a Block Table entry or copy pair outside [0, num_blocks) */
+#define PKV_DEV_BAD_SLOT 0x2   /* a slot >= num_blocks * block_size */
+#define PKV_DEV_BAD_LEN 0x4    /* context_len < 0, > max_context_len or > max_blocks_per_seq * block_size */
+#define PKV_DEV_TIMEOUT 0x8    /* a copy into shared memory did not complete within ~1 s */
+
+typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Shape of one layer's block pool (shared by k_cache and v_cache). */
+typedef struct {
+  int32_t num_blocks;   /* N >= 1 */
+  int32_t block_size;   /* B: tokens per block; 8, 16, 32 or 64 */
+  int32_t num_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim;     /* D: 64 or 128 */
+  pkv_dtype dtype;      /* element type of both pools, of queries and outputs */
+} pkv_cache_desc;
+
+/*
+ * pkv_reshape_and_cache - write this step's new K/V tokens into their slots.
+ *
+ * Passage: the append rule of lshu.cn/news/11644 "方案：页式内存管理" (a new
+ * token goes into the next free position of the sequence's last block, or of a
+ * block newly taken from the free pool) together with zzmblog.top
+ * "Transformer推理与KV缓存" (the step's K, V are appended before attention).
+ * The host decides the slots; this call performs the writes:
+ *   for t < num_tokens with p = slot_mapping[t] >= 0, for every kv head h:
+ *     k_cache[p / B][h][p % B][:] = key[t][h][:]   and the same for value.
+ * A negative slot marks a padding token and writes nothing.  Plain bit copy.
+ *
+ * key, value      device, [num_tokens][num_kv_heads][head_dim] with a token
+ *                 stride of key_token_stride / value_token_stride elements
+ *                 (0 means num_kv_heads*head_dim); heads of a token contiguous.
+ * k_cache,v_cache device, layout above, 16-byte aligned.
+ * slot_mapping    device, int64 [num_tokens].
+ * Errors: NULL pointers (when num_tokens > 0), bad desc -> status; a slot
+ *   >= num_blocks*B -> PKV_DEV_BAD_SLOT, that token skipped.  Two tokens with
+ *   the same slot in one call race (caller error, result unspecified).
+ */
+PKV_API pkv_status pkv_reshape_and_cache(const void *key, const void *value, int64_t key_token_stride,
+                                 int64_t value_token_stride, void *k_cache, void *v_cache,
+                                 pkv_cache_desc cache, const int64_t *slot_mapping,
+                                 int32_t num_tokens, int32_t *d_status, pkv_stream_t stream);
+
+/*
+ * pkv_paged_attention_workspace_size - bytes of scratch that
+ * pkv_paged_attention_decode needs for these sizes (0 when no sequence can
+ * span more than one partition).  partition_size follows the rules of
+ * pkv_paged_attention_decode (0 = automatic).  Returns 0 for invalid sizes.
+ */
+PKV_API size_t pkv_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t block_size, int32_t max_context_len,
+                                          int32_t partition_size);
+
+/*
+ * pkv_paged_attention_partition_size - the partition size (tokens) that
+ * pkv_paged_attention_decode uses for these arguments: partition_size itself
+ * when it is non-zero, otherwise the automatic choice.  Returns -1 for invalid
+ * arguments.  A result >= max_context_len means no sequence is split.
+ */
+PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num_kv_heads,
+                                           int32_t block_size, int32_t max_context_len,
+                                           int32_t partition_size);
+
+/*
+ * pkv_paged_attention_decode - single-token decode attention over the paged
+ * cache.
+ *
+ * Passage: lshu.cn/news/11644 "方案：页式内存管理" - the attention kernel reads
+ * each request's scattered blocks through its Block Table and treats them as
+ * one logically contiguous K/V sequence; "性能关键路径与瓶颈" - decode time is
+ * the KV bytes over memory bandwidth, and the kernel should keep table lookups
+ * cheap.  The attention itself is textbook softmax attention:
+ *   for sequence s, query head h, kv head g = h / (num_q_heads / num_kv_heads):
+ *     z_i = scale * <query[s][h], K_s[g][i]>  for i < context_lens[s],
+ *     out[s][h] = sum_i softmax(z)_i * V_s[g][i],
+ *   where K_s[g][i] = k_cache[block_tables[s][i / B]][g][i % B] (same for V).
+ * Long contexts are cut into partitions of partition_size tokens; each
+ * partition yields (max score, sum of exponentials, unnormalised output) and a
+ * second kernel merges them by log-sum-exp.  Arithmetic: fp16/bf16 products,
+ * fp32 accumulation and softmax; the output is rounded once to fp16/bf16.
+ *
+ * out              device, [num_seqs][num_q_heads][head_dim], cache dtype.
+ * query            device, [num_seqs][num_q_heads][head_dim], cache dtype.
+ * k_cache, v_cache device, 16-byte aligned, layout above.
+ * block_tables     device, int32 [num_seqs][max_blocks_per_seq]; entries at
+ *                  or past ceil(context_len / B) are never read.
+ * context_lens     device, int32 [num_seqs]: tokens attended by each sequence
+ *                  (including the one written this step); 0 gives a zero row.
+ * max_context_len  host bound >= every context_lens[s]; it sizes the grid.
+ * num_q_heads      multiple of num_kv_heads; num_q_heads / num_kv_heads <= 16.
+ * scale            softmax scale (e.g. 1/sqrt(head_dim)), > 0.
+ * partition_size   0 = automatic; otherwise a positive multiple of B.
+ * workspace        device, >= pkv_paged_attention_workspace_size(...) bytes,
+ *                  16-byte aligned; may be NULL when that size is 0.
+ * Errors: host checks -> status.  A table entry outside [0, num_blocks) ->
+ *   PKV_DEV_BAD_BLOCK and that block is treated as empty; a context length
+ *   outside [0, min(max_context_len, max_blocks_per_seq*B)] -> PKV_DEV_BAD_LEN
+ *   and the length is clamped into that range.
+ */
+PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *query, const void *k_cache,
+                                      const void *v_cache, pkv_cache_desc cache,
+                                      const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t *context_lens, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t max_context_len, float scale,
+                                      int32_t partition_size, void *workspace,
+                                      size_t workspace_bytes, int32_t *d_status,
+                                      pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks - copy-on-write of shared blocks.
+ *
+ * Passage: lshu.cn/news/11644 "内存共享" - requests with the same prompt prefix
+ * read the same physical blocks; a later divergence is handled by copying the
+ * block before writing to it.  For every pair i, block block_pairs[2i+1] of
+ * both pools becomes a bit copy of block block_pairs[2i] (every kv head, every
+ * position).
+ *
+ * block_pairs  device, int64 [num_pairs][2] = (src, dst).
+ * Errors: a src or dst outside [0, num_blocks) -> PKV_DEV_BAD_BLOCK and that
+ *   pair is skipped.  A dst that repeats, or that is also a src in the same
+ *   call, races (caller error, result unspecified).
+ */
+PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_desc cache,
+                           const int64_t *block_pairs, int32_t num_pairs, int32_t *d_status,
+                           pkv_stream_t stream);
+
+/* Static English text for a status code. */
+PKV_API const char *pkv_status_string(pkv_status status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+PKV_API int32_t pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,22 @@
+"""paged_kv_cache_407_b200: the decode hot path of a paged KV cache on B200.
+
+The compute lives in ``libpkv.so`` (C ABI, ``include/pkv.h``); this package is
+its thin binding plus host-side byte accounting.
+"""
+
+from .binding import (  # noqa: F401
+    DEV_BAD_BLOCK,
+    DEV_BAD_LEN,
+    DEV_BAD_SLOT,
+    DEV_TIMEOUT,
+    LIB_PATH,
+    PkvError,
+    cache_desc,
+    copy_blocks,
+    library,
+    paged_attention_decode,
+    partition_size,
+    reshape_and_cache,
+    version,
+    workspace_size,
+)

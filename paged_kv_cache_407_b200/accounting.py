@@ -1,0 +1,65 @@
+"""Algorithmic byte counts of the hot-path calls (host arithmetic only).
+
+These are the bytes a call must move at minimum, used for GB/s and roofline
+fractions: every byte counted once, K/V at their exact token counts (the tail
+of a partially filled block is not counted), no re-reads, no workspace.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+def decode_bytes(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                 block_size: int, elem_bytes: int = 2) -> dict:
+    """Bytes of one decode-attention call: K and V of every context token,
+    the queries, the outputs, the Block Table entries in use and the lengths."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    S = lens.size
+    kv = int(lens.sum()) * num_kv_heads * head_dim * elem_bytes * 2
+    q = S * num_q_heads * head_dim * elem_bytes
+    out = q
+    tables = int(((lens + block_size - 1) // block_size).sum()) * 4
+    return {"kv": kv, "q": q, "out": out, "tables": tables, "lens": 4 * S,
+            "total": kv + q + out + tables + 4 * S}
+
+
+def decode_bytes_padded_kv(context_lens, num_kv_heads: int, head_dim: int, block_size: int,
+                           elem_bytes: int = 2) -> int:
+    """K+V bytes when every used block is counted whole (what a block-granular
+    reader may fetch)."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    nb = (lens + block_size - 1) // block_size
+    return int(nb.sum()) * block_size * num_kv_heads * head_dim * elem_bytes * 2
+
+
+def reshape_and_cache_bytes(num_tokens: int, num_kv_heads: int, head_dim: int,
+                            elem_bytes: int = 2) -> int:
+    """Read the new K and V rows, write them into the pool, read the slots."""
+    rows = num_tokens * num_kv_heads * head_dim * elem_bytes * 2
+    return 2 * rows + 8 * num_tokens
+
+
+def copy_blocks_bytes(num_pairs: int, num_kv_heads: int, block_size: int, head_dim: int,
+                      elem_bytes: int = 2) -> int:
+    """Read and write one whole block of each pool per pair, plus the pairs."""
+    block = num_kv_heads * block_size * head_dim * elem_bytes
+    return num_pairs * (2 * 2 * block + 16)
+
+
+def kv_bytes_per_token(num_layers: int, hidden: int, elem_bytes: int = 2) -> int:
+    """KV-cache bytes one token occupies across a model: K and V of every layer."""
+    return 2 * num_layers * hidden * elem_bytes
+
+
+def static_reservation_waste(reserved_slots: int, used_slots: int) -> float:
+    """Fraction of a statically reserved KV region that stays unused."""
+    return 1.0 - used_slots / reserved_slots
+
+
+def block_fragmentation(context_lens, block_size: int) -> float:
+    """Fraction of allocated block slots that hold no token (internal
+    fragmentation of the last block of every sequence)."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    alloc = ((lens + block_size - 1) // block_size) * block_size
+    return float((alloc - lens).sum() / alloc.sum())

@@ -1,0 +1,196 @@
+"""Thin Python binding of libpkv (``include/pkv.h``) over torch tensors.
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels of ``libpkv.so``.  There is no fallback: if the library is missing or
+the device is not a B200 the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libpkv.so")
+
+# pkv_status
+OK = 0
+STATUS_NAMES = {
+    0: "PKV_OK", 1: "PKV_ERR_NULL_POINTER", 2: "PKV_ERR_BAD_DTYPE", 3: "PKV_ERR_BAD_SHAPE",
+    4: "PKV_ERR_MISALIGNED", 5: "PKV_ERR_WORKSPACE", 6: "PKV_ERR_BAD_PARTITION",
+    7: "PKV_ERR_TOO_LARGE", 8: "PKV_ERR_CUDA", 9: "PKV_ERR_DEVICE",
+}
+# device-side flags
+DEV_BAD_BLOCK = 0x1
+DEV_BAD_SLOT = 0x2
+DEV_BAD_LEN = 0x4
+DEV_TIMEOUT = 0x8
+
+PKV_F16 = 0
+PKV_BF16 = 1
+_DTYPES = {torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
+
+# Every function declared in include/pkv.h, with (restype, argtypes).
+_c_void_p, _i32, _i64, _f32, _size_t = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+class CacheDesc(ctypes.Structure):
+    """``pkv_cache_desc``."""
+
+    _fields_ = [
+        ("num_blocks", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+SIGNATURES = {
+    "pkv_reshape_and_cache": (ctypes.c_int, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p,
+                                             CacheDesc, _c_void_p, _i32, _c_void_p, _c_void_p]),
+    "pkv_paged_attention_workspace_size": (_size_t, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "pkv_paged_attention_partition_size": (_i32, [_i32, _i32, _i32, _i32, _i32]),
+    "pkv_paged_attention_decode": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc,
+                                                  _c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _f32,
+                                                  _i32, _c_void_p, _size_t, _c_void_p, _c_void_p]),
+    "pkv_copy_blocks": (ctypes.c_int, [_c_void_p, _c_void_p, CacheDesc, _c_void_p, _i32, _c_void_p,
+                                       _c_void_p]),
+    "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "pkv_version": (_i32, []),
+}
+
+_lib = None
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = STATUS_NAMES.get(status, str(status))
+        text = library().pkv_status_string(status).decode()
+        super().__init__(f"{where}: {name} ({text})")
+
+
+def library() -> ctypes.CDLL:
+    """Load libpkv.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_407_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise PkvError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def cache_desc(k_cache: torch.Tensor) -> CacheDesc:
+    """Descriptor of a ``[num_blocks, num_kv_heads, block_size, head_dim]`` pool."""
+    if k_cache.dim() != 4 or not k_cache.is_contiguous():
+        raise ValueError("cache must be a contiguous [num_blocks, num_kv_heads, block_size, head_dim] tensor")
+    if k_cache.dtype not in _DTYPES:
+        raise TypeError(f"cache dtype must be float16 or bfloat16, got {k_cache.dtype}")
+    N, Hkv, B, D = k_cache.shape
+    return CacheDesc(N, B, Hkv, D, _DTYPES[k_cache.dtype])
+
+
+def _same_pool(k_cache, v_cache):
+    if v_cache.shape != k_cache.shape or v_cache.dtype != k_cache.dtype or not v_cache.is_contiguous():
+        raise ValueError("k_cache and v_cache must have the same shape, dtype and layout")
+
+
+def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, d_status=None, stream=None):
+    """Write new tokens ``key/value [T, Hkv, D]`` into the slots ``slot_mapping [T]`` (int64)."""
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    T = key.shape[0]
+    for t in (key, value):
+        if t.dim() != 3 or t.shape[1:] != k_cache.shape[1:2] + k_cache.shape[3:4] or t.dtype != k_cache.dtype:
+            raise ValueError("key/value must be [T, num_kv_heads, head_dim] in the cache dtype")
+        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("key/value heads and dims must be contiguous within a token")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T or not slot_mapping.is_contiguous():
+        raise ValueError("slot_mapping must be a contiguous int64 tensor with one entry per token")
+    st = library().pkv_reshape_and_cache(
+        _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(k_cache), _ptr(v_cache), desc,
+        _ptr(slot_mapping), T, _ptr(d_status), _stream(stream, k_cache.device))
+    _check(st, "pkv_reshape_and_cache")
+
+
+def workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                   partition_size=0) -> int:
+    return int(library().pkv_paged_attention_workspace_size(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len, partition_size))
+
+
+def partition_size(num_seqs, num_kv_heads, block_size, max_context_len, partition_size=0) -> int:
+    return int(library().pkv_paged_attention_partition_size(
+        num_seqs, num_kv_heads, block_size, max_context_len, partition_size))
+
+
+def paged_attention_decode(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                           scale, partition_size=0, workspace=None, d_status=None, stream=None):
+    """Decode attention: ``out [S, Hq, D] = attention(query [S, Hq, D], paged K/V)``.
+
+    ``workspace``: a device tensor of at least ``workspace_size(...)`` bytes;
+    when None and one is needed it is allocated with torch (the library
+    itself never allocates).
+    """
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    S, Hq, D = query.shape
+    if out.shape != query.shape or out.dtype != k_cache.dtype or query.dtype != k_cache.dtype:
+        raise ValueError("query/out must be [S, Hq, head_dim] in the cache dtype")
+    if not (query.is_contiguous() and out.is_contiguous()):
+        raise ValueError("query/out must be contiguous")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S \
+            or not block_tables.is_contiguous():
+        raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
+    if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
+        raise ValueError("context_lens must be a contiguous int32 [S] tensor")
+    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = library().pkv_paged_attention_decode(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
+        int(partition_size), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device))
+    _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def copy_blocks(k_cache, v_cache, block_pairs, d_status=None, stream=None):
+    """Copy-on-write: block ``pairs[i, 1]`` of both pools becomes a copy of ``pairs[i, 0]``."""
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    if block_pairs.dtype != torch.int64 or block_pairs.dim() != 2 or block_pairs.shape[1] != 2 \
+            or not block_pairs.is_contiguous():
+        raise ValueError("block_pairs must be a contiguous int64 [num_pairs, 2] tensor")
+    st = library().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), desc, _ptr(block_pairs),
+                                   block_pairs.shape[0], _ptr(d_status), _stream(stream, k_cache.device))
+    _check(st, "pkv_copy_blocks")
+
+
+def version() -> int:
+    return int(library().pkv_version())

@@ -1,0 +1,83 @@
+// Host helpers: status strings, descriptor and device checks, tensor maps.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "pkv_host.h"
+
+namespace pkv {
+
+pkv_status check_cache_desc(const pkv_cache_desc &c) {
+  if (!valid_dtype(c.dtype)) return PKV_ERR_BAD_DTYPE;
+  if (c.num_blocks < 1 || c.num_kv_heads < 1) return PKV_ERR_BAD_SHAPE;
+  if (c.block_size != 8 && c.block_size != 16 && c.block_size != 32 && c.block_size != 64)
+    return PKV_ERR_BAD_SHAPE;
+  if (c.head_dim != 64 && c.head_dim != 128) return PKV_ERR_BAD_SHAPE;
+  // Slots are int64 but block coordinates and per-pool element offsets are
+  // formed in 64-bit; tensor-map dimensions must stay below 2^32.
+  const long long rows = static_cast<long long>(c.num_blocks) * c.num_kv_heads;
+  if (rows >= (1ll << 31)) return PKV_ERR_TOO_LARGE;
+  return PKV_OK;
+}
+
+pkv_status check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return PKV_ERR_CUDA;
+  return (major == 10 && minor == 0) ? PKV_OK : PKV_ERR_DEVICE;
+}
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+}  // namespace
+
+pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
+  auto fn = encoder();
+  if (fn == nullptr) return PKV_ERR_CUDA;
+  const cuuint64_t esz = 2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
+                        static_cast<cuuint64_t>(c.num_kv_heads),
+                        static_cast<cuuint64_t>(c.num_blocks)};
+  cuuint64_t strides[3] = {dims[0] * esz, dims[0] * dims[1] * esz, dims[0] * dims[1] * dims[2] * esz};
+  cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(c.block_size), 1u, 1u};
+  cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void *>(pool), dims, strides,
+                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace pkv
+
+extern "C" const char *pkv_status_string(pkv_status s) {
+  switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_NULL_POINTER: return "a required pointer is NULL";
+    case PKV_ERR_BAD_DTYPE: return "dtype must be PKV_F16 or PKV_BF16";
+    case PKV_ERR_BAD_SHAPE: return "unsupported shape (head_dim 64/128, block_size 8/16/32/64, head counts)";
+    case PKV_ERR_MISALIGNED: return "pointer or stride breaks the required alignment";
+    case PKV_ERR_WORKSPACE: return "workspace missing or smaller than pkv_paged_attention_workspace_size";
+    case PKV_ERR_BAD_PARTITION: return "partition_size must be a positive multiple of block_size";
+    case PKV_ERR_TOO_LARGE: return "a size exceeds what the kernels can index";
+    case PKV_ERR_CUDA: return "a CUDA runtime or driver call failed";
+    case PKV_ERR_DEVICE: return "current device is not compute capability 10.0 (B200, sm_100a)";
+  }
+  return "unknown pkv_status";
+}
+
+extern "C" int32_t pkv_version(void) { return 100; }

@@ -1,0 +1,33 @@
+// Host-side helpers shared by the libpkv entry points.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pkv.h"
+
+namespace pkv {
+
+inline bool aligned(const void *p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline bool valid_dtype(pkv_dtype t) { return t == PKV_F16 || t == PKV_BF16; }
+
+// Checks shared by every call that takes a cache descriptor.
+pkv_status check_cache_desc(const pkv_cache_desc &c);
+
+// PKV_ERR_DEVICE unless the current device is compute capability 10.0.
+pkv_status check_device();
+
+// Encode a rank-4 tiled tensor map over one cache pool viewed as
+// [N][Hkv][B][D] (fastest last), box = 64 elements x B rows, 128-byte swizzle.
+pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
+
+inline pkv_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace pkv

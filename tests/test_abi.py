@@ -1,0 +1,92 @@
+"""libpkv.so loads and exports the C ABI of include/pkv.h; host-side
+validation returns its status codes without touching a device (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_407_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_407_b200.build import build
+    build()
+    return bd.library()
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for n in ("pkv_reshape_and_cache", "pkv_paged_attention_decode", "pkv_copy_blocks",
+              "pkv_paged_attention_workspace_size", "pkv_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(bd.SIGNATURES), "binding and header disagree"
+
+
+def test_only_declared_symbols_are_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", bd.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if l.split()[-2:-1] == ["T"]}
+    ours = {s for s in exported if s.startswith("pkv_")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    for code in range(10):
+        assert lib.pkv_status_string(code)
+    assert lib.pkv_status_string(0) == b"ok"
+    assert bd.version() >= 100
+
+
+def _desc(N=16, B=16, H=4, D=64, dt=0):
+    return bd.CacheDesc(N, B, H, D, dt)
+
+
+def test_host_validation_without_device(lib):
+    null = None
+    # NULL key with tokens to write
+    assert lib.pkv_reshape_and_cache(null, null, 0, 0, null, null, _desc(), null, 1, null, null) == 1
+    # zero tokens: nothing to do, no device needed
+    assert lib.pkv_reshape_and_cache(null, null, 0, 0, null, null, _desc(), null, 0, null, null) == 0
+    # bad dtype / block size / head dim
+    assert lib.pkv_copy_blocks(null, null, _desc(dt=7), null, 1, null, null) == 2
+    assert lib.pkv_copy_blocks(null, null, _desc(B=12), null, 1, null, null) == 3
+    assert lib.pkv_copy_blocks(null, null, _desc(D=96), null, 1, null, null) == 3
+    dec = lib.pkv_paged_attention_decode
+    args = lambda **k: [k.get("out"), null, null, null, k.get("desc", _desc()), null, 4, null,
+                        k.get("S", 2), k.get("Hq", 4), 64, ctypes.c_float(k.get("scale", 0.125)),
+                        k.get("P", 0), null, 0, null, null]
+    assert dec(*args(P=24)) == 6            # not a multiple of block_size
+    assert dec(*args(Hq=6)) == 3            # Hq not a multiple of Hkv
+    assert dec(*args(Hq=4 * 17, desc=_desc(H=4))) == 3  # group larger than 16
+    assert dec(*args(scale=0.0)) == 3
+    assert dec(*args(S=0)) == 0             # nothing to do
+    assert dec(*args()) == 1                # NULL pointers
+
+
+def test_workspace_and_partition_queries(lib):
+    # 16-token blocks, automatic partition of 256 tokens
+    assert bd.partition_size(64, 32, 16, 2048) == 256
+    assert bd.partition_size(4, 8, 32, 131072, 512) == 512
+    assert bd.partition_size(4, 8, 32, 131072, 500) == -1
+    # no split needed -> no workspace
+    assert bd.workspace_size(4, 4, 4, 64, 16, 33) == 0
+    # 131072 tokens in 512-token partitions: 256 partials of (D + 2) floats per (seq, head)
+    assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 512) == 4 * 32 * 256 * 130 * 4
+    assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 24) == 0  # invalid partition

@@ -1,0 +1,43 @@
+"""Byte accounting against the closed forms the pages print (CPU)."""
+
+import numpy as np
+
+from paged_kv_cache_407_b200 import accounting as A
+
+
+def test_kv_bytes_per_token_7b():
+    """lshu.cn/news/11644, "问题：KV Cache 的内存困境": a 7B model produces about
+    0.5 MB of fp16 KV cache per token (32 layers, hidden size 4096)."""
+    assert A.kv_bytes_per_token(32, 4096, 2) == 512 * 1024
+
+
+def test_static_reservation_waste():
+    """Same section: 2048 reserved slots of which requests use 256 on average
+    leave about 87% of the KV cache idle."""
+    assert abs(A.static_reservation_waste(2048, 256) - 0.875) < 1e-12
+
+
+def test_decode_bytes_small():
+    lens = [1, 15, 16, 33]
+    b = A.decode_bytes(lens, num_q_heads=4, num_kv_heads=4, head_dim=64, block_size=16)
+    assert b["kv"] == 65 * 4 * 64 * 2 * 2
+    assert b["q"] == b["out"] == 4 * 4 * 64 * 2
+    assert b["tables"] == (1 + 1 + 1 + 3) * 4
+    assert b["total"] == b["kv"] + 2 * b["q"] + b["tables"] + 16
+    assert A.decode_bytes_padded_kv(lens, 4, 64, 16) == 6 * 16 * 4 * 64 * 4
+
+
+def test_fragmentation_under_one_block_per_sequence():
+    """Paging wastes at most the unused tail of each sequence's last block
+    (ypxx.net, "2.1 PagedAttention分页注意力核心机制": waste under 4%)."""
+    rng = np.random.default_rng(0)
+    lens = rng.integers(128, 2049, size=64)
+    f = A.block_fragmentation(lens, 16)
+    assert 0 < f < 0.04
+    assert A.block_fragmentation([16, 32], 16) == 0.0
+    assert abs(A.block_fragmentation([1], 16) - 15 / 16) < 1e-12
+
+
+def test_copy_and_write_bytes():
+    assert A.copy_blocks_bytes(128, 8, 16, 128) == 128 * (4 * 8 * 16 * 128 * 2 + 16)
+    assert A.reshape_and_cache_bytes(256, 8, 128) == 2 * 256 * 8 * 128 * 2 * 2 + 8 * 256
