@@ -4,7 +4,7 @@ binding and compare with the oracle.
 Tolerance for attention outputs (fp16/bf16 storage, fp32 accumulation), per
 element: |gpu - oracle| <= ATOL + RTOL * |oracle|, with ATOL = 2e-3 and
 RTOL = 1e-2.  Rounding the exact result to bf16 alone moves it by up to
-2^-9 |x| (3.9e-3 at |x| ~ 2), so a plain absolute bound of 2e-3 cannot hold
+2^-8 |x| (3.9e-3 at |x| = 1), so a plain absolute bound of 2e-3 cannot hold
 for every element of a bf16 output; the combined bound can.  Cache writes and
 block copies must match bit for bit.
 """

@@ -388,3 +388,46 @@ WORKLOADS = {
     "prefix_share": prefix_share,
     "long_context": long_context,
 }
+
+
+def shard_batch(batch: PagedBatch, rank: int, world: int) -> PagedBatch:
+    """The sequences of one data-parallel shard, with a pool of their own.
+
+    Sequences are split into ``world`` contiguous ranges; shard ``rank`` keeps
+    its range, only the blocks those sequences reference (renumbered in
+    order of first use), and their new tokens and copy pairs.  Pure data
+    movement: the shard's decode outputs are the global batch's rows.
+    """
+    S = batch.num_seqs
+    lo, hi = (S * rank) // world, (S * (rank + 1)) // world
+    tables = batch.block_tables[lo:hi]
+    before = None if batch.block_tables_before_cow is None else batch.block_tables_before_cow[lo:hi]
+    used = [b for b in tables.ravel().tolist() if b >= 0]
+    if before is not None:
+        used += [b for b in before.ravel().tolist() if b >= 0]
+    keep = list(dict.fromkeys(used))  # first-use order, unique
+    remap = {b: i for i, b in enumerate(keep)}
+
+    def rt(t):
+        return np.vectorize(lambda b: remap.get(int(b), -1), otypes=[np.int32])(t) if t.size else t
+
+    N = max(1, len(keep))
+    kc = batch.k_cache[keep] if keep else batch.k_cache[:1]
+    vc = batch.v_cache[keep] if keep else batch.v_cache[:1]
+    B = batch.block_size
+    slot_block = batch.slot_mapping // B
+    tok = np.array([b in remap for b in slot_block.tolist()], dtype=bool)
+    slots = np.array([remap[int(b)] * B + int(s) % B for b, s in zip(slot_block[tok], batch.slot_mapping[tok])],
+                     dtype=np.int64)
+    pairs = [(remap[int(a)], remap[int(b)]) for a, b in batch.cow_pairs.tolist()
+             if int(a) in remap and int(b) in remap]
+    return PagedBatch(
+        name=f"{batch.name}[{rank}/{world}]", dtype=batch.dtype, num_q_heads=batch.num_q_heads,
+        num_kv_heads=batch.num_kv_heads, head_dim=batch.head_dim, block_size=B, scale=batch.scale,
+        q=batch.q[lo:hi], k_cache=np.ascontiguousarray(kc), v_cache=np.ascontiguousarray(vc),
+        block_tables=rt(tables), context_lens=batch.context_lens[lo:hi],
+        key=batch.key[tok], value=batch.value[tok], slot_mapping=slots,
+        cow_pairs=np.asarray(pairs, dtype=np.int64).reshape(-1, 2),
+        block_tables_before_cow=None if before is None else rt(before),
+        partition_size=batch.partition_size, seed=batch.seed,
+    )
