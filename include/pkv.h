@@ -191,6 +191,37 @@ PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_desc 
                            const int64_t *block_pairs, int32_t num_pairs, int32_t *d_status,
                            pkv_stream_t stream);
 
+/*
+ * pkv_paged_attention_decode_noalloc - pkv_paged_attention_decode without a
+ * caller-supplied workspace.  No counterpart in the paper: it exists for callers
+ * that cannot allocate device memory, such as a serving engine that has already
+ * reserved all free device memory for its block pool, a C host without a device
+ * allocator of its own, or a loop that cannot afford cudaMalloc's implicit
+ * device-wide synchronisation.
+ *
+ * Arguments, layouts, results and device flags are those of
+ * pkv_paged_attention_decode minus (workspace, workspace_bytes).  The split-K
+ * scratch is a buffer of PKV_NOALLOC_SCRATCH_BYTES compiled into the library;
+ * every GPU that loads the library holds it until the process exits.  This call
+ * allocates nothing and frees nothing.
+ *   - Limit: when pkv_paged_attention_workspace_size(...) for these sizes
+ *     exceeds PKV_NOALLOC_SCRATCH_BYTES the call returns PKV_ERR_TOO_LARGE
+ *     before anything is queued; use pkv_paged_attention_decode instead.
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one buffer and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero (each partial is written
+ *     before it is read within a call), but two calls whose kernels overlap on
+ *     the GPU (for example on two streams) race on it.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+PKV_API pkv_status pkv_paged_attention_decode_noalloc(
+    void *out, const void *query, const void *k_cache, const void *v_cache, pkv_cache_desc cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
+    int32_t partition_size, int32_t *d_status, pkv_stream_t stream);
+
 /* Static English text for a status code. */
 PKV_API const char *pkv_status_string(pkv_status status);
 

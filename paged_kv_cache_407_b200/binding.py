@@ -56,6 +56,9 @@ SIGNATURES = {
     "pkv_paged_attention_decode": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc,
                                                   _c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _f32,
                                                   _i32, _c_void_p, _size_t, _c_void_p, _c_void_p]),
+    "pkv_paged_attention_decode_noalloc": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                                          CacheDesc, _c_void_p, _i32, _c_void_p, _i32,
+                                                          _i32, _i32, _f32, _i32, _c_void_p, _c_void_p]),
     "pkv_copy_blocks": (ctypes.c_int, [_c_void_p, _c_void_p, CacheDesc, _c_void_p, _i32, _c_void_p,
                                        _c_void_p]),
     "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -177,6 +180,46 @@ def paged_attention_decode(out, query, k_cache, v_cache, block_tables, context_l
         block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
         int(partition_size), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device))
     _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+# Capacity of the library's built-in split-K scratch (PKV_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def paged_attention_decode_noalloc(out, query, k_cache, v_cache, block_tables, context_lens,
+                                   max_context_len, scale, partition_size=0, d_status=None, stream=None):
+    """Decode attention that allocates nothing, neither here nor in the library.
+
+    For callers that cannot allocate device memory (their memory is all
+    reserved up front, or they cannot afford cudaMalloc's device-wide
+    synchronisation): the split-K scratch is the library's built-in buffer of
+    ``NOALLOC_SCRATCH_BYTES`` per device.  Sizes that need more raise
+    ``PkvError`` (PKV_ERR_TOO_LARGE); calls that overlap on the GPU race on
+    the shared buffer.  Same arguments and result as ``paged_attention_decode``
+    without ``workspace``.
+    """
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    S, Hq, D = query.shape
+    if out.shape != query.shape or out.dtype != k_cache.dtype or query.dtype != k_cache.dtype:
+        raise ValueError("query/out must be [S, Hq, head_dim] in the cache dtype")
+    if not (query.is_contiguous() and out.is_contiguous()):
+        raise ValueError("query/out must be contiguous")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S \
+            or not block_tables.is_contiguous():
+        raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
+    if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
+        raise ValueError("context_lens must be a contiguous int32 [S] tensor")
+    st = library().pkv_paged_attention_decode_noalloc(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
+        int(partition_size), _ptr(d_status), _stream(stream, query.device))
+    if st == 7:
+        need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
+        raise PkvError(st, f"pkv_paged_attention_decode_noalloc: these sizes need {need} bytes of split-K "
+                           f"scratch, more than the built-in {NOALLOC_SCRATCH_BYTES}")
+    _check(st, "pkv_paged_attention_decode_noalloc")
     return out
 
 

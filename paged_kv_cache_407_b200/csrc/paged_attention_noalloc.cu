@@ -1,0 +1,71 @@
+// pkv_paged_attention_decode_noalloc: decode attention for callers that must
+// not allocate device memory.
+//
+// The regular entry point asks the caller for a split-K workspace.  Some callers
+// cannot provide one: a serving engine that reserved all free device memory for
+// its block pool up front (so any later cudaMalloc fails), a plain C host with no
+// device allocator of its own, or a latency-critical loop where cudaMalloc's
+// implicit device-wide synchronisation is unacceptable.  For them the scratch
+// lives in a fixed buffer compiled into this library, PKV_NOALLOC_SCRATCH_BYTES
+// per device; the caller still passes every input and output.
+#include <mutex>
+
+#include "pkv_host.h"
+
+// The scratch itself.  Every GPU that loads this library holds it until the
+// process exits.  Host code must not pass `g_noalloc_scratch` to a kernel: in
+// host code that name is only a host-side stand-in; the device address comes
+// from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+namespace pkv {
+namespace {
+
+constexpr size_t kScratchBytes = PKV_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 128;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxDevices];  // device address of the buffer, per device ordinal
+
+// Device address of the buffer on the current device, looked up once per device
+// (with that device current) and cached.
+pkv_status scratch_address(void **addr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return PKV_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *addr = g_scratch_addr[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attention_decode_noalloc(
+    void *out, const void *query, const void *k_cache, const void *v_cache, pkv_cache_desc cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
+    int32_t partition_size, int32_t *d_status, pkv_stream_t stream) {
+  using namespace pkv;
+  // Sizes whose split-K partials do not fit the buffer are refused up front.
+  const size_t need = pkv_paged_attention_workspace_size(num_seqs, num_q_heads, cache.num_kv_heads,
+                                                         cache.head_dim, cache.block_size,
+                                                         max_context_len, partition_size);
+  if (need > kScratchBytes) return PKV_ERR_TOO_LARGE;
+  pkv_status st = check_device();
+  if (st != PKV_OK) return st;
+  void *scratch = nullptr;
+  if ((st = scratch_address(&scratch)) != PKV_OK) return st;
+  // Nothing in the buffer has to start at zero: every partial result that the
+  // merge kernel reads is written earlier in the same call.  Two calls whose
+  // kernels overlap on the GPU (e.g. on two streams) share the buffer and race.
+  return pkv_paged_attention_decode(out, query, k_cache, v_cache, cache, block_tables,
+                                    max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                                    max_context_len, scale, partition_size, scratch, kScratchBytes,
+                                    d_status, stream);
+}
