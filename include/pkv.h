@@ -142,8 +142,9 @@ PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num
  *     out[s][h] = sum_i softmax(z)_i * V_s[g][i],
  *   where K_s[g][i] = k_cache[block_tables[s][i / B]][g][i % B] (same for V).
  * Long contexts are cut into partitions of partition_size tokens; each
- * partition yields (max score, sum of exponentials, unnormalised output) and a
- * second kernel merges them by log-sum-exp.  Arithmetic: fp16/bf16 products,
+ * partition yields (max score, sum of exponentials, unnormalised output) and
+ * they are merged by log-sum-exp (by the last partition of each sequence to
+ * finish, or by a second kernel for splits of more than 32 partitions).  Arithmetic: fp16/bf16 products,
  * fp32 accumulation and softmax; the output is rounded once to fp16/bf16.
  *
  * out              device, [num_seqs][num_q_heads][head_dim], cache dtype.
@@ -158,7 +159,10 @@ PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num
  * scale            softmax scale (e.g. 1/sqrt(head_dim)), > 0.
  * partition_size   0 = automatic; otherwise a positive multiple of B.
  * workspace        device, >= pkv_paged_attention_workspace_size(...) bytes,
- *                  16-byte aligned; may be NULL when that size is 0.
+ *                  16-byte aligned; may be NULL when that size is 0.  Holds
+ *                  the partials and one arrival counter per (sequence, kv
+ *                  head); the call zeroes the counters itself (an async
+ *                  memset on `stream`), so no content is expected on entry.
  * Errors: host checks -> status.  A table entry outside [0, num_blocks) ->
  *   PKV_DEV_BAD_BLOCK and that block is treated as empty; a context length
  *   outside [0, min(max_context_len, max_blocks_per_seq*B)] -> PKV_DEV_BAD_LEN
@@ -211,9 +215,10 @@ PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_desc 
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.
  *   - All calls on a device share the one buffer and it keeps the last call's
- *     contents.  Nothing in it needs to start at zero (each partial is written
- *     before it is read within a call), but two calls whose kernels overlap on
- *     the GPU (for example on two streams) race on it.
+ *     contents.  The call clears the part that must start at zero (the split
+ *     arrival counters) and writes every partial before reading it, but two
+ *     calls whose kernels overlap on the GPU (for example on two streams) race
+ *     on it.
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 PKV_API pkv_status pkv_paged_attention_decode_noalloc(

@@ -29,8 +29,11 @@
 //     shuffles; the output is rescaled only when some row's max grows.
 //   * At the end the warps' (m, l, O) states are merged through shared
 //     memory; a single-partition sequence writes its output directly, other
-//     partitions write (m, l, unnormalised O) to the workspace and a second
-//     kernel merges them by log-sum-exp.
+//     partitions write (m, l, unnormalised O) to the workspace and count
+//     themselves in on a per-(sequence, kv head) counter; the last partition
+//     to arrive merges them all by log-sum-exp and resets the counter.  Only
+//     splits of more than kFuseMaxParts partitions use the separate merge
+//     kernel.
 #include <algorithm>
 
 #include "pkv_device.cuh"
@@ -50,9 +53,11 @@ struct DecodeArgs {
   float *ws_m;  // [S][Hq][max_parts]
   float *ws_l;  // [S][Hq][max_parts]
   float *ws_o;  // [S][Hq][max_parts][D]
+  int32_t *counters;  // [S][Hkv] arrivals of split partitions (zero between calls)
   int32_t *d_status;
   int max_blocks_per_seq;
   int num_q_heads;
+  int num_kv_heads;
   int group;       // query heads per kv head
   int num_blocks;  // pool size
   int len_limit;   // largest valid context length
@@ -61,13 +66,20 @@ struct DecodeArgs {
   float scale_log2;  // scale * log2(e)
 };
 
-// Launch shape per (head_dim, block_size): warps per CTA and ring depth.
+// Launch shape per (head_dim, block_size): warps per CTA and ring depth,
+// chosen so a CTA's rings take about 64 KB of shared memory and three CTAs fit
+// on an SM (measured best on B200 for 8..64-token blocks).
 template <int D, int BS>
 struct Tune {
   static constexpr int kStage = 2 * BS * D * 2;  // bytes of one K+V stage
-  static constexpr int kWarps = (BS == 64) ? 2 : 4;
-  static constexpr int kStages = kStage <= 4096 ? 4 : (kStage <= 8192 ? 3 : 2);
+  static constexpr int kWarps = kStage >= 16384 ? 2 : 4;
+  static constexpr int kFit = 65536 / (kWarps * kStage);
+  static constexpr int kStages = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
 };
+
+// Split sequences with at most this many partitions are merged inside the
+// attention kernel by the last CTA to finish; longer splits use the merge kernel.
+constexpr int kFuseMaxParts = 32;
 
 template <int D, int BS, int WARPS, int NST>
 struct Layout {
@@ -446,6 +458,40 @@ __global__ void __launch_bounds__(WARPS * 32)
       }
     }
   }
+  if (single || nparts > kFuseMaxParts) return;
+
+  // ---- split sequence: the last of its partitions to finish merges them ---
+  __shared__ int s_last;
+  __syncthreads();  // this CTA's partials are written
+  if (threadIdx.x == 0) {
+    __threadfence();  // publish them before counting this partition in
+    int *cnt = a.counters + static_cast<size_t>(s) * a.num_kv_heads + g;
+    const int last = atomicAdd(cnt, 1) == nparts - 1;
+    if (last) {
+      *cnt = 0;  // leave the counter at zero for the next call
+      __threadfence();
+    }
+    s_last = last;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  for (int e = threadIdx.x; e < G * D; e += WARPS * 32) {
+    const int h = e / D;
+    const int d = e - h * D;
+    const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
+    const size_t base = row * a.max_parts;
+    float M = -INFINITY;
+    for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(a.ws_m + base + p));
+    float acc = 0.f, lsum = 0.f;
+    if (M != -INFINITY) {
+      for (int p = 0; p < nparts; ++p) {
+        const float wt = fast_exp2(__ldcg(a.ws_m + base + p) - M);
+        acc += wt * __ldcg(a.ws_o + (base + p) * D + d);
+        lsum += wt * __ldcg(a.ws_l + base + p);
+      }
+    }
+    out[row * D + d] = PK::from_float(lsum > 0.f ? acc / lsum : 0.f);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -491,7 +537,7 @@ __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
   len = len < 0 ? 0 : (len > c.len_limit ? c.len_limit : len);
   const int nb = (len + c.block_size - 1) / c.block_size;
   const int nparts = nb > c.part_blocks ? (nb + c.part_blocks - 1) / c.part_blocks : 1;
-  if (nparts <= 1) return;  // written by the attention kernel
+  if (nparts <= kFuseMaxParts) return;  // written by the attention kernel
   const size_t row = static_cast<size_t>(s) * c.num_q_heads + h;
   const float *pm = c.ws_m + row * c.max_parts;
   const float *pl = c.ws_l + row * c.max_parts;
@@ -524,9 +570,8 @@ __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
 // Host side
 // ---------------------------------------------------------------------------
 int auto_part_blocks(int block_size) {
-  // Sixteen blocks per partition: 256 tokens at block_size 16, 512 at 32.
-  (void)block_size;
-  return 16;
+  // 512-token partitions (at least 8 blocks): 32 blocks of 16 tokens, 16 of 32.
+  return block_size >= 64 ? 8 : 512 / block_size;
 }
 
 bool valid_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
@@ -538,10 +583,10 @@ struct Plan {
 };
 
 // Resolve the partitioning; false for invalid arguments.
-bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t block_size,
-               int32_t max_context_len, int32_t partition_size, Plan *plan) {
-  if (!valid_block_size(block_size) || num_seqs < 0 || num_q_heads < 1 || head_dim < 1 ||
-      max_context_len < 0 || partition_size < 0)
+bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+               int32_t block_size, int32_t max_context_len, int32_t partition_size, Plan *plan) {
+  if (!valid_block_size(block_size) || num_seqs < 0 || num_q_heads < 1 || num_kv_heads < 1 ||
+      head_dim < 1 || max_context_len < 0 || partition_size < 0)
     return false;
   int part_blocks;
   if (partition_size == 0) {
@@ -554,8 +599,10 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t 
   const long long parts = nb_max > part_blocks ? (nb_max + part_blocks - 1) / part_blocks : 1;
   plan->part_blocks = part_blocks;
   plan->max_parts = static_cast<int>(std::min<long long>(parts, 1ll << 30));
+  // partials (o, m, l) then one arrival counter per (sequence, kv head)
   plan->ws_bytes = parts > 1 ? static_cast<size_t>(num_seqs) * num_q_heads * parts *
-                                   (static_cast<size_t>(head_dim) + 2) * sizeof(float)
+                                       (static_cast<size_t>(head_dim) + 2) * sizeof(float) +
+                                   static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t)
                              : 0;
   return true;
 }
@@ -609,8 +656,8 @@ extern "C" size_t pkv_paged_attention_workspace_size(int32_t num_seqs, int32_t n
                                                      int32_t block_size, int32_t max_context_len,
                                                      int32_t partition_size) {
   pkv::Plan plan;
-  if (num_kv_heads < 1 || !pkv::make_plan(num_seqs, num_q_heads, head_dim, block_size,
-                                          max_context_len, partition_size, &plan))
+  if (!pkv::make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                      partition_size, &plan))
     return 0;
   return plan.ws_bytes;
 }
@@ -619,8 +666,8 @@ extern "C" int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t 
                                                       int32_t block_size, int32_t max_context_len,
                                                       int32_t partition_size) {
   pkv::Plan plan;
-  if (num_kv_heads < 1 ||
-      !pkv::make_plan(num_seqs, num_kv_heads, 64, block_size, max_context_len, partition_size, &plan))
+  if (!pkv::make_plan(num_seqs, num_kv_heads, num_kv_heads, 64, block_size, max_context_len,
+                      partition_size, &plan))
     return -1;
   return plan.part_blocks * block_size;
 }
@@ -650,8 +697,8 @@ extern "C" pkv_status pkv_paged_attention_decode(
     return PKV_ERR_MISALIGNED;
 
   Plan plan;
-  if (!make_plan(num_seqs, num_q_heads, cache.head_dim, cache.block_size, max_context_len,
-                 partition_size, &plan))
+  if (!make_plan(num_seqs, num_q_heads, cache.num_kv_heads, cache.head_dim, cache.block_size,
+                 max_context_len, partition_size, &plan))
     return PKV_ERR_BAD_PARTITION;
   if (plan.max_parts > 65535) return PKV_ERR_TOO_LARGE;
   if (plan.ws_bytes > 0) {
@@ -674,9 +721,12 @@ extern "C" pkv_status pkv_paged_attention_decode(
   args.ws_o = plan.ws_bytes ? ws : nullptr;
   args.ws_m = plan.ws_bytes ? ws + rows * cache.head_dim : nullptr;
   args.ws_l = plan.ws_bytes ? ws + rows * (cache.head_dim + 1) : nullptr;
+  args.counters =
+      plan.ws_bytes ? reinterpret_cast<int32_t *>(ws + rows * (cache.head_dim + 2)) : nullptr;
   args.d_status = d_status;
   args.max_blocks_per_seq = max_blocks_per_seq;
   args.num_q_heads = num_q_heads;
+  args.num_kv_heads = cache.num_kv_heads;
   args.group = num_q_heads / cache.num_kv_heads;
   args.num_blocks = cache.num_blocks;
   args.len_limit = static_cast<int>(std::min<long long>(
@@ -686,6 +736,11 @@ extern "C" pkv_status pkv_paged_attention_decode(
   args.scale_log2 = scale * kLog2e;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (plan.max_parts > 1 &&
+      cudaMemsetAsync(args.counters, 0,
+                      static_cast<size_t>(num_seqs) * cache.num_kv_heads * sizeof(int32_t),
+                      s) != cudaSuccess)
+    return PKV_ERR_CUDA;
   const bool big = args.group > 8;
   const bool bf16 = cache.dtype == PKV_BF16;
   if (cache.head_dim == 128)
@@ -698,7 +753,7 @@ extern "C" pkv_status pkv_paged_attention_decode(
                                                  cache.num_kv_heads, num_seqs, s)
               : launch_for_dim<__half, 64>(cache.block_size, big, tmk, tmv, args,
                                            cache.num_kv_heads, num_seqs, s);
-  if (st != PKV_OK || plan.max_parts <= 1) return st;
+  if (st != PKV_OK || plan.max_parts <= kFuseMaxParts) return st;
 
   CombineArgs c{};
   c.out = out;

@@ -61,9 +61,10 @@ extern "C" pkv_status pkv_paged_attention_decode_noalloc(
   if (st != PKV_OK) return st;
   void *scratch = nullptr;
   if ((st = scratch_address(&scratch)) != PKV_OK) return st;
-  // Nothing in the buffer has to start at zero: every partial result that the
-  // merge kernel reads is written earlier in the same call.  Two calls whose
-  // kernels overlap on the GPU (e.g. on two streams) share the buffer and race.
+  // The regular entry point clears what must start at zero (its split arrival
+  // counters, with an async memset on the stream) and writes every partial
+  // before reading it.  Two calls whose kernels overlap on the GPU (e.g. on two
+  // streams) share the buffer and race.
   return pkv_paged_attention_decode(out, query, k_cache, v_cache, cache, block_tables,
                                     max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
                                     max_context_len, scale, partition_size, scratch, kScratchBytes,
