@@ -40,6 +40,7 @@ METRIC = "paged decode attention KV GB/s and tokens/s on 1 B200; % of HBM roofli
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/paged_attention.cu",
+                  "paged_kv_cache_407_b200/csrc/decode_core.cuh",
                   "paged_kv_cache_407_b200/csrc/pkv_device.cuh"]
 
 

@@ -109,9 +109,12 @@ PKV_API pkv_status pkv_reshape_and_cache(const void *key, const void *value, int
 
 /*
  * pkv_paged_attention_workspace_size - bytes of scratch that
- * pkv_paged_attention_decode needs for these sizes (0 when no sequence can
- * span more than one partition).  partition_size follows the rules of
- * pkv_paged_attention_decode (0 = automatic).  Returns 0 for invalid sizes.
+ * pkv_paged_attention_decode needs for these sizes: 0 when no sequence can
+ * span more than one partition; otherwise num_seqs * num_kv_heads int32
+ * arrival counters (padded to 16 bytes) followed by num_seqs * num_q_heads *
+ * max_partitions * (head_dim + 2) floats of partials.  partition_size follows
+ * the rules of pkv_paged_attention_decode (0 = automatic).  Returns 0 for
+ * invalid sizes.
  */
 PKV_API size_t pkv_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                           int32_t num_kv_heads, int32_t head_dim,
@@ -121,7 +124,9 @@ PKV_API size_t pkv_paged_attention_workspace_size(int32_t num_seqs, int32_t num_
 /*
  * pkv_paged_attention_partition_size - the partition size (tokens) that
  * pkv_paged_attention_decode uses for these arguments: partition_size itself
- * when it is non-zero, otherwise the automatic choice.  Returns -1 for invalid
+ * when it is non-zero, otherwise the automatic choice (1024 tokens, halved
+ * down to 256 while num_seqs * num_kv_heads * ceil(max_context_len / size)
+ * stays below 1776, i.e. about 12 work units per SM).  Returns -1 for invalid
  * arguments.  A result >= max_context_len means no sequence is split.
  */
 PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num_kv_heads,
@@ -160,8 +165,8 @@ PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num
  * partition_size   0 = automatic; otherwise a positive multiple of B.
  * workspace        device, >= pkv_paged_attention_workspace_size(...) bytes,
  *                  16-byte aligned; may be NULL when that size is 0.  Holds
- *                  the partials and one arrival counter per (sequence, kv
- *                  head); the call zeroes the counters itself (an async
+ *                  one arrival counter per (sequence, kv head) and the split
+ *                  partials; the call zeroes the counters itself (an async
  *                  memset on `stream`), so no content is expected on entry.
  * Errors: host checks -> status.  A table entry outside [0, num_blocks) ->
  *   PKV_DEV_BAD_BLOCK and that block is treated as empty; a context length

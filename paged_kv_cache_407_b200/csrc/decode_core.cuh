@@ -1,0 +1,266 @@
+// Per-warp decode-attention state and the math of one K/V block, shared by the
+// attention kernels.
+//
+// A warp holds the softmax state of the query heads of one group (rows of an
+// m16n8k16 tile, query head h of the group on row h) over the blocks it has
+// seen: running max m and sum l per row (log2 domain), and the unnormalised
+// output O[16 x D] as mma accumulator fragments.  One call of `block` folds
+// one K/V block (B tokens) into that state:
+//   S^T = Q K^T on mma.sync with the query heads on M, scale and mask,
+//   online softmax update, O = O * 2^(m_old - m_new) + P V.
+// The score accumulator fragment is, element for element, the A fragment of
+// P V, so P never moves between lanes.  P enters the second MMA as a 16-bit
+// high part plus a 16-bit residual, which keeps it at about fp32 precision.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr uint32_t kFullMask = 0xffffffffu;
+
+// Byte offset of 16-byte chunk `chunk` (= d / 8) of token row `tok` inside a
+// tile of D/64 boxes, each BS rows x 128 B, written by TMA with the 128-byte
+// swizzle (chunk index XOR row index within each 8-row, 1024-byte group).
+template <int BS>
+__device__ __forceinline__ uint32_t tile_off(int tok, int chunk) {
+  return static_cast<uint32_t>((chunk >> 3) * (BS * 128) + tok * 128 +
+                               (((chunk & 7) ^ (tok & 7)) << 4));
+}
+
+template <typename T, int D, int BS, bool BIG>
+struct DecodeState {
+  static constexpr int kNT = BS / 8;  // 8-token column tiles per block
+  static constexpr int kDT = D / 8;   // 8-wide column tiles of the output
+  static constexpr int kKS = D / 16;  // 16-deep steps of the score product
+  using MMA = Mma<T>;
+  using PK = Pack<T>;
+
+  uint32_t qa0[kKS], qa1[kKS], qa2[kKS], qa3[kKS];  // Q as A fragments (rows r, r + 8)
+  float m0, m1, l0, l1;                             // running max / sum, rows r and r + 8
+  float o[kDT][4];                                  // O accumulators
+
+  // Query rows of the group: q points at G consecutive rows of D elements.
+  __device__ __forceinline__ void load_q(const T *q, int G, int lane) {
+    const int r = lane >> 2;
+    const int c2 = (lane & 3) * 2;
+    const uint32_t *q32 = reinterpret_cast<const uint32_t *>(q);
+#pragma unroll
+    for (int kk = 0; kk < kKS; ++kk) {
+      qa0[kk] = r < G ? q32[(r * D + 16 * kk + c2) >> 1] : 0u;
+      qa2[kk] = r < G ? q32[(r * D + 16 * kk + 8 + c2) >> 1] : 0u;
+      if constexpr (BIG) {
+        qa1[kk] = r + 8 < G ? q32[((r + 8) * D + 16 * kk + c2) >> 1] : 0u;
+        qa3[kk] = r + 8 < G ? q32[((r + 8) * D + 16 * kk + 8 + c2) >> 1] : 0u;
+      } else {
+        qa1[kk] = 0u;
+        qa3[kk] = 0u;
+      }
+    }
+  }
+
+  __device__ __forceinline__ void reset() {
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+#pragma unroll
+    for (int dt = 0; dt < kDT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+  }
+
+  // Fold one block into the state.  kb / vb: shared-memory addresses of the
+  // block's K and V tiles; nv: tokens of the block inside the context (the
+  // rest are masked, whatever the tile holds).
+  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int nv, float scale_log2,
+                                        int lane) {
+    const int mi = lane >> 3;  // ldmatrix: which 8x8 matrix this lane addresses
+    const int ri = lane & 7;   // ldmatrix: which row of it
+    const int c2 = (lane & 3) * 2;
+
+    // ---- S^T[16 x BS] = Q[16 x D] . K^T ----------------------------------
+    float sc[kNT][4];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+    if constexpr (BS >= 16) {
+#pragma unroll
+      for (int kk = 0; kk < kKS; ++kk) {
+#pragma unroll
+        for (int tp = 0; tp < BS / 16; ++tp) {
+          uint32_t b0r, b1r, b2r, b3r;
+          ldsm_x4(kb + tile_off<BS>(tp * 16 + ri + ((mi >> 1) << 3), 2 * kk + (mi & 1)), b0r, b1r,
+                  b2r, b3r);
+          MMA::k16(sc[2 * tp], qa0[kk], qa1[kk], qa2[kk], qa3[kk], b0r, b1r);
+          MMA::k16(sc[2 * tp + 1], qa0[kk], qa1[kk], qa2[kk], qa3[kk], b2r, b3r);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < kKS; kk += 2) {
+        uint32_t b0r, b1r, b2r, b3r;
+        ldsm_x4(kb + tile_off<BS>(ri, 2 * kk + mi), b0r, b1r, b2r, b3r);
+        MMA::k16(sc[0], qa0[kk], qa1[kk], qa2[kk], qa3[kk], b0r, b1r);
+        MMA::k16(sc[0], qa0[kk + 1], qa1[kk + 1], qa2[kk + 1], qa3[kk + 1], b2r, b3r);
+      }
+    }
+
+    // ---- scale, mask past the context, online softmax --------------------
+    const bool partial = nv < BS;
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float v = sc[nt][j] * scale_log2;
+        if (partial && nt * 8 + c2 + (j & 1) >= nv) v = -INFINITY;
+        sc[nt][j] = v;
+      }
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
+      if constexpr (BIG) mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, 2));
+    const float mn0 = fmaxf(m0, mx0);
+    const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+    const float al0 = fast_exp2(m0 - base0);
+    m0 = mn0;
+    float al1 = 1.f, base1 = 0.f;
+    if constexpr (BIG) {
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, 2));
+      const float mn1 = fmaxf(m1, mx1);
+      base1 = mn1 == -INFINITY ? 0.f : mn1;
+      al1 = fast_exp2(m1 - base1);
+      m1 = mn1;
+    }
+    float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      sc[nt][0] = fast_exp2(sc[nt][0] - base0);
+      sc[nt][1] = fast_exp2(sc[nt][1] - base0);
+      rs0 += sc[nt][0] + sc[nt][1];
+      if constexpr (BIG) {
+        sc[nt][2] = fast_exp2(sc[nt][2] - base1);
+        sc[nt][3] = fast_exp2(sc[nt][3] - base1);
+        rs1 += sc[nt][2] + sc[nt][3];
+      }
+    }
+    l0 = l0 * al0 + rs0;
+    if constexpr (BIG) l1 = l1 * al1 + rs1;
+    const bool moved = BIG ? (al0 != 1.f || al1 != 1.f) : (al0 != 1.f);
+    if (__any_sync(kFullMask, moved)) {
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) {
+        o[dt][0] *= al0;
+        o[dt][1] *= al0;
+        if constexpr (BIG) {
+          o[dt][2] *= al1;
+          o[dt][3] *= al1;
+        }
+      }
+    }
+
+    // ---- O[16 x D] += P[16 x BS] . V --------------------------------------
+    if constexpr (BS >= 16) {
+#pragma unroll
+      for (int tp = 0; tp < BS / 16; ++tp) {
+        const uint32_t h0 = PK::pack(sc[2 * tp][0], sc[2 * tp][1]);
+        const uint32_t h2 = PK::pack(sc[2 * tp + 1][0], sc[2 * tp + 1][1]);
+        const float2 f0 = PK::unpack(h0);
+        const float2 f2 = PK::unpack(h2);
+        const uint32_t e0 = PK::pack(sc[2 * tp][0] - f0.x, sc[2 * tp][1] - f0.y);
+        const uint32_t e2 = PK::pack(sc[2 * tp + 1][0] - f2.x, sc[2 * tp + 1][1] - f2.y);
+        uint32_t h1 = 0u, h3 = 0u, e1 = 0u, e3 = 0u;
+        if constexpr (BIG) {
+          h1 = PK::pack(sc[2 * tp][2], sc[2 * tp][3]);
+          h3 = PK::pack(sc[2 * tp + 1][2], sc[2 * tp + 1][3]);
+          const float2 f1 = PK::unpack(h1);
+          const float2 f3 = PK::unpack(h3);
+          e1 = PK::pack(sc[2 * tp][2] - f1.x, sc[2 * tp][3] - f1.y);
+          e3 = PK::pack(sc[2 * tp + 1][2] - f3.x, sc[2 * tp + 1][3] - f3.y);
+        }
+        const bool vmask = partial && (tp * 16 + 16 > nv);
+        const int t0 = tp * 16 + c2;
+        const uint32_t mlo = (t0 < nv ? 0x0000ffffu : 0u) | (t0 + 1 < nv ? 0xffff0000u : 0u);
+        const uint32_t mhi = (t0 + 8 < nv ? 0x0000ffffu : 0u) | (t0 + 9 < nv ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int dp = 0; dp < kDT / 2; ++dp) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_trans(vb + tile_off<BS>(tp * 16 + ri + ((mi & 1) << 3), 2 * dp + (mi >> 1)), v0,
+                        v1, v2, v3);
+          if (vmask) {
+            v0 &= mlo;
+            v2 &= mlo;
+            v1 &= mhi;
+            v3 &= mhi;
+          }
+          MMA::k16(o[2 * dp], h0, h1, h2, h3, v0, v1);
+          MMA::k16(o[2 * dp], e0, e1, e2, e3, v0, v1);
+          MMA::k16(o[2 * dp + 1], h0, h1, h2, h3, v2, v3);
+          MMA::k16(o[2 * dp + 1], e0, e1, e2, e3, v2, v3);
+        }
+      }
+    } else {
+      const uint32_t h0 = PK::pack(sc[0][0], sc[0][1]);
+      const float2 f0 = PK::unpack(h0);
+      const uint32_t e0 = PK::pack(sc[0][0] - f0.x, sc[0][1] - f0.y);
+      uint32_t h1 = 0u, e1 = 0u;
+      if constexpr (BIG) {
+        h1 = PK::pack(sc[0][2], sc[0][3]);
+        const float2 f1 = PK::unpack(h1);
+        e1 = PK::pack(sc[0][2] - f1.x, sc[0][3] - f1.y);
+      }
+      const uint32_t mlo = (c2 < nv ? 0x0000ffffu : 0u) | (c2 + 1 < nv ? 0xffff0000u : 0u);
+#pragma unroll
+      for (int dq = 0; dq < kDT / 4; ++dq) {
+        uint32_t v[4];
+        ldsm_x4_trans(vb + tile_off<BS>(ri, 4 * dq + mi), v[0], v[1], v[2], v[3]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (partial) v[j] &= mlo;
+          MMA::k8(o[4 * dq + j], h0, h1, v[j]);
+          MMA::k8(o[4 * dq + j], e0, e1, v[j]);
+        }
+      }
+    }
+  }
+
+  // Sum l over the four lanes that share a row.
+  __device__ __forceinline__ void reduce_l() {
+    l0 += __shfl_xor_sync(kFullMask, l0, 1);
+    l0 += __shfl_xor_sync(kFullMask, l0, 2);
+    if constexpr (BIG) {
+      l1 += __shfl_xor_sync(kFullMask, l1, 1);
+      l1 += __shfl_xor_sync(kFullMask, l1, 2);
+    }
+  }
+
+  // Write rows < G of the state to shared memory: O as [row][D] floats at
+  // `mo`, m and l per row at `mm`, `ml` (call after reduce_l).
+  __device__ __forceinline__ void store_rows(float *mo, float *mm, float *ml, int G, int lane) const {
+    const int r = lane >> 2;
+    const int c2 = (lane & 3) * 2;
+    if (r < G) {
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt)
+        *reinterpret_cast<float2 *>(&mo[r * D + dt * 8 + c2]) = make_float2(o[dt][0], o[dt][1]);
+      if ((lane & 3) == 0) {
+        mm[r] = m0;
+        ml[r] = l0;
+      }
+    }
+    if constexpr (BIG) {
+      if (r + 8 < G) {
+#pragma unroll
+        for (int dt = 0; dt < kDT; ++dt)
+          *reinterpret_cast<float2 *>(&mo[(r + 8) * D + dt * 8 + c2]) =
+              make_float2(o[dt][2], o[dt][3]);
+        if ((lane & 3) == 0) {
+          mm[r + 8] = m1;
+          ml[r + 8] = l1;
+        }
+      }
+    }
+  }
+};
+
+}  // namespace pkv

@@ -9,115 +9,227 @@
 // 瓶颈" in the same page: decode is bound by the bytes of KV cache read, and
 // Block Table lookups are an overhead to keep small.
 //
-// How (B200 design):
-//   * One CTA per (kv head g, sequence s, partition p).  All query heads of
-//     the group g share each K/V block, so every block is read from HBM once.
-//   * Every warp streams its own share of the partition's blocks (blocks
-//     w, w + WARPS, ...) through a private ring of NST shared-memory stages.
-//     One stage = one block's K tile and V tile, each loaded by tiled TMA
-//     (rank-4 tensor map over [N][Hkv][B][D], box 64 x B, 128-byte swizzle)
-//     and counted on an mbarrier.  Block Table entries are fetched 32 at a
-//     time per warp with one coalesced load, prefetched a window ahead.
-//   * Scores S^T = Q K^T and the update O += P V run on mma.sync.m16n8k16
-//     (fp16/bf16 in, fp32 accumulate) with the group's query heads on M, so
-//     the score accumulator fragment is already the A operand of P V.  P is
-//     split into a 16-bit high part and a 16-bit residual (two MMAs), which
-//     keeps the probabilities at about fp32 precision.  Tensor cores are used
-//     to keep instruction issue far below the HBM rate, not for throughput.
-//   * Online softmax in the log2 domain (scores pre-multiplied by
-//     scale*log2 e), max/sum reduced over the 4 lanes that share a row with
-//     shuffles; the output is rescaled only when some row's max grows.
-//   * At the end the warps' (m, l, O) states are merged through shared
-//     memory; a single-partition sequence writes its output directly, other
-//     partitions write (m, l, unnormalised O) to the workspace and count
-//     themselves in on a per-(sequence, kv head) counter; the last partition
-//     to arrive merges them all by log-sum-exp and resets the counter.  Only
-//     splits of more than kFuseMaxParts partitions use the separate merge
-//     kernel.
+// Work unit: one partition (up to part_blocks consecutive blocks) of one
+// (sequence s, kv head g).  All query heads of group g share each K/V block,
+// so every block is read from HBM once.  A sequence with several partitions
+// leaves one (m, l, unnormalised O) partial per partition in the workspace;
+// the partitions count themselves in on a per-(s, g) counter and the last to
+// arrive merges them by log-sum-exp (splits of more than kFuseMaxParts
+// partitions are merged by lse_combine_kernel instead).
+//
+// One CTA per (g, s, partition) slot, three CTAs per SM (about 64 KB of
+// shared memory each); slots past a sequence's last partition exit at once.
+// Every warp of the CTA streams its share of the unit's blocks (w, w + WARPS,
+// ...) through a private ring of shared-memory stages: each stage is one
+// block's K and V tiles, loaded by tiled TMA (rank-4 tensor map over
+// [N][Hkv][B][D], box 64 x B, 128-byte swizzle, L2 evict-first) and counted
+// on an mbarrier; Block Table entries are read 32 at a time per warp, a
+// window ahead.  The per-block math is decode_core.cuh.  At the end of the
+// unit the warps merge through shared memory, one warp per query head row.
 #include <algorithm>
 
-#include "pkv_device.cuh"
+#include "decode_core.cuh"
 #include "pkv_host.h"
 
 namespace pkv {
 namespace {
 
-constexpr uint32_t kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Split sequences with at most this many partitions are merged inside the
+// attention kernel by the last partition to finish; longer splits use the
+// merge kernel.
+constexpr int kFuseMaxParts = 32;
 
 struct DecodeArgs {
   const void *query;
   void *out;
   const int32_t *block_tables;
   const int32_t *context_lens;
-  float *ws_m;  // [S][Hq][max_parts]
-  float *ws_l;  // [S][Hq][max_parts]
-  float *ws_o;  // [S][Hq][max_parts][D]
-  int32_t *counters;  // [S][Hkv] arrivals of split partitions (zero between calls)
+  float *ws_m;        // [S][Hq][max_parts]
+  float *ws_l;        // [S][Hq][max_parts]
+  float *ws_o;        // [S][Hq][max_parts][D]
+  int32_t *counters;  // [S][Hkv] arrivals of split partitions (zeroed per call)
   int32_t *d_status;
+  int num_seqs;
   int max_blocks_per_seq;
   int num_q_heads;
   int num_kv_heads;
-  int group;       // query heads per kv head
-  int num_blocks;  // pool size
-  int len_limit;   // largest valid context length
-  int part_blocks; // blocks per partition
+  int group;        // query heads per kv head
+  int num_blocks;   // pool size
+  int len_limit;    // largest valid context length
+  int part_blocks;  // blocks per partition
   int max_parts;
   float scale_log2;  // scale * log2(e)
 };
 
-// Launch shape per (head_dim, block_size): warps per CTA and ring depth,
-// chosen so a CTA's rings take about 64 KB of shared memory and three CTAs fit
-// on an SM (measured best on B200 for 8..64-token blocks).
+// ---------------------------------------------------------------------------
+// Result of one work unit, shared by both kernels.
+// ---------------------------------------------------------------------------
+
+// Store the result of one unit from `nw` deposited warp states (o at
+// mo + w*G*D as [row][D] floats, m/l at mm/ml + w*G), one warp, rows
+// h = h0, h0 + hstep, ... of the group.  Lane j owns dims j*VPL .. j*VPL+VPL-1.
+// One partition: write the normalised output.  Otherwise write the partial.
+template <typename T, int D>
+__device__ __forceinline__ void store_unit_warp(const DecodeArgs &a, const float *mo,
+                                                const float *mm, const float *ml, int nw, int s,
+                                                int g, int part, int nparts, int h0, int hstep,
+                                                int lane) {
+  constexpr int VPL = D / 32;
+  const int G = a.group;
+  for (int h = h0; h < G; h += hstep) {
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmaxf(M, mm[w * G + h]);
+    float acc[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) acc[j] = 0.f;
+    float lsum = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < nw; ++w) {
+        const float wt = fast_exp2(mm[w * G + h] - M);
+        lsum += wt * ml[w * G + h];
+        const float *src = mo + (w * G + h) * D + lane * VPL;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) acc[j] += wt * src[j];
+      }
+    }
+    const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
+    if (nparts == 1) {
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
+#pragma unroll
+      for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
+    } else {
+      const size_t idx = row * a.max_parts + part;
+      float *dst = a.ws_o + idx * D + lane * VPL;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) dst[j] = acc[j];
+      if (lane == 0) {
+        a.ws_m[idx] = M;
+        a.ws_l[idx] = lsum;
+      }
+    }
+  }
+}
+
+// Count one partition of (s, g) in; true for the last of its nparts
+// partitions, which also resets the counter.  Call from a single thread after
+// the partition's partials are written by its thread group.
+__device__ __forceinline__ bool arrive_partition(const DecodeArgs &a, int s, int g, int nparts) {
+  __threadfence();  // publish this partition's partials before counting it in
+  int *cnt = a.counters + static_cast<size_t>(s) * a.num_kv_heads + g;
+  const bool last = atomicAdd(cnt, 1) == nparts - 1;
+  if (last) {
+    *cnt = 0;  // leave the counter at zero for the next call
+    __threadfence();
+  }
+  return last;
+}
+
+// Merge the nparts (<= 32) partials of (s, g) from the workspace into the
+// output, one warp, rows h = h0, h0 + hstep, ...: lane p reads partition p's
+// (m, l); the maximum and the weighted sum are warp reductions; the partial
+// outputs are read eight partitions at a time so their loads overlap.
+template <typename T, int D>
+__device__ __forceinline__ void merge_partials_warp(const DecodeArgs &a, int s, int g, int nparts,
+                                                    int h0, int hstep, int lane) {
+  constexpr int VPL = D / 32;
+  const int G = a.group;
+  for (int h = h0; h < G; h += hstep) {
+    const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
+    const size_t base = row * a.max_parts;
+    const float mp = lane < nparts ? __ldcg(a.ws_m + base + lane) : -INFINITY;
+    const float lp = lane < nparts ? __ldcg(a.ws_l + base + lane) : 0.f;
+    float M = mp;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, off));
+    const float w = (lane < nparts && M != -INFINITY) ? fast_exp2(mp - M) : 0.f;
+    float L = w * lp;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(kFullMask, L, off);
+    float acc[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) acc[j] = 0.f;
+    const float *o = a.ws_o + base * D + lane * VPL;
+    for (int p0 = 0; p0 < nparts; p0 += 8) {
+      float v[8][VPL];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+          v[u][j] = p0 + u < nparts ? __ldcg(o + static_cast<size_t>(p0 + u) * D + j) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float wu = __shfl_sync(kFullMask, w, (p0 + u) & 31);
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) acc[j] += wu * v[u][j];
+      }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
+#pragma unroll
+    for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
+  }
+}
+
+__device__ __forceinline__ int clamp_len(const DecodeArgs &a, int s, bool report) {
+  int len = a.context_lens[s];
+  if (len < 0 || len > a.len_limit) {
+    if (report) raise_flag(a.d_status, PKV_DEV_BAD_LEN);
+    len = len < 0 ? 0 : a.len_limit;
+  }
+  return len;
+}
+
+__device__ __forceinline__ int parts_of(int nb, int part_blocks) {
+  return nb > part_blocks ? (nb + part_blocks - 1) / part_blocks : 1;
+}
+
+// Issue the TMA loads of one block (K and V tiles) into a stage.
 template <int D, int BS>
-struct Tune {
-  static constexpr int kStage = 2 * BS * D * 2;  // bytes of one K+V stage
+__device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap *tmk,
+                                           const CUtensorMap *tmv, uint32_t bar, int g, int id,
+                                           uint64_t policy) {
+  constexpr int kBoxBytes = BS * 128;
+  constexpr int kTileBytes = (D / 64) * kBoxBytes;
+  mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+#pragma unroll
+  for (int bx = 0; bx < D / 64; ++bx) {
+    tma_load_4d(dst + bx * kBoxBytes, tmk, bar, bx * 64, 0, g, id, policy);
+    tma_load_4d(dst + kTileBytes + bx * kBoxBytes, tmv, bar, bx * 64, 0, g, id, policy);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Grid kernel: one CTA per (kv head, sequence, partition)
+// ---------------------------------------------------------------------------
+
+// Launch shape: a CTA's rings take about 64 KB so three CTAs fit on an SM.
+template <int D, int BS>
+struct GridTune {
+  static constexpr int kStage = 2 * BS * D * 2;
   static constexpr int kWarps = kStage >= 16384 ? 2 : 4;
   static constexpr int kFit = 65536 / (kWarps * kStage);
   static constexpr int kStages = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
+  static constexpr int kRing = kWarps * kStages * kStage;
+  static constexpr int kMerge = kWarps * 16 * (D + 2) * 4;
+  static constexpr int kData = kRing > kMerge ? kRing : kMerge;
+  static constexpr int kBarOff = (kData + 1023) / 1024 * 1024;
+  static constexpr int kNvOff = kBarOff + kWarps * kStages * 8;
+  static constexpr int kSmem = kNvOff + kWarps * kStages * 4 + 1024;
 };
-
-// Split sequences with at most this many partitions are merged inside the
-// attention kernel by the last CTA to finish; longer splits use the merge kernel.
-constexpr int kFuseMaxParts = 32;
-
-template <int D, int BS, int WARPS, int NST>
-struct Layout {
-  static constexpr int kBoxes = D / 64;                     // TMA boxes per tile
-  static constexpr int kBoxBytes = BS * 128;                // BS rows of 128 B
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;     // one K (or V) tile
-  static constexpr int kStageBytes = 2 * kTileBytes;        // K + V
-  static constexpr int kRingBytes = WARPS * NST * kStageBytes;
-  static constexpr int kMergeBytes = WARPS * 16 * (D + 2) * 4;
-  static constexpr int kDataBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-  static constexpr int kBarOff = (kDataBytes + 1023) / 1024 * 1024;
-  static constexpr int kNvOff = kBarOff + WARPS * NST * 8;
-  static constexpr int kSmem = kNvOff + WARPS * NST * 4 + 1024;  // + base alignment slack
-  static constexpr int kNT = BS / 8;  // 8-token column tiles per block
-  static constexpr int kDT = D / 8;   // 8-wide column tiles of the output
-  static constexpr int kKS = D / 16;  // 16-deep steps of the score product
-};
-
-// Byte offset of 16-byte chunk `chunk` (= d / 8) of token row `tok` inside a
-// tile of D/64 boxes, each BS rows x 128 B, written by TMA with the 128-byte
-// swizzle (chunk index XOR row index within each 8-row, 1024-byte group).
-template <int BS>
-__device__ __forceinline__ uint32_t tile_off(int tok, int chunk) {
-  return static_cast<uint32_t>((chunk >> 3) * (BS * 128) + tok * 128 +
-                               (((chunk & 7) ^ (tok & 7)) << 4));
-}
 
 template <typename T, int D, int BS, int WARPS, int NST, bool BIG>
 __global__ void __launch_bounds__(WARPS * 32)
-    paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
-  using Lt = Layout<D, BS, WARPS, NST>;
-  using MMA = Mma<T>;
-  using PK = Pack<T>;
+    paged_decode_grid_kernel(const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
+  using TN = GridTune<D, BS>;
+  constexpr int kStageBytes = 2 * BS * D * 2;
+  using State = DecodeState<T, D, BS, BIG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-
   const int g = blockIdx.x;
   const int s = blockIdx.y;
   const int part = blockIdx.z;
@@ -125,24 +237,18 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int lane = threadIdx.x & 31;
   const int G = a.group;
 
-  // ---- sequence bounds -------------------------------------------------
-  int len = a.context_lens[s];
-  if (len < 0 || len > a.len_limit) {
-    if (threadIdx.x == 0 && g == 0 && part == 0) raise_flag(a.d_status, PKV_DEV_BAD_LEN);
-    len = len < 0 ? 0 : a.len_limit;
-  }
+  const int len = clamp_len(a, s, g == 0 && part == 0 && threadIdx.x == 0);
   const int nb = (len + BS - 1) / BS;
-  const int nparts = nb > a.part_blocks ? (nb + a.part_blocks - 1) / a.part_blocks : 1;
+  const int nparts = parts_of(nb, a.part_blocks);
   if (part >= nparts) return;  // uniform over the CTA, before any barrier
   const int b0 = part * a.part_blocks;
   const int nblk = min(nb - b0, a.part_blocks);
-  const int tail_nv = len - (nb - 1) * BS;  // valid tokens of the sequence's last block
+  const int tail_nv = len - (nb - 1) * BS;
   const int cnt = nblk > warp ? (nblk - warp + WARPS - 1) / WARPS : 0;
 
-  // ---- per-warp ring and barriers --------------------------------------
-  const uint32_t ring = smem_addr(smem) + warp * NST * Lt::kStageBytes;
-  const uint32_t bars = smem_addr(smem + Lt::kBarOff) + warp * NST * 8;
-  volatile int *stage_nv = reinterpret_cast<volatile int *>(smem + Lt::kNvOff) + warp * NST;
+  const uint32_t ring = smem_addr(smem) + warp * NST * kStageBytes;
+  const uint32_t bars = smem_addr(smem + TN::kBarOff) + warp * NST * 8;
+  volatile int *stage_nv = reinterpret_cast<volatile int *>(smem + TN::kNvOff) + warp * NST;
   if (lane == 0) {
 #pragma unroll
     for (int st = 0; st < NST; ++st) mbar_init(bars + 8 * st, 1);
@@ -152,27 +258,13 @@ __global__ void __launch_bounds__(WARPS * 32)
   }
   __syncwarp();
 
-  // ---- query fragments (A operand: rows = query heads of the group) ----
-  const int r = lane >> 2;        // fragment row of this lane
-  const int c2 = (lane & 3) * 2;  // fragment column pair of this lane
-  const uint32_t *q32 = reinterpret_cast<const uint32_t *>(
-      static_cast<const T *>(a.query) +
-      (static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G) * D);
-  uint32_t qa0[Lt::kKS], qa1[Lt::kKS], qa2[Lt::kKS], qa3[Lt::kKS];
-#pragma unroll
-  for (int kk = 0; kk < Lt::kKS; ++kk) {
-    qa0[kk] = r < G ? q32[(r * D + 16 * kk + c2) >> 1] : 0u;
-    qa2[kk] = r < G ? q32[(r * D + 16 * kk + 8 + c2) >> 1] : 0u;
-    if constexpr (BIG) {
-      qa1[kk] = r + 8 < G ? q32[((r + 8) * D + 16 * kk + c2) >> 1] : 0u;
-      qa3[kk] = r + 8 < G ? q32[((r + 8) * D + 16 * kk + 8 + c2) >> 1] : 0u;
-    } else {
-      qa1[kk] = 0u;
-      qa3[kk] = 0u;
-    }
-  }
+  State st_;
+  st_.load_q(static_cast<const T *>(a.query) +
+                 (static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G) * D,
+             G, lane);
+  st_.reset();
 
-  // ---- Block Table window: lane j holds the id of block 32*w + j ---------
+  // Block Table window: lane j holds the id of this warp's block 32*w + j.
   const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + b0 + warp;
   auto load_window = [&](int w) -> int {
     const int k = (w << 5) + lane;
@@ -187,7 +279,7 @@ __global__ void __launch_bounds__(WARPS * 32)
       win_cur = win_next;
       win_next = load_window((k >> 5) + 1);
     }
-    const int id = __shfl_sync(kFull, win_cur, k & 31);
+    const int id = __shfl_sync(kFullMask, win_cur, k & 31);
     if (lane == 0) {
       const int st = k % NST;
       const uint32_t bar = bars + 8 * st;
@@ -195,14 +287,7 @@ __global__ void __launch_bounds__(WARPS * 32)
       if (static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks)) {
         stage_nv[st] = (blk == nb - 1) ? tail_nv : BS;
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(bar, Lt::kStageBytes);
-        const uint32_t dst = ring + st * Lt::kStageBytes;
-#pragma unroll
-        for (int bx = 0; bx < Lt::kBoxes; ++bx) {
-          tma_load_4d(dst + bx * Lt::kBoxBytes, &tm_k, bar, bx * 64, 0, g, id, policy);
-          tma_load_4d(dst + Lt::kTileBytes + bx * Lt::kBoxBytes, &tm_v, bar, bx * 64, 0, g, id,
-                      policy);
-        }
+        load_block<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar, g, id, policy);
       } else {
         raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
         stage_nv[st] = 0;  // the whole block is masked
@@ -212,176 +297,15 @@ __global__ void __launch_bounds__(WARPS * 32)
   };
 
   int kp = 0;
-  {
-    const int pro = cnt < NST ? cnt : NST;
-    for (; kp < pro; ++kp) issue(kp);
-  }
-
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float o[Lt::kDT][4];
-#pragma unroll
-  for (int dt = 0; dt < Lt::kDT; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-
-  const int mi = lane >> 3;  // ldmatrix: which 8x8 matrix this lane addresses
-  const int ri = lane & 7;   // ldmatrix: which row of it
+  for (const int pro = cnt < NST ? cnt : NST; kp < pro; ++kp) issue(kp);
   int k = 0;
   bool ok = true;
   for (; k < cnt; ++k) {
     const int st = k % NST;
-    ok = __all_sync(kFull, mbar_wait(bars + 8 * st, (k / NST) & 1));
+    ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (k / NST) & 1));
     if (!ok) break;
-    const int nv = stage_nv[st];
-    const uint32_t kb = ring + st * Lt::kStageBytes;
-    const uint32_t vb = kb + Lt::kTileBytes;
-
-    // ---- S^T[16 x BS] = Q[16 x D] . K^T --------------------------------
-    float sc[Lt::kNT][4];
-#pragma unroll
-    for (int nt = 0; nt < Lt::kNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-    if constexpr (BS >= 16) {
-#pragma unroll
-      for (int kk = 0; kk < Lt::kKS; ++kk) {
-#pragma unroll
-        for (int tp = 0; tp < BS / 16; ++tp) {
-          uint32_t b0r, b1r, b2r, b3r;
-          ldsm_x4(kb + tile_off<BS>(tp * 16 + ri + ((mi >> 1) << 3), 2 * kk + (mi & 1)), b0r, b1r,
-                  b2r, b3r);
-          MMA::k16(sc[2 * tp], qa0[kk], qa1[kk], qa2[kk], qa3[kk], b0r, b1r);
-          MMA::k16(sc[2 * tp + 1], qa0[kk], qa1[kk], qa2[kk], qa3[kk], b2r, b3r);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int kk = 0; kk < Lt::kKS; kk += 2) {
-        uint32_t b0r, b1r, b2r, b3r;
-        ldsm_x4(kb + tile_off<BS>(ri, 2 * kk + mi), b0r, b1r, b2r, b3r);
-        MMA::k16(sc[0], qa0[kk], qa1[kk], qa2[kk], qa3[kk], b0r, b1r);
-        MMA::k16(sc[0], qa0[kk + 1], qa1[kk + 1], qa2[kk + 1], qa3[kk + 1], b2r, b3r);
-      }
-    }
-
-    // ---- scale, mask past the context, online softmax ------------------
-    const bool partial = nv < BS;
-#pragma unroll
-    for (int nt = 0; nt < Lt::kNT; ++nt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float v = sc[nt][j] * a.scale_log2;
-        if (partial && nt * 8 + c2 + (j & 1) >= nv) v = -INFINITY;
-        sc[nt][j] = v;
-      }
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < Lt::kNT; ++nt) {
-      mx0 = fmaxf(mx0, fmaxf(sc[nt][0], sc[nt][1]));
-      if constexpr (BIG) mx1 = fmaxf(mx1, fmaxf(sc[nt][2], sc[nt][3]));
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
-    const float mn0 = fmaxf(m0, mx0);
-    const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-    const float al0 = fast_exp2(m0 - base0);
-    m0 = mn0;
-    float al1 = 1.f, base1 = 0.f;
-    if constexpr (BIG) {
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
-      const float mn1 = fmaxf(m1, mx1);
-      base1 = mn1 == -INFINITY ? 0.f : mn1;
-      al1 = fast_exp2(m1 - base1);
-      m1 = mn1;
-    }
-    float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < Lt::kNT; ++nt) {
-      sc[nt][0] = fast_exp2(sc[nt][0] - base0);
-      sc[nt][1] = fast_exp2(sc[nt][1] - base0);
-      rs0 += sc[nt][0] + sc[nt][1];
-      if constexpr (BIG) {
-        sc[nt][2] = fast_exp2(sc[nt][2] - base1);
-        sc[nt][3] = fast_exp2(sc[nt][3] - base1);
-        rs1 += sc[nt][2] + sc[nt][3];
-      }
-    }
-    l0 = l0 * al0 + rs0;
-    if constexpr (BIG) l1 = l1 * al1 + rs1;
-    const bool moved = BIG ? (al0 != 1.f || al1 != 1.f) : (al0 != 1.f);
-    if (__any_sync(kFull, moved)) {
-#pragma unroll
-      for (int dt = 0; dt < Lt::kDT; ++dt) {
-        o[dt][0] *= al0;
-        o[dt][1] *= al0;
-        if constexpr (BIG) {
-          o[dt][2] *= al1;
-          o[dt][3] *= al1;
-        }
-      }
-    }
-
-    // ---- O[16 x D] += P[16 x BS] . V ------------------------------------
-    if constexpr (BS >= 16) {
-#pragma unroll
-      for (int tp = 0; tp < BS / 16; ++tp) {
-        const uint32_t h0 = PK::pack(sc[2 * tp][0], sc[2 * tp][1]);
-        const uint32_t h2 = PK::pack(sc[2 * tp + 1][0], sc[2 * tp + 1][1]);
-        const float2 f0 = PK::unpack(h0);
-        const float2 f2 = PK::unpack(h2);
-        const uint32_t e0 = PK::pack(sc[2 * tp][0] - f0.x, sc[2 * tp][1] - f0.y);
-        const uint32_t e2 = PK::pack(sc[2 * tp + 1][0] - f2.x, sc[2 * tp + 1][1] - f2.y);
-        uint32_t h1 = 0u, h3 = 0u, e1 = 0u, e3 = 0u;
-        if constexpr (BIG) {
-          h1 = PK::pack(sc[2 * tp][2], sc[2 * tp][3]);
-          h3 = PK::pack(sc[2 * tp + 1][2], sc[2 * tp + 1][3]);
-          const float2 f1 = PK::unpack(h1);
-          const float2 f3 = PK::unpack(h3);
-          e1 = PK::pack(sc[2 * tp][2] - f1.x, sc[2 * tp][3] - f1.y);
-          e3 = PK::pack(sc[2 * tp + 1][2] - f3.x, sc[2 * tp + 1][3] - f3.y);
-        }
-        const bool vmask = partial && (tp * 16 + 16 > nv);
-        const int t0 = tp * 16 + c2;
-        const uint32_t mlo = (t0 < nv ? 0x0000ffffu : 0u) | (t0 + 1 < nv ? 0xffff0000u : 0u);
-        const uint32_t mhi = (t0 + 8 < nv ? 0x0000ffffu : 0u) | (t0 + 9 < nv ? 0xffff0000u : 0u);
-#pragma unroll
-        for (int dp = 0; dp < Lt::kDT / 2; ++dp) {
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_trans(vb + tile_off<BS>(tp * 16 + ri + ((mi & 1) << 3), 2 * dp + (mi >> 1)), v0,
-                        v1, v2, v3);
-          if (vmask) {
-            v0 &= mlo;
-            v2 &= mlo;
-            v1 &= mhi;
-            v3 &= mhi;
-          }
-          MMA::k16(o[2 * dp], h0, h1, h2, h3, v0, v1);
-          MMA::k16(o[2 * dp], e0, e1, e2, e3, v0, v1);
-          MMA::k16(o[2 * dp + 1], h0, h1, h2, h3, v2, v3);
-          MMA::k16(o[2 * dp + 1], e0, e1, e2, e3, v2, v3);
-        }
-      }
-    } else {
-      const uint32_t h0 = PK::pack(sc[0][0], sc[0][1]);
-      const float2 f0 = PK::unpack(h0);
-      const uint32_t e0 = PK::pack(sc[0][0] - f0.x, sc[0][1] - f0.y);
-      uint32_t h1 = 0u, e1 = 0u;
-      if constexpr (BIG) {
-        h1 = PK::pack(sc[0][2], sc[0][3]);
-        const float2 f1 = PK::unpack(h1);
-        e1 = PK::pack(sc[0][2] - f1.x, sc[0][3] - f1.y);
-      }
-      const uint32_t mlo = (c2 < nv ? 0x0000ffffu : 0u) | (c2 + 1 < nv ? 0xffff0000u : 0u);
-#pragma unroll
-      for (int dq = 0; dq < Lt::kDT / 4; ++dq) {
-        uint32_t v[4];
-        ldsm_x4_trans(vb + tile_off<BS>(ri, 4 * dq + mi), v[0], v[1], v[2], v[3]);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (partial) v[j] &= mlo;
-          MMA::k8(o[4 * dq + j], h0, h1, v[j]);
-          MMA::k8(o[4 * dq + j], e0, e1, v[j]);
-        }
-      }
-    }
-
+    const uint32_t kb = ring + st * kStageBytes;
+    st_.block(kb, kb + kStageBytes / 2, stage_nv[st], a.scale_log2, lane);
     __syncwarp();
     if (kp < cnt) {
       issue(kp);
@@ -394,108 +318,25 @@ __global__ void __launch_bounds__(WARPS * 32)
     for (int j = k; j < kp; ++j) (void)mbar_wait(bars + 8 * (j % NST), (j / NST) & 1);
   }
 
-  // ---- merge the warps' softmax states ---------------------------------
-  l0 += __shfl_xor_sync(kFull, l0, 1);
-  l0 += __shfl_xor_sync(kFull, l0, 2);
-  if constexpr (BIG) {
-    l1 += __shfl_xor_sync(kFull, l1, 1);
-    l1 += __shfl_xor_sync(kFull, l1, 2);
-  }
+  st_.reduce_l();
   __syncthreads();  // every ring is drained; reuse it for the merge
-  float *mo = reinterpret_cast<float *>(smem);  // [WARPS][16][D]
-  float *mm = mo + WARPS * 16 * D;              // [WARPS][16]
-  float *ml = mm + WARPS * 16;                  // [WARPS][16]
-  if (r < G) {
-#pragma unroll
-    for (int dt = 0; dt < Lt::kDT; ++dt)
-      *reinterpret_cast<float2 *>(&mo[(warp * 16 + r) * D + dt * 8 + c2]) =
-          make_float2(o[dt][0], o[dt][1]);
-    if ((lane & 3) == 0) {
-      mm[warp * 16 + r] = m0;
-      ml[warp * 16 + r] = l0;
-    }
-  }
-  if constexpr (BIG) {
-    if (r + 8 < G) {
-#pragma unroll
-      for (int dt = 0; dt < Lt::kDT; ++dt)
-        *reinterpret_cast<float2 *>(&mo[(warp * 16 + r + 8) * D + dt * 8 + c2]) =
-            make_float2(o[dt][2], o[dt][3]);
-      if ((lane & 3) == 0) {
-        mm[warp * 16 + r + 8] = m1;
-        ml[warp * 16 + r + 8] = l1;
-      }
-    }
-  }
+  float *mo = reinterpret_cast<float *>(smem);  // [WARPS][G][D]
+  float *mm = mo + WARPS * 16 * D;              // [WARPS][G]
+  float *ml = mm + WARPS * 16;                  // [WARPS][G]
+  st_.store_rows(mo + warp * G * D, mm + warp * G, ml + warp * G, G, lane);
   __syncthreads();
+  store_unit_warp<T, D>(a, mo, mm, ml, WARPS, s, g, part, nparts, warp, WARPS, lane);
+  if (nparts == 1 || nparts > kFuseMaxParts) return;
 
-  const bool single = nparts == 1;
-  T *out = static_cast<T *>(a.out);
-  for (int e = threadIdx.x; e < G * D; e += WARPS * 32) {
-    const int h = e / D;
-    const int d = e - h * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, mm[w * 16 + h]);
-    float acc = 0.f, lsum = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < WARPS; ++w) {
-        const float wt = fast_exp2(mm[w * 16 + h] - M);
-        acc += wt * mo[(w * 16 + h) * D + d];
-        lsum += wt * ml[w * 16 + h];
-      }
-    }
-    const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
-    if (single) {
-      out[row * D + d] = PK::from_float(lsum > 0.f ? acc / lsum : 0.f);
-    } else {
-      const size_t idx = row * a.max_parts + part;
-      a.ws_o[idx * D + d] = acc;
-      if (d == 0) {
-        a.ws_m[idx] = M;
-        a.ws_l[idx] = lsum;
-      }
-    }
-  }
-  if (single || nparts > kFuseMaxParts) return;
-
-  // ---- split sequence: the last of its partitions to finish merges them ---
   __shared__ int s_last;
   __syncthreads();  // this CTA's partials are written
-  if (threadIdx.x == 0) {
-    __threadfence();  // publish them before counting this partition in
-    int *cnt = a.counters + static_cast<size_t>(s) * a.num_kv_heads + g;
-    const int last = atomicAdd(cnt, 1) == nparts - 1;
-    if (last) {
-      *cnt = 0;  // leave the counter at zero for the next call
-      __threadfence();
-    }
-    s_last = last;
-  }
+  if (threadIdx.x == 0) s_last = arrive_partition(a, s, g, nparts);
   __syncthreads();
-  if (!s_last) return;
-  for (int e = threadIdx.x; e < G * D; e += WARPS * 32) {
-    const int h = e / D;
-    const int d = e - h * D;
-    const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
-    const size_t base = row * a.max_parts;
-    float M = -INFINITY;
-    for (int p = 0; p < nparts; ++p) M = fmaxf(M, __ldcg(a.ws_m + base + p));
-    float acc = 0.f, lsum = 0.f;
-    if (M != -INFINITY) {
-      for (int p = 0; p < nparts; ++p) {
-        const float wt = fast_exp2(__ldcg(a.ws_m + base + p) - M);
-        acc += wt * __ldcg(a.ws_o + (base + p) * D + d);
-        lsum += wt * __ldcg(a.ws_l + base + p);
-      }
-    }
-    out[row * D + d] = PK::from_float(lsum > 0.f ? acc / lsum : 0.f);
-  }
+  if (s_last) merge_partials_warp<T, D>(a, s, g, nparts, warp, WARPS, lane);
 }
 
 // ---------------------------------------------------------------------------
-// Log-sum-exp merge of the partitions of each (sequence, query head):
+// Log-sum-exp merge of long splits (more than kFuseMaxParts partitions):
 //   M = max_p m_p,  w_p = 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p l_p.
 // ---------------------------------------------------------------------------
 struct CombineArgs {
@@ -515,7 +356,7 @@ template <int NT>
 __device__ __forceinline__ float block_reduce(float v, bool is_max, float *scratch) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    const float x = __shfl_xor_sync(kFull, v, off);
+    const float x = __shfl_xor_sync(kFullMask, v, off);
     v = is_max ? fmaxf(v, x) : v + x;
   }
   const int warp = threadIdx.x >> 5;
@@ -536,7 +377,7 @@ __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
   int len = c.context_lens[s];
   len = len < 0 ? 0 : (len > c.len_limit ? c.len_limit : len);
   const int nb = (len + c.block_size - 1) / c.block_size;
-  const int nparts = nb > c.part_blocks ? (nb + c.part_blocks - 1) / c.part_blocks : 1;
+  const int nparts = parts_of(nb, c.part_blocks);
   if (nparts <= kFuseMaxParts) return;  // written by the attention kernel
   const size_t row = static_cast<size_t>(s) * c.num_q_heads + h;
   const float *pm = c.ws_m + row * c.max_parts;
@@ -569,9 +410,18 @@ __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-int auto_part_blocks(int block_size) {
-  // 512-token partitions (at least 8 blocks): 32 blocks of 16 tokens, 16 of 32.
-  return block_size >= 64 ? 8 : 512 / block_size;
+// Automatic partition size: 1024 tokens, halved (down to 256) while the grid
+// would hold fewer than about 12 units per SM of a 148-SM B200, judged from
+// the largest possible batch (every sequence at max_context_len).
+int auto_part_blocks(int block_size, int num_seqs, int num_kv_heads, int max_context_len) {
+  int tokens = 1024;
+  const long long want = 148ll * 12;
+  while (tokens > 256) {
+    const long long parts = (max_context_len + tokens - 1) / tokens;
+    if (static_cast<long long>(num_seqs) * num_kv_heads * std::max(1ll, parts) >= want) break;
+    tokens /= 2;
+  }
+  return std::max(1, tokens / block_size);
 }
 
 bool valid_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 64; }
@@ -579,10 +429,14 @@ bool valid_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 
 struct Plan {
   int part_blocks;
   int max_parts;
+  size_t ctrl_bytes;  // arrival counters, zeroed per call
   size_t ws_bytes;
 };
 
-// Resolve the partitioning; false for invalid arguments.
+// Resolve the partitioning and the workspace; false for invalid arguments.
+// Workspace (only when a sequence can span several partitions):
+//   [arrival counters S*Hkv int32, padded to 16 B]
+//   [o partials S*Hq*max_parts*D][m ...][l ...] (fp32).
 bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                int32_t block_size, int32_t max_context_len, int32_t partition_size, Plan *plan) {
   if (!valid_block_size(block_size) || num_seqs < 0 || num_q_heads < 1 || num_kv_heads < 1 ||
@@ -590,7 +444,7 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int3
     return false;
   int part_blocks;
   if (partition_size == 0) {
-    part_blocks = auto_part_blocks(block_size);
+    part_blocks = auto_part_blocks(block_size, num_seqs, num_kv_heads, max_context_len);
   } else {
     if (partition_size % block_size != 0) return false;
     part_blocks = partition_size / block_size;
@@ -599,38 +453,42 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int3
   const long long parts = nb_max > part_blocks ? (nb_max + part_blocks - 1) / part_blocks : 1;
   plan->part_blocks = part_blocks;
   plan->max_parts = static_cast<int>(std::min<long long>(parts, 1ll << 30));
-  // partials (o, m, l) then one arrival counter per (sequence, kv head)
-  plan->ws_bytes = parts > 1 ? static_cast<size_t>(num_seqs) * num_q_heads * parts *
-                                       (static_cast<size_t>(head_dim) + 2) * sizeof(float) +
-                                   static_cast<size_t>(num_seqs) * num_kv_heads * sizeof(int32_t)
-                             : 0;
+  const bool split = parts > 1 && num_seqs > 0;
+  plan->ctrl_bytes = split ? (static_cast<size_t>(num_seqs) * num_kv_heads * 4 + 15) / 16 * 16 : 0;
+  plan->ws_bytes = plan->ctrl_bytes +
+                   (split ? static_cast<size_t>(num_seqs) * num_q_heads * parts *
+                                (static_cast<size_t>(head_dim) + 2) * sizeof(float)
+                          : 0);
   return true;
 }
 
 template <typename T, int D, int BS, bool BIG>
-pkv_status launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
-                         int num_kv_heads, int num_seqs, cudaStream_t stream) {
-  constexpr int WARPS = Tune<D, BS>::kWarps;
-  constexpr int NST = Tune<D, BS>::kStages;
-  using Lt = Layout<D, BS, WARPS, NST>;
-  auto kern = paged_decode_kernel<T, D, BS, WARPS, NST, BIG>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lt::kSmem) !=
+pkv_status launch_grid(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
+                       cudaStream_t stream) {
+  using TN = GridTune<D, BS>;
+  auto kern = paged_decode_grid_kernel<T, D, BS, TN::kWarps, TN::kStages, BIG>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TN::kSmem) !=
       cudaSuccess)
     return PKV_ERR_CUDA;
-  dim3 grid(static_cast<unsigned>(num_kv_heads), static_cast<unsigned>(num_seqs),
+  dim3 grid(static_cast<unsigned>(args.num_kv_heads), static_cast<unsigned>(args.num_seqs),
             static_cast<unsigned>(args.max_parts));
-  kern<<<grid, WARPS * 32, Lt::kSmem, stream>>>(tmk, tmv, args);
+  kern<<<grid, TN::kWarps * 32, TN::kSmem, stream>>>(tmk, tmv, args);
   return launch_status();
+}
+
+template <typename T, int D, int BS, bool BIG>
+pkv_status launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
+                         cudaStream_t stream) {
+  return launch_grid<T, D, BS, BIG>(tmk, tmv, args, stream);
 }
 
 template <typename T, int D>
 pkv_status launch_for_dim(int block_size, bool big, const CUtensorMap &tmk, const CUtensorMap &tmv,
-                          const DecodeArgs &args, int num_kv_heads, int num_seqs,
-                          cudaStream_t stream) {
-#define PKV_BS_CASE(BSV)                                                                       \
-  case BSV:                                                                                    \
-    return big ? launch_decode<T, D, BSV, true>(tmk, tmv, args, num_kv_heads, num_seqs, stream) \
-               : launch_decode<T, D, BSV, false>(tmk, tmv, args, num_kv_heads, num_seqs, stream);
+                          const DecodeArgs &args, cudaStream_t stream) {
+#define PKV_BS_CASE(BSV)                                                      \
+  case BSV:                                                                   \
+    return big ? launch_decode<T, D, BSV, true>(tmk, tmv, args, stream)       \
+               : launch_decode<T, D, BSV, false>(tmk, tmv, args, stream);
   switch (block_size) {
     PKV_BS_CASE(8)
     PKV_BS_CASE(16)
@@ -716,14 +574,16 @@ extern "C" pkv_status pkv_paged_attention_decode(
   args.out = out;
   args.block_tables = block_tables;
   args.context_lens = context_lens;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  args.counters = reinterpret_cast<int32_t *>(ws);
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * plan.max_parts;
-  float *ws = static_cast<float *>(workspace);
-  args.ws_o = plan.ws_bytes ? ws : nullptr;
-  args.ws_m = plan.ws_bytes ? ws + rows * cache.head_dim : nullptr;
-  args.ws_l = plan.ws_bytes ? ws + rows * (cache.head_dim + 1) : nullptr;
-  args.counters =
-      plan.ws_bytes ? reinterpret_cast<int32_t *>(ws + rows * (cache.head_dim + 2)) : nullptr;
+  float *part = reinterpret_cast<float *>(ws + plan.ctrl_bytes);
+  const bool split = plan.max_parts > 1;
+  args.ws_o = split ? part : nullptr;
+  args.ws_m = split ? part + rows * cache.head_dim : nullptr;
+  args.ws_l = split ? part + rows * (cache.head_dim + 1) : nullptr;
   args.d_status = d_status;
+  args.num_seqs = num_seqs;
   args.max_blocks_per_seq = max_blocks_per_seq;
   args.num_q_heads = num_q_heads;
   args.num_kv_heads = cache.num_kv_heads;
@@ -736,23 +596,16 @@ extern "C" pkv_status pkv_paged_attention_decode(
   args.scale_log2 = scale * kLog2e;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (plan.max_parts > 1 &&
-      cudaMemsetAsync(args.counters, 0,
-                      static_cast<size_t>(num_seqs) * cache.num_kv_heads * sizeof(int32_t),
-                      s) != cudaSuccess)
+  if (plan.ctrl_bytes > 0 && cudaMemsetAsync(ws, 0, plan.ctrl_bytes, s) != cudaSuccess)
     return PKV_ERR_CUDA;
   const bool big = args.group > 8;
   const bool bf16 = cache.dtype == PKV_BF16;
   if (cache.head_dim == 128)
-    st = bf16 ? launch_for_dim<__nv_bfloat16, 128>(cache.block_size, big, tmk, tmv, args,
-                                                  cache.num_kv_heads, num_seqs, s)
-              : launch_for_dim<__half, 128>(cache.block_size, big, tmk, tmv, args,
-                                            cache.num_kv_heads, num_seqs, s);
+    st = bf16 ? launch_for_dim<__nv_bfloat16, 128>(cache.block_size, big, tmk, tmv, args, s)
+              : launch_for_dim<__half, 128>(cache.block_size, big, tmk, tmv, args, s);
   else
-    st = bf16 ? launch_for_dim<__nv_bfloat16, 64>(cache.block_size, big, tmk, tmv, args,
-                                                 cache.num_kv_heads, num_seqs, s)
-              : launch_for_dim<__half, 64>(cache.block_size, big, tmk, tmv, args,
-                                           cache.num_kv_heads, num_seqs, s);
+    st = bf16 ? launch_for_dim<__nv_bfloat16, 64>(cache.block_size, big, tmk, tmv, args, s)
+              : launch_for_dim<__half, 64>(cache.block_size, big, tmk, tmv, args, s);
   if (st != PKV_OK || plan.max_parts <= kFuseMaxParts) return st;
 
   CombineArgs c{};

@@ -81,14 +81,17 @@ def test_host_validation_without_device(lib):
 
 
 def test_workspace_and_partition_queries(lib):
-    # automatic partitions of 512 tokens
-    assert bd.partition_size(64, 32, 16, 2048) == 512
-    assert bd.partition_size(4, 8, 32, 131072) == 512
+    # automatic partitions of 1024 tokens, smaller when the grid would be thin
+    assert bd.partition_size(64, 32, 16, 2048) == 1024
+    assert bd.partition_size(4, 8, 32, 131072) == 1024
+    assert bd.partition_size(1, 8, 16, 32768) == 256
+    assert bd.partition_size(4, 8, 16, 32768) == 512
     assert bd.partition_size(4, 8, 32, 131072, 512) == 512
     assert bd.partition_size(4, 8, 32, 131072, 500) == -1
-    # no split needed -> no workspace
+    # no split, no workspace
     assert bd.workspace_size(4, 4, 4, 64, 16, 33) == 0
-    # 131072 tokens in 512-token partitions: 256 partials of (D + 2) floats per
-    # (seq, head), then one int32 arrival counter per (seq, kv head)
-    assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 512) == 4 * 32 * 256 * 130 * 4 + 4 * 8 * 4
+    # 131072 tokens in 512-token partitions: one int32 arrival counter per
+    # (seq, kv head), then 256 partials of (D + 2) floats per (seq, head)
+    assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 512) == 4 * 8 * 4 + 4 * 32 * 256 * 130 * 4
+    assert bd.workspace_size(3, 4, 1, 64, 16, 2000, 256) == 16 + 3 * 4 * 8 * 66 * 4
     assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 24) == 0  # invalid partition
