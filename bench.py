@@ -376,35 +376,59 @@ def run_ours(args):
     clock = clocks.summary()
 
     # -------- end to end through the public API, host buffers -----------
+    # Every step copies its inputs from pinned host memory to the device and
+    # its output back.  As a serving loop would, the copies run on their own
+    # streams with double-buffered device tensors, so step i's upload and step
+    # i-1's read-back overlap step i-1's and step i's compute; every copy is
+    # inside the timed region.
     e2e = None
     if not args.no_e2e:
-        h_in = {n: t.detach().cpu().pin_memory() for n, t in
-                (("q", db.q), ("key", db.key), ("value", db.value), ("slots", db.slot_mapping),
-                 ("tables", db.block_tables), ("lens", db.context_lens))}
-        d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
-        h_out = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
+        names = ("q", "key", "value", "slots", "tables", "lens")
+        srcs = (db.q, db.key, db.value, db.slot_mapping, db.block_tables, db.context_lens)
+        h_in = {n: t.detach().cpu().pin_memory() for n, t in zip(names, srcs)}
+        d_in = [{n: torch.empty_like(t, device=dev) for n, t in h_in.items()} for _ in range(2)]
+        d_out = [torch.empty_like(db.out) for _ in range(2)]
+        h_out = [torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory() for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in h_in.values())
-        d2h = h_out.numel() * h_out.element_size()
+        d2h = h_out[0].numel() * h_out[0].element_size()
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for n in h_in:
-                d_in[n].copy_(h_in[n], non_blocking=True)
-            step(q=d_in["q"], out=db.out, key=d_in["key"], value=d_in["value"], slots=d_in["slots"],
-                 tables=d_in["tables"], lens=d_in["lens"])
-            h_out.copy_(db.out, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            up.wait_event(ev_done[b])  # step i-2 has consumed input buffer b
+            with torch.cuda.stream(up):
+                for n in names:
+                    d_in[b][n].copy_(h_in[n], non_blocking=True)
+                ev_in[b].record(up)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])  # step i-2's output has been read back
+            step(q=d_in[b]["q"], out=d_out[b], key=d_in[b]["key"], value=d_in[b]["value"],
+                 slots=d_in[b]["slots"], tables=d_in[b]["tables"], lens=d_in[b]["lens"])
+            ev_done[b].record(stream)
+            down.wait_event(ev_done[b])
+            with torch.cuda.stream(down):
+                h_out[b].copy_(d_out[b], non_blocking=True)
+                ev_out[b].record(down)
 
-        for _ in range(max(3, args.warmup)):
-            e2e_step()
+        for i in range(max(3, args.warmup)):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         e0.record(stream)
-        for _ in range(K):
-            e2e_step()
+        up.wait_event(e0)
+        for i in range(K):
+            e2e_step(i)
+        stream.wait_stream(down)
         e1.record(stream)
         torch.cuda.synchronize(dev)
+        if not torch.equal(h_out[(K - 1) % 2].view(torch.int16), db.out.view(torch.int16).cpu()):
+            raise RuntimeError("end-to-end output differs from the device-resident run")
         e2e = {"ms": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h}
 
     if int(status.item()) != 0:
@@ -468,7 +492,9 @@ def run_ours(args):
     if e2e:
         line["e2e"] = {"value": round(total_att_bytes / (e2e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": round(e2e_ms / K, 5)}
+                       "ms_per_step": round(e2e_ms / K, 5),
+                       "pipelining": "inputs uploaded and outputs read back on two copy streams, "
+                                     "double-buffered, overlapping compute of neighbouring steps"}
     if cpu:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
