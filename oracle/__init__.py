@@ -13,13 +13,19 @@ from .paged_kv import (  # noqa: F401
     copy_blocks,
     decode_bits,
     decode_sequence,
+    e4m3_decode,
+    e4m3_encode,
     encode_bits,
     free_request,
     kv_head_of,
     lse_combine,
     materialize,
+    materialize_fp8,
     paged_attention_decode,
+    paged_attention_decode_fp8,
     partial_state,
+    quantize_e4m3,
     reshape_and_cache,
+    reshape_and_cache_fp8,
     slot_location,
 )

@@ -240,3 +240,112 @@ def lse_combine(ms: np.ndarray, ls: np.ndarray, os: np.ndarray) -> np.ndarray:
     den = (w * ls).sum(axis=0)
     out[live] = num[live] / den[live][:, None]
     return out
+
+
+# ---------------------------------------------------------------------------
+# 8-bit KV cache (E4M3)
+# ---------------------------------------------------------------------------
+# lshu.cn/news/11644, "性能关键路径与瓶颈": quantising the KV cache to FP8/INT8
+# halves the bytes decode must read.  Format (OCP 8-bit floating point, E4M3):
+# 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+# holds subnormals m * 2^-9; there is no infinity; S.1111.111 is NaN, so the
+# largest finite magnitude is 1.75 * 2^8 = 448.  Values are stored as
+# e4m3(x / scale) with one fp32 scale per pool, rounded to nearest (ties to
+# even) and saturated to +-448; they read back as e4m3 * scale.
+# Pool layouts: K as [N][Hkv][B][D] (one row of D codes per token), V as
+# [N][Hkv][D][B] (one row of B codes per dimension).
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Exact float64 value of E4M3 codes (NaN for S.1111.111)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.ldexp(1.0, e - 7))
+    mag = np.where((e == 0xF) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """Round values to the nearest E4M3 code (ties to even), saturating
+    magnitudes above 448 to 448; NaN maps to 0x7F."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = np.signbit(x)
+    a = np.abs(x)
+    nan = np.isnan(a)
+    a = np.where(nan, 0.0, a)
+    # quantum of the binade: 2^(e-3) for normals (e >= -6), 2^-9 below
+    _, ex = np.frexp(a)  # a = f * 2^ex, 0.5 <= f < 1  ->  floor(log2 a) = ex - 1
+    e = np.maximum(ex - 1, -6)
+    quantum = np.ldexp(1.0, e - 3)
+    q = np.rint(a / quantum) * quantum  # np.rint rounds half to even
+    q = np.minimum(q, E4M3_MAX)
+    # encode the (exactly representable) rounded magnitude
+    _, ex2 = np.frexp(q)
+    e2 = ex2 - 1
+    normal = q >= 2.0 ** -6
+    exp_field = np.where(normal, e2 + 7, 0)
+    mant = np.where(normal, np.rint((q / np.ldexp(1.0, e2) - 1.0) * 8.0), np.rint(q / 2.0 ** -9))
+    code = (exp_field.astype(np.int64) << 3) | mant.astype(np.int64)
+    code = np.where(q == 0.0, 0, code)
+    code = code | np.where(sign, 0x80, 0)
+    code = np.where(nan, 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def quantize_e4m3(x_bits: np.ndarray, dtype: str, scale: float) -> np.ndarray:
+    """Codes stored for fp16/bf16 values x: e4m3(fp32(x) / fp32(scale)), the
+    division done once in IEEE fp32 (round to nearest)."""
+    x32 = decode_bits(x_bits, dtype).astype(np.float32)
+    return e4m3_encode((x32 / np.float32(scale)).astype(np.float64))
+
+
+def reshape_and_cache_fp8(k_cache, v_cache, key, value, slot_mapping, block_size, k_scale, v_scale,
+                          dtype):
+    """Quantising cache write: for t with slot p >= 0, K codes of token t go to
+    k_cache[p // B][h][p % B][:] and V codes to v_cache[p // B][h][:][p % B].
+    Returns updated copies."""
+    kc = np.array(k_cache, copy=True)
+    vc = np.array(v_cache, copy=True)
+    kq = quantize_e4m3(key, dtype, k_scale)
+    vq = quantize_e4m3(value, dtype, v_scale)
+    for t, slot in enumerate(np.asarray(slot_mapping).tolist()):
+        if slot < 0:
+            continue
+        b, o = slot_location(slot, block_size)
+        kc[b, :, o, :] = kq[t]
+        vc[b, :, :, o] = vq[t]
+    return kc, vc
+
+
+def materialize_fp8(k_cache, v_cache, table_row, length, block_size):
+    """Contiguous K, V codes [Hkv, length, D] of one sequence from the 8-bit
+    pools (V pool stored with dimensions before token positions)."""
+    pos = np.arange(length)
+    blocks = np.asarray(table_row)[pos // block_size].astype(np.int64)
+    offs = pos % block_size
+    K = k_cache[blocks, :, offs, :]  # [L, Hkv, D]
+    V = v_cache[blocks, :, :, offs]  # [L, Hkv, D]
+    return np.ascontiguousarray(K.transpose(1, 0, 2)), np.ascontiguousarray(V.transpose(1, 0, 2))
+
+
+def paged_attention_decode_fp8(q_bits, k_cache, v_cache, block_tables, context_lens, block_size, scale,
+                               k_scale, v_scale, dtype, seqs=None) -> np.ndarray:
+    """Decode attention over 8-bit pools: K and V read back as code * scale
+    (exactly, in float64), then textbook softmax attention."""
+    S, Hq, D = q_bits.shape
+    Hkv = k_cache.shape[1]
+    out = np.full((S, Hq, D), np.nan)
+    for s in (range(S) if seqs is None else seqs):
+        L = int(context_lens[s])
+        q = decode_bits(q_bits[s], dtype)
+        Kc, Vc = materialize_fp8(k_cache, v_cache, block_tables[s], L, block_size)
+        for g in range(Hkv):
+            rows = [h for h in range(Hq) if kv_head_of(h, Hq, Hkv) == g]
+            K = e4m3_decode(Kc[g]) * k_scale
+            V = e4m3_decode(Vc[g]) * v_scale
+            out[s, rows] = attend(q[rows], K, V, scale)
+    return out

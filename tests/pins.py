@@ -382,3 +382,88 @@ ALL_CHECKS = [
     check_copy_blocks_example,
     check_storage_formats,
 ]
+
+
+# ---------------------------------------------------------------------------
+# 8-bit (E4M3) pools
+# ---------------------------------------------------------------------------
+
+def check_e4m3_known_codes():
+    """Codes fixed by the format (1 sign, 4 exponent bits with bias 7, 3
+    mantissa bits, subnormals m * 2^-9, largest finite 448, S.1111.111 NaN),
+    round to nearest with ties to even, saturation to 448."""
+    vals = np.array([1.0, -2.0, 448.0, 500.0, -1e9, 2.0 ** -9, 2.0 ** -6, 0.0, 1.0625, 1.1875,
+                     1.5 * 2.0 ** -9, 0.9 * 2.0 ** -10, 240.0, 232.0])
+    want = [0x38, 0xC0, 0x7E, 0x7E, 0xFE, 0x01, 0x08, 0x00, 0x38, 0x3A, 0x02, 0x00, 0x77, 0x76]
+    assert O.e4m3_encode(vals).tolist() == want
+    assert O.e4m3_decode(np.array([0x38, 0x7E, 0x01, 0x08, 0xB9], np.uint8)).tolist() == \
+        [1.0, 448.0, 2.0 ** -9, 2.0 ** -6, -1.125]
+    assert np.isnan(O.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+
+
+def check_e4m3_all_codes_roundtrip():
+    codes = np.arange(256, dtype=np.uint8)
+    v = O.e4m3_decode(codes)
+    fin = ~np.isnan(v)
+    assert fin.sum() == 254
+    assert np.array_equal(O.e4m3_encode(v[fin]), codes[fin])
+    pos = np.sort(v[fin][v[fin] > 0])
+    assert pos[0] == 2.0 ** -9 and pos[-1] == 448.0 and len(pos) == 126
+
+
+def check_e4m3_against_torch():
+    """Library special case: torch's float8_e4m3fn conversion (round to
+    nearest even) agrees on in-range values."""
+    import torch
+
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-9, 6, 100000))).astype(np.float32)
+    x = x[np.abs(x) < 448]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x.astype(np.float64)), ref)
+
+
+def check_fp8_cache_write_example():
+    """Two tokens into 8-token blocks: slot 3 and slot 13 (block 1, position 5);
+    K lands in row (block, head, position), V in column (block, head, :, position)."""
+    N, H, B, D = 3, 2, 8, 4
+    kc = np.full((N, H, B, D), 0x7F, np.uint8)
+    vc = np.full((N, H, D, B), 0x7F, np.uint8)
+    one, two = 0x3C00, 0x4000  # fp16 1.0, 2.0
+    key = np.array([[[one] * D] * H, [[two] * D] * H], np.uint16)
+    value = key.copy()
+    k2, v2 = O.reshape_and_cache_fp8(kc, vc, key, value, np.array([3, 13]), B, 0.5, 2.0, W.F16)
+    # 1.0 / 0.5 = 2 -> 0x40; 2.0 / 0.5 = 4 -> 0x48; 1.0 / 2 = 0.5 -> 0x30; 2.0 / 2 = 1 -> 0x38
+    ek, ev = kc.copy(), vc.copy()
+    ek[0, :, 3, :] = 0x40
+    ek[1, :, 5, :] = 0x48
+    ev[0, :, :, 3] = 0x30
+    ev[1, :, :, 5] = 0x38
+    assert np.array_equal(k2, ek) and np.array_equal(v2, ev)
+
+
+def check_fp8_decode_matches_fp16_decode():
+    """With scales that are powers of two every E4M3 value is exact in fp16:
+    decoding the 8-bit pools equals decoding fp16 pools that hold those
+    values in the fp16 layout (pins the 8-bit layouts to the fp16 path)."""
+    base = W.small_case(51, num_seqs=5, num_q_heads=8, num_kv_heads=2, head_dim=16, block_size=8,
+                        dtype=W.F16, max_len=40, write_new_token=False)
+    f8 = W.fp8_variant(base, 52, k_scale=0.25, v_scale=2.0)
+    kv = O.e4m3_decode(f8.k_cache) * 0.25
+    vv = O.e4m3_decode(f8.v_cache) * 2.0
+    k16 = O.encode_bits(kv, W.F16)
+    v16 = O.encode_bits(vv.transpose(0, 1, 3, 2), W.F16)
+    ref = O.paged_attention_decode(base.q, k16, v16, base.block_tables, base.context_lens, 8, base.scale, W.F16)
+    got = O.paged_attention_decode_fp8(base.q, f8.k_cache, f8.v_cache, base.block_tables, base.context_lens,
+                                       8, base.scale, 0.25, 2.0, W.F16)
+    assert np.array_equal(got, ref)
+
+
+FP8_CHECKS = [
+    check_e4m3_known_codes,
+    check_e4m3_all_codes_roundtrip,
+    check_e4m3_against_torch,
+    check_fp8_cache_write_example,
+    check_fp8_decode_matches_fp16_decode,
+]
+ALL_CHECKS += FP8_CHECKS

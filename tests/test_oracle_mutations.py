@@ -80,6 +80,26 @@ def _encode_truncate(x, dtype):
     return x.astype(np.float16).view(np.uint16)
 
 
+_orig_e4m3 = O.e4m3_encode
+
+
+def _e4m3_truncating(x):
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(a)
+    q = np.ldexp(np.floor(np.ldexp(a, -(np.maximum(ex - 1, -6) - 3))), np.maximum(ex - 1, -6) - 3)
+    return _orig_e4m3(np.copysign(q, x))
+
+
+def _materialize_fp8_v_untransposed(k_cache, v_cache, table_row, length, block_size):
+    pos = np.arange(length)
+    blocks = np.asarray(table_row)[pos // block_size].astype(np.int64)
+    offs = pos % block_size
+    K = k_cache[blocks, :, offs, :]
+    V = v_cache.transpose(0, 1, 3, 2)[blocks, :, offs, :]
+    return np.ascontiguousarray(K.transpose(1, 0, 2)), np.ascontiguousarray(V.transpose(1, 0, 2))
+
+
 MUTANTS = {
     "attend_drops_scale": ("attend", _attend_no_scale),
     "attend_uses_keys_as_values": ("attend", _attend_values_from_keys),
@@ -93,6 +113,8 @@ MUTANTS = {
     "lse_combine_unweighted_sum": ("lse_combine", _lse_unweighted_l),
     "append_without_filling_block": ("append_token", _append_always_new_block),
     "bf16_truncates_instead_of_rounding": ("encode_bits", _encode_truncate),
+    "e4m3_truncates_instead_of_rounding": ("e4m3_encode", _e4m3_truncating),
+    "fp8_v_pool_read_untransposed": ("materialize_fp8", _materialize_fp8_v_untransposed),
 }
 
 

@@ -431,3 +431,63 @@ def shard_batch(batch: PagedBatch, rank: int, world: int) -> PagedBatch:
         block_tables_before_cow=None if before is None else rt(before),
         partition_size=batch.partition_size, seed=batch.seed,
     )
+
+
+# --------------------------------------------------------------------------
+# 8-bit (E4M3) pools
+# --------------------------------------------------------------------------
+FP8_POISON = 0x7F  # an E4M3 NaN code
+
+
+def random_e4m3_codes(rng: np.random.Generator, shape, exp_lo: int = 4, exp_hi: int = 10) -> np.ndarray:
+    """Random E4M3 codes drawn field by field (no rounding involved): a random
+    sign, an exponent field uniform on [exp_lo, exp_hi] and a uniform 3-bit
+    mantissa; magnitudes span 2^(exp_lo-7) .. 1.875 * 2^(exp_hi-7)."""
+    sign = rng.integers(0, 2, size=shape, dtype=np.uint8) << 7
+    exp = rng.integers(exp_lo, exp_hi + 1, size=shape, dtype=np.uint8) << 3
+    man = rng.integers(0, 8, size=shape, dtype=np.uint8)
+    return (sign | exp | man).astype(np.uint8)
+
+
+@dataclass
+class Fp8Batch:
+    """A decode step over 8-bit pools: the fp16/bf16 batch's queries, new
+    tokens, tables and lengths, with K [N][Hkv][B][D] and V [N][Hkv][D][B]
+    pools of E4M3 codes and one scale per pool."""
+
+    base: PagedBatch
+    k_cache: np.ndarray  # uint8 [N, Hkv, B, D]
+    v_cache: np.ndarray  # uint8 [N, Hkv, D, B]
+    k_scale: float
+    v_scale: float
+
+    def __getattr__(self, name):
+        return getattr(self.base, name)
+
+
+def fp8_variant(batch: PagedBatch, seed: int, k_scale: float = 0.125, v_scale: float = 0.0625) -> Fp8Batch:
+    """Replace the pools of ``batch`` by 8-bit pools: every position a sequence
+    attends to (except this step's new tokens, which the step writes) holds a
+    random code; every other slot holds the NaN code."""
+    rng = np.random.default_rng(seed)
+    N, Hkv, B, D = batch.k_cache.shape
+    kc = np.full((N, Hkv, B, D), FP8_POISON, dtype=np.uint8)
+    vc = np.full((N, Hkv, D, B), FP8_POISON, dtype=np.uint8)
+    for s in range(batch.num_seqs):
+        L = int(batch.context_lens[s])
+        if L == 0:
+            continue
+        kt = random_e4m3_codes(rng, (L, Hkv, D))
+        vt = random_e4m3_codes(rng, (L, Hkv, D))
+        nb = _blocks_for(L, B)
+        pad = nb * B - L
+        kp = np.concatenate([kt, np.full((pad, Hkv, D), FP8_POISON, np.uint8)]).reshape(nb, B, Hkv, D)
+        vp = np.concatenate([vt, np.full((pad, Hkv, D), FP8_POISON, np.uint8)]).reshape(nb, B, Hkv, D)
+        rows = batch.block_tables[s, :nb]
+        kc[rows] = kp.transpose(0, 2, 1, 3)
+        vc[rows] = vp.transpose(0, 2, 3, 1)
+    for slot in batch.slot_mapping.tolist():  # slots this step writes start poisoned
+        if slot >= 0:
+            kc[slot // B, :, slot % B, :] = FP8_POISON
+            vc[slot // B, :, :, slot % B] = FP8_POISON
+    return Fp8Batch(base=batch, k_cache=kc, v_cache=vc, k_scale=k_scale, v_scale=v_scale)
