@@ -96,7 +96,7 @@ def _materialize_fp8_v_untransposed(k_cache, v_cache, table_row, length, block_s
     blocks = np.asarray(table_row)[pos // block_size].astype(np.int64)
     offs = pos % block_size
     K = k_cache[blocks, :, offs, :]
-    V = v_cache.transpose(0, 1, 3, 2)[blocks, :, offs, :]
+    V = v_cache[blocks, :, offs, :]  # reads a dimension row as if it were a token row
     return np.ascontiguousarray(K.transpose(1, 0, 2)), np.ascontiguousarray(V.transpose(1, 0, 2))
 
 
