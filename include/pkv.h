@@ -70,7 +70,7 @@ typedef enum {
 #define PKV_DEV_BAD_LEN 0x4    /* context_len < 0, > max_context_len or > max_blocks_per_seq * block_size */
 #define PKV_DEV_TIMEOUT 0x8    /* a copy into shared memory did not complete within ~1 s */
 
-typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+typedef enum { PKV_F16 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
 
 /* Shape of one layer's block pool (shared by k_cache and v_cache). */
 typedef struct {
@@ -78,8 +78,24 @@ typedef struct {
   int32_t block_size;   /* B: tokens per block; 8, 16, 32 or 64 */
   int32_t num_kv_heads; /* Hkv >= 1 */
   int32_t head_dim;     /* D: 64 or 128 */
-  pkv_dtype dtype;      /* element type of both pools, of queries and outputs */
+  pkv_dtype dtype;      /* element type of both pools (and, for fp16/bf16 pools,
+                           of queries and outputs) */
 } pkv_cache_desc;
+
+/*
+ * 8-bit pools (dtype PKV_FP8_E4M3).  Source: lshu.cn/news/11644, "性能关键路径
+ * 与瓶颈": quantising the KV cache to FP8/INT8 is the most effective decode
+ * optimisation, halving the bytes read.  Codes are OCP E4M3 (1 sign, 4
+ * exponent bits with bias 7, 3 mantissa bits, subnormals, no infinity, largest
+ * finite 448).  A value x is stored as e4m3(x / scale), the division done in
+ * IEEE fp32 and the result rounded to nearest even and saturated to +-448;
+ * it reads back as code * scale, with one fp32 scale per pool (k_scale,
+ * v_scale).  Layouts: k_cache [num_blocks][num_kv_heads][block_size][head_dim]
+ * (one row of head_dim codes per token) and v_cache
+ * [num_blocks][num_kv_heads][head_dim][block_size] (one row of block_size
+ * codes per dimension).  Supported: head_dim 128, block_size 16, 32 or 64.
+ * pkv_copy_blocks works on 8-bit pools as on fp16/bf16 ones.
+ */
 
 /*
  * pkv_reshape_and_cache - write this step's new K/V tokens into their slots.
@@ -98,9 +114,10 @@ typedef struct {
  *                 (0 means num_kv_heads*head_dim); heads of a token contiguous.
  * k_cache,v_cache device, layout above, 16-byte aligned.
  * slot_mapping    device, int64 [num_tokens].
- * Errors: NULL pointers (when num_tokens > 0), bad desc -> status; a slot
- *   >= num_blocks*B -> PKV_DEV_BAD_SLOT, that token skipped.  Two tokens with
- *   the same slot in one call race (caller error, result unspecified).
+ * Errors: NULL pointers (when num_tokens > 0), bad desc or 8-bit pools
+ *   -> status; a slot >= num_blocks*B -> PKV_DEV_BAD_SLOT, that token skipped.
+ *   Two tokens with the same slot in one call race (caller error, result
+ *   unspecified).
  */
 PKV_API pkv_status pkv_reshape_and_cache(const void *key, const void *value, int64_t key_token_stride,
                                  int64_t value_token_stride, void *k_cache, void *v_cache,
@@ -231,6 +248,37 @@ PKV_API pkv_status pkv_paged_attention_decode_noalloc(
     const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
     int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
     int32_t partition_size, int32_t *d_status, pkv_stream_t stream);
+
+/*
+ * pkv_reshape_and_cache_fp8 - pkv_reshape_and_cache into 8-bit pools: every
+ * new K and V value is quantised as described above, K codes go to
+ * k_cache[p / B][h][p % B][:] and V codes to v_cache[p / B][h][:][p % B].
+ * key, value: fp16 or bf16 (input_dtype), same layout and strides as
+ * pkv_reshape_and_cache; cache.dtype must be PKV_FP8_E4M3; k_scale, v_scale > 0.
+ * Errors as pkv_reshape_and_cache.
+ */
+PKV_API pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *value,
+                                             int64_t key_token_stride, int64_t value_token_stride,
+                                             pkv_dtype input_dtype, void *k_cache, void *v_cache,
+                                             pkv_cache_desc cache, const int64_t *slot_mapping,
+                                             int32_t num_tokens, float k_scale, float v_scale,
+                                             int32_t *d_status, pkv_stream_t stream);
+
+/*
+ * pkv_paged_attention_decode_fp8 - pkv_paged_attention_decode over 8-bit
+ * pools: K and V read back as code * k_scale and code * v_scale.  query and
+ * out are fp16 or bf16 (query_dtype); the products run on fp16 operands
+ * (E4M3 codes are exact in fp16; bf16 queries are converted to fp16, exact
+ * for magnitudes in [2^-24, 65504]) with fp32 accumulation.  cache.dtype must
+ * be PKV_FP8_E4M3.  Other arguments, the workspace and errors as
+ * pkv_paged_attention_decode.
+ */
+PKV_API pkv_status pkv_paged_attention_decode_fp8(
+    void *out, const void *query, pkv_dtype query_dtype, const void *k_cache, const void *v_cache,
+    pkv_cache_desc cache, const int32_t *block_tables, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+    float scale, float k_scale, float v_scale, int32_t partition_size, void *workspace,
+    size_t workspace_bytes, int32_t *d_status, pkv_stream_t stream);
 
 /* Static English text for a status code. */
 PKV_API const char *pkv_status_string(pkv_status status);

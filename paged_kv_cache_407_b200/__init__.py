@@ -13,10 +13,13 @@ from .binding import (  # noqa: F401
     PkvError,
     cache_desc,
     copy_blocks,
+    fp8_cache_desc,
     library,
     paged_attention_decode,
+    paged_attention_decode_fp8,
     partition_size,
     reshape_and_cache,
+    reshape_and_cache_fp8,
     version,
     workspace_size,
 )

@@ -11,12 +11,15 @@ import numpy as np
 
 
 def decode_bytes(context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 block_size: int, elem_bytes: int = 2) -> dict:
+                 block_size: int, elem_bytes: int = 2, kv_elem_bytes: int | None = None) -> dict:
     """Bytes of one decode-attention call: K and V of every context token,
-    the queries, the outputs, the Block Table entries in use and the lengths."""
+    the queries, the outputs, the Block Table entries in use and the lengths.
+    ``kv_elem_bytes``: bytes per cached K/V element (1 for 8-bit pools;
+    default ``elem_bytes``)."""
     lens = np.asarray(context_lens, dtype=np.int64)
     S = lens.size
-    kv = int(lens.sum()) * num_kv_heads * head_dim * elem_bytes * 2
+    kv_b = elem_bytes if kv_elem_bytes is None else kv_elem_bytes
+    kv = int(lens.sum()) * num_kv_heads * head_dim * kv_b * 2
     q = S * num_q_heads * head_dim * elem_bytes
     out = q
     tables = int(((lens + block_size - 1) // block_size).sum()) * 4
@@ -34,10 +37,11 @@ def decode_bytes_padded_kv(context_lens, num_kv_heads: int, head_dim: int, block
 
 
 def reshape_and_cache_bytes(num_tokens: int, num_kv_heads: int, head_dim: int,
-                            elem_bytes: int = 2) -> int:
+                            elem_bytes: int = 2, cache_elem_bytes: int | None = None) -> int:
     """Read the new K and V rows, write them into the pool, read the slots."""
-    rows = num_tokens * num_kv_heads * head_dim * elem_bytes * 2
-    return 2 * rows + 8 * num_tokens
+    c_b = elem_bytes if cache_elem_bytes is None else cache_elem_bytes
+    rows = num_tokens * num_kv_heads * head_dim * 2
+    return rows * elem_bytes + rows * c_b + 8 * num_tokens
 
 
 def copy_blocks_bytes(num_pairs: int, num_kv_heads: int, block_size: int, head_dim: int,

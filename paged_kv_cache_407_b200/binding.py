@@ -30,7 +30,9 @@ DEV_TIMEOUT = 0x8
 
 PKV_F16 = 0
 PKV_BF16 = 1
+PKV_FP8_E4M3 = 2
 _DTYPES = {torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
+_FP8_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 
 # Every function declared in include/pkv.h, with (restype, argtypes).
 _c_void_p, _i32, _i64, _f32, _size_t = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -61,6 +63,13 @@ SIGNATURES = {
                                                           _i32, _i32, _f32, _i32, _c_void_p, _c_void_p]),
     "pkv_copy_blocks": (ctypes.c_int, [_c_void_p, _c_void_p, CacheDesc, _c_void_p, _i32, _c_void_p,
                                        _c_void_p]),
+    "pkv_reshape_and_cache_fp8": (ctypes.c_int, [_c_void_p, _c_void_p, _i64, _i64, ctypes.c_int, _c_void_p,
+                                                 _c_void_p, CacheDesc, _c_void_p, _i32, _f32, _f32,
+                                                 _c_void_p, _c_void_p]),
+    "pkv_paged_attention_decode_fp8": (ctypes.c_int, [_c_void_p, _c_void_p, ctypes.c_int, _c_void_p, _c_void_p,
+                                                      CacheDesc, _c_void_p, _i32, _c_void_p, _i32, _i32, _i32,
+                                                      _f32, _f32, _f32, _i32, _c_void_p, _size_t, _c_void_p,
+                                                      _c_void_p]),
     "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "pkv_version": (_i32, []),
 }
@@ -223,10 +232,78 @@ def paged_attention_decode_noalloc(out, query, k_cache, v_cache, block_tables, c
     return out
 
 
+def fp8_cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor) -> CacheDesc:
+    """Descriptor of 8-bit pools: K ``[N, Hkv, B, D]``, V ``[N, Hkv, D, B]`` of
+    E4M3 codes (``torch.uint8`` or ``torch.float8_e4m3fn``)."""
+    if k_cache.dtype not in _FP8_DTYPES or v_cache.dtype not in _FP8_DTYPES:
+        raise TypeError("8-bit pools must be torch.uint8 or torch.float8_e4m3fn")
+    if k_cache.dim() != 4 or not (k_cache.is_contiguous() and v_cache.is_contiguous()):
+        raise ValueError("8-bit pools must be contiguous 4-d tensors")
+    N, Hkv, B, D = k_cache.shape
+    if tuple(v_cache.shape) != (N, Hkv, D, B):
+        raise ValueError("v_cache must be [num_blocks, num_kv_heads, head_dim, block_size]")
+    return CacheDesc(N, B, Hkv, D, PKV_FP8_E4M3)
+
+
+def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, d_status=None,
+                          stream=None):
+    """Quantising write of new tokens ``key/value [T, Hkv, D]`` (fp16/bf16) into
+    8-bit pools: codes e4m3(x / scale)."""
+    desc = fp8_cache_desc(k_cache, v_cache)
+    T = key.shape[0]
+    for t in (key, value):
+        if t.dim() != 3 or tuple(t.shape[1:]) != (desc.num_kv_heads, desc.head_dim) or t.dtype not in _DTYPES:
+            raise ValueError("key/value must be fp16/bf16 [T, num_kv_heads, head_dim]")
+        if t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("key/value heads and dims must be contiguous within a token")
+    if value.dtype != key.dtype:
+        raise ValueError("key and value must have the same dtype")
+    if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T or not slot_mapping.is_contiguous():
+        raise ValueError("slot_mapping must be a contiguous int64 tensor with one entry per token")
+    st = library().pkv_reshape_and_cache_fp8(
+        _ptr(key), _ptr(value), key.stride(0), value.stride(0), _DTYPES[key.dtype], _ptr(k_cache),
+        _ptr(v_cache), desc, _ptr(slot_mapping), T, float(k_scale), float(v_scale), _ptr(d_status),
+        _stream(stream, k_cache.device))
+    _check(st, "pkv_reshape_and_cache_fp8")
+
+
+def paged_attention_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                               scale, k_scale, v_scale, partition_size=0, workspace=None, d_status=None,
+                               stream=None):
+    """Decode attention over 8-bit pools (K, V read back as code * scale);
+    query/out fp16 or bf16 ``[S, Hq, D]``."""
+    desc = fp8_cache_desc(k_cache, v_cache)
+    S, Hq, D = query.shape
+    if query.dtype not in _DTYPES or out.dtype != query.dtype or out.shape != query.shape:
+        raise ValueError("query/out must be fp16/bf16 [S, Hq, head_dim] of one dtype")
+    if not (query.is_contiguous() and out.is_contiguous()):
+        raise ValueError("query/out must be contiguous")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S \
+            or not block_tables.is_contiguous():
+        raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
+    if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
+        raise ValueError("context_lens must be a contiguous int32 [S] tensor")
+    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = library().pkv_paged_attention_decode_fp8(
+        _ptr(out), _ptr(query), _DTYPES[query.dtype], _ptr(k_cache), _ptr(v_cache), desc,
+        _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len),
+        float(scale), float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
+        _ptr(d_status), _stream(stream, query.device))
+    _check(st, "pkv_paged_attention_decode_fp8")
+    return out
+
+
 def copy_blocks(k_cache, v_cache, block_pairs, d_status=None, stream=None):
-    """Copy-on-write: block ``pairs[i, 1]`` of both pools becomes a copy of ``pairs[i, 0]``."""
-    desc = cache_desc(k_cache)
-    _same_pool(k_cache, v_cache)
+    """Copy-on-write: block ``pairs[i, 1]`` of both pools becomes a copy of
+    ``pairs[i, 0]`` (fp16/bf16 pools, or 8-bit pools)."""
+    if k_cache.dtype in _FP8_DTYPES:
+        desc = fp8_cache_desc(k_cache, v_cache)
+    else:
+        desc = cache_desc(k_cache)
+        _same_pool(k_cache, v_cache)
     if block_pairs.dtype != torch.int64 or block_pairs.dim() != 2 or block_pairs.shape[1] != 2 \
             or not block_pairs.is_contiguous():
         raise ValueError("block_pairs must be a contiguous int64 [num_pairs, 2] tensor")

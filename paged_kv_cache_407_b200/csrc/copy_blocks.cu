@@ -56,8 +56,8 @@ extern "C" pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_de
     return PKV_ERR_MISALIGNED;
   if (num_pairs > 2147483647 / 2) return PKV_ERR_TOO_LARGE;
   if ((st = check_device()) != PKV_OK) return st;
-  const int64_t block_vecs =
-      static_cast<int64_t>(cache.num_kv_heads) * cache.block_size * cache.head_dim / 8;
+  const int64_t block_vecs = static_cast<int64_t>(cache.num_kv_heads) * cache.block_size *
+                             cache.head_dim * elem_bytes(cache.dtype) / 16;
   const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyUnroll;
   const unsigned slices = static_cast<unsigned>(std::min<int64_t>((block_vecs + per_cta - 1) / per_cta, 64));
   dim3 grid(static_cast<unsigned>(num_pairs), 2u, slices);

@@ -11,7 +11,19 @@
 // The score accumulator fragment is, element for element, the A fragment of
 // P V, so P never moves between lanes.  P enters the second MMA as a 16-bit
 // high part plus a 16-bit residual, which keeps it at about fp32 precision.
+//
+// 8-bit pools (KV8): K tiles hold one 128-byte row of E4M3 codes per token, V
+// tiles one row of BS codes per dimension (V stored transposed).  ldmatrix on
+// such rows hands each lane four consecutive codes, which two cvt
+// instructions turn into the two fp16 pairs of an MMA fragment.  To make the
+// token order of the score fragment match those V fragments, the K rows of
+// 8-token column tile 2t+u are tokens {0,1,4,5,8,9,12,13} + 2u of the 16-token
+// group t, so a lane's scores are tokens 4c..4c+3 of the group (c = lane % 4);
+// the head-dimension order inside each 16-wide step is permuted the same way
+// for Q and K.  Operands are fp16 (E4M3 codes are exact in fp16).
 #pragma once
+
+#include <type_traits>
 
 #include "pkv_device.cuh"
 
@@ -28,13 +40,23 @@ __device__ __forceinline__ uint32_t tile_off(int tok, int chunk) {
                                (((chunk & 7) ^ (tok & 7)) << 4));
 }
 
-template <typename T, int D, int BS, bool BIG>
+// Byte offset of 16-byte chunk `chunk` of row `row` in an 8-bit V tile whose
+// rows are BS bytes, written by TMA with a BS-byte swizzle span (none at 16).
+template <int BS>
+__device__ __forceinline__ uint32_t v8_off(int row, int chunk) {
+  if constexpr (BS == 16) return static_cast<uint32_t>(row * 16);
+  if constexpr (BS == 32) return static_cast<uint32_t>(row * 32 + ((chunk ^ ((row >> 2) & 1)) << 4));
+  return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+
+template <typename T, int D, int BS, bool BIG, bool KV8 = false>
 struct DecodeState {
   static constexpr int kNT = BS / 8;  // 8-token column tiles per block
   static constexpr int kDT = D / 8;   // 8-wide column tiles of the output
   static constexpr int kKS = D / 16;  // 16-deep steps of the score product
-  using MMA = Mma<T>;
-  using PK = Pack<T>;
+  using OP = typename std::conditional<KV8, __half, T>::type;  // MMA operand type
+  using MMA = Mma<OP>;
+  using PK = Pack<OP>;
 
   uint32_t qa0[kKS], qa1[kKS], qa2[kKS], qa3[kKS];  // Q as A fragments (rows r, r + 8)
   float m0, m1, l0, l1;                             // running max / sum, rows r and r + 8
@@ -42,6 +64,10 @@ struct DecodeState {
 
   // Query rows of the group: q points at G consecutive rows of D elements.
   __device__ __forceinline__ void load_q(const T *q, int G, int lane) {
+    if constexpr (KV8) {
+      load_q_kv8(q, G, lane);
+      return;
+    }
     const int r = lane >> 2;
     const int c2 = (lane & 3) * 2;
     const uint32_t *q32 = reinterpret_cast<const uint32_t *>(q);
@@ -52,6 +78,35 @@ struct DecodeState {
       if constexpr (BIG) {
         qa1[kk] = r + 8 < G ? q32[((r + 8) * D + 16 * kk + c2) >> 1] : 0u;
         qa3[kk] = r + 8 < G ? q32[((r + 8) * D + 16 * kk + 8 + c2) >> 1] : 0u;
+      } else {
+        qa1[kk] = 0u;
+        qa3[kk] = 0u;
+      }
+    }
+  }
+
+  // Two consecutive query elements as one fp16x2 operand word.
+  static __device__ __forceinline__ uint32_t q_pair(const T *p) {
+    if constexpr (std::is_same<T, __half>::value) {
+      return *reinterpret_cast<const uint32_t *>(p);
+    } else {
+      const float2 f = Pack<T>::unpack(*reinterpret_cast<const uint32_t *>(p));
+      return Pack<__half>::pack(f.x, f.y);
+    }
+  }
+
+  // KV8 order: within each 16-wide step kk, lane c's k-slots {2c, 2c+1} are
+  // dims 16kk + 4c + {0, 1} and k-slots {2c+8, 2c+9} are dims 16kk + 4c + {2, 3}.
+  __device__ __forceinline__ void load_q_kv8(const T *q, int G, int lane) {
+    const int r = lane >> 2;
+    const int c4 = (lane & 3) * 4;
+#pragma unroll
+    for (int kk = 0; kk < kKS; ++kk) {
+      qa0[kk] = r < G ? q_pair(q + r * D + 16 * kk + c4) : 0u;
+      qa2[kk] = r < G ? q_pair(q + r * D + 16 * kk + c4 + 2) : 0u;
+      if constexpr (BIG) {
+        qa1[kk] = r + 8 < G ? q_pair(q + (r + 8) * D + 16 * kk + c4) : 0u;
+        qa3[kk] = r + 8 < G ? q_pair(q + (r + 8) * D + 16 * kk + c4 + 2) : 0u;
       } else {
         qa1[kk] = 0u;
         qa3[kk] = 0u;
@@ -79,7 +134,29 @@ struct DecodeState {
     float sc[kNT][4];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-    if constexpr (BS >= 16) {
+    if constexpr (KV8) {
+      // matrices: 0 = tile 2tp, step 2kk2; 1 = tile 2tp+1, step 2kk2; 2, 3 = step 2kk2+1
+      const int perm = (ri >> 1) * 4 + (ri & 1) + ((mi & 1) << 1);
+#pragma unroll
+      for (int kk2 = 0; kk2 < kKS / 2; ++kk2) {
+#pragma unroll
+        for (int tp = 0; tp < BS / 16; ++tp) {
+          uint32_t r0, r1, r2, r3;
+          const int tok = tp * 16 + perm;
+          const int chunk = 2 * kk2 + (mi >> 1);
+          ldsm_x4(kb + tok * 128 + (((chunk ^ (tok & 7)) & 7) << 4), r0, r1, r2, r3);
+          const int k0 = 2 * kk2, k1 = 2 * kk2 + 1;
+          MMA::k16(sc[2 * tp], qa0[k0], qa1[k0], qa2[k0], qa3[k0], e4m3x2_to_f16x2(r0),
+                   e4m3x2_to_f16x2(r0 >> 16));
+          MMA::k16(sc[2 * tp + 1], qa0[k0], qa1[k0], qa2[k0], qa3[k0], e4m3x2_to_f16x2(r1),
+                   e4m3x2_to_f16x2(r1 >> 16));
+          MMA::k16(sc[2 * tp], qa0[k1], qa1[k1], qa2[k1], qa3[k1], e4m3x2_to_f16x2(r2),
+                   e4m3x2_to_f16x2(r2 >> 16));
+          MMA::k16(sc[2 * tp + 1], qa0[k1], qa1[k1], qa2[k1], qa3[k1], e4m3x2_to_f16x2(r3),
+                   e4m3x2_to_f16x2(r3 >> 16));
+        }
+      }
+    } else if constexpr (BS >= 16) {
 #pragma unroll
       for (int kk = 0; kk < kKS; ++kk) {
 #pragma unroll
@@ -108,7 +185,11 @@ struct DecodeState {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float v = sc[nt][j] * scale_log2;
-        if (partial && nt * 8 + c2 + (j & 1) >= nv) v = -INFINITY;
+        // token of this score: tile nt column c2 + (j & 1), or in KV8 order
+        // group nt/2, tokens 4c + 2 * (nt & 1) + (j & 1)
+        const int tok = KV8 ? (nt >> 1) * 16 + 2 * c2 + ((nt & 1) << 1) + (j & 1)
+                            : nt * 8 + c2 + (j & 1);
+        if (partial && tok >= nv) v = -INFINITY;
         sc[nt][j] = v;
       }
     float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -160,7 +241,45 @@ struct DecodeState {
     }
 
     // ---- O[16 x D] += P[16 x BS] . V --------------------------------------
-    if constexpr (BS >= 16) {
+    if constexpr (KV8) {
+#pragma unroll
+      for (int tp = 0; tp < BS / 16; ++tp) {
+        // a lane's P for the group: tokens 4c, 4c+1 (k-slots 2c, 2c+1) and
+        // 4c+2, 4c+3 (k-slots 2c+8, 2c+9)
+        const uint32_t h0 = PK::pack(sc[2 * tp][0], sc[2 * tp][1]);
+        const uint32_t h2 = PK::pack(sc[2 * tp + 1][0], sc[2 * tp + 1][1]);
+        const float2 f0 = PK::unpack(h0);
+        const float2 f2 = PK::unpack(h2);
+        const uint32_t e0 = PK::pack(sc[2 * tp][0] - f0.x, sc[2 * tp][1] - f0.y);
+        const uint32_t e2 = PK::pack(sc[2 * tp + 1][0] - f2.x, sc[2 * tp + 1][1] - f2.y);
+        uint32_t h1 = 0u, h3 = 0u, e1 = 0u, e3 = 0u;
+        if constexpr (BIG) {
+          h1 = PK::pack(sc[2 * tp][2], sc[2 * tp][3]);
+          h3 = PK::pack(sc[2 * tp + 1][2], sc[2 * tp + 1][3]);
+          const float2 f1 = PK::unpack(h1);
+          const float2 f3 = PK::unpack(h3);
+          e1 = PK::pack(sc[2 * tp][2] - f1.x, sc[2 * tp][3] - f1.y);
+          e3 = PK::pack(sc[2 * tp + 1][2] - f3.x, sc[2 * tp + 1][3] - f3.y);
+        }
+        const int t0 = tp * 16 + 2 * c2;  // first of this lane's four tokens
+        const bool vmask = partial && (tp * 16 + 16 > nv);
+        const uint32_t bmask = (t0 < nv ? 0x000000ffu : 0u) | (t0 + 1 < nv ? 0x0000ff00u : 0u) |
+                               (t0 + 2 < nv ? 0x00ff0000u : 0u) | (t0 + 3 < nv ? 0xff000000u : 0u);
+#pragma unroll
+        for (int dq = 0; dq < D / 32; ++dq) {
+          uint32_t v[4];
+          ldsm_x4(vb + v8_off<BS>(32 * dq + 8 * mi + ri, tp), v[0], v[1], v[2], v[3]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t vv = vmask ? (v[j] & bmask) : v[j];
+            const uint32_t b01 = e4m3x2_to_f16x2(vv);
+            const uint32_t b23 = e4m3x2_to_f16x2(vv >> 16);
+            MMA::k16(o[4 * dq + j], h0, h1, h2, h3, b01, b23);
+            MMA::k16(o[4 * dq + j], e0, e1, e2, e3, b01, b23);
+          }
+        }
+      }
+    } else if constexpr (BS >= 16) {
 #pragma unroll
       for (int tp = 0; tp < BS / 16; ++tp) {
         const uint32_t h0 = PK::pack(sc[2 * tp][0], sc[2 * tp][1]);

@@ -60,7 +60,8 @@ struct DecodeArgs {
   int len_limit;    // largest valid context length
   int part_blocks;  // blocks per partition
   int max_parts;
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // softmax scale * log2(e) (times k_scale for 8-bit pools)
+  float out_scale;   // 1, or v_scale for 8-bit pools
 };
 
 // ---------------------------------------------------------------------------
@@ -96,7 +97,7 @@ __device__ __forceinline__ void store_unit_warp(const DecodeArgs &a, const float
     }
     const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
     if (nparts == 1) {
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const float inv = lsum > 0.f ? a.out_scale / lsum : 0.f;
       uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
 #pragma unroll
       for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
@@ -166,7 +167,7 @@ __device__ __forceinline__ void merge_partials_warp(const DecodeArgs &a, int s, 
         for (int j = 0; j < VPL; ++j) acc[j] += wu * v[u][j];
       }
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const float inv = L > 0.f ? a.out_scale / L : 0.f;
     uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
 #pragma unroll
     for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
@@ -184,6 +185,17 @@ __device__ __forceinline__ int clamp_len(const DecodeArgs &a, int s, bool report
 
 __device__ __forceinline__ int parts_of(int nb, int part_blocks) {
   return nb > part_blocks ? (nb + part_blocks - 1) / part_blocks : 1;
+}
+
+// Issue the TMA loads of one block of 8-bit pools (K tile of BS rows x D
+// codes, V tile of D rows x BS codes) into a stage.
+template <int D, int BS>
+__device__ __forceinline__ void load_block_fp8(uint32_t dst, const CUtensorMap *tmk,
+                                               const CUtensorMap *tmv, uint32_t bar, int g, int id,
+                                               uint64_t policy) {
+  mbar_arrive_expect_tx(bar, 2 * BS * D);
+  tma_load_4d(dst, tmk, bar, 0, 0, g, id, policy);
+  tma_load_4d(dst + BS * D, tmv, bar, 0, 0, g, id, policy);
 }
 
 // Issue the TMA loads of one block (K and V tiles) into a stage.
@@ -206,9 +218,9 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap *tmk,
 // ---------------------------------------------------------------------------
 
 // Launch shape: a CTA's rings take about 64 KB so three CTAs fit on an SM.
-template <int D, int BS>
+template <int D, int BS, int ESZ = 2>
 struct GridTune {
-  static constexpr int kStage = 2 * BS * D * 2;
+  static constexpr int kStage = 2 * BS * D * ESZ;
   static constexpr int kWarps = kStage >= 16384 ? 2 : 4;
   static constexpr int kFit = 65536 / (kWarps * kStage);
   static constexpr int kStages = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
@@ -220,13 +232,13 @@ struct GridTune {
   static constexpr int kSmem = kNvOff + kWarps * kStages * 4 + 1024;
 };
 
-template <typename T, int D, int BS, int WARPS, int NST, bool BIG>
+template <typename T, int D, int BS, int WARPS, int NST, bool BIG, bool KV8>
 __global__ void __launch_bounds__(WARPS * 32)
     paged_decode_grid_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
-  using TN = GridTune<D, BS>;
-  constexpr int kStageBytes = 2 * BS * D * 2;
-  using State = DecodeState<T, D, BS, BIG>;
+  using TN = GridTune<D, BS, KV8 ? 1 : 2>;
+  constexpr int kStageBytes = 2 * BS * D * (KV8 ? 1 : 2);
+  using State = DecodeState<T, D, BS, BIG, KV8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -287,7 +299,10 @@ __global__ void __launch_bounds__(WARPS * 32)
       if (static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks)) {
         stage_nv[st] = (blk == nb - 1) ? tail_nv : BS;
         fence_proxy_async_smem();
-        load_block<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar, g, id, policy);
+        if constexpr (KV8)
+          load_block_fp8<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar, g, id, policy);
+        else
+          load_block<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar, g, id, policy);
       } else {
         raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
         stage_nv[st] = 0;  // the whole block is masked
@@ -350,6 +365,7 @@ struct CombineArgs {
   int len_limit;
   int part_blocks;
   int max_parts;
+  float out_scale;
 };
 
 template <int NT>
@@ -404,7 +420,7 @@ __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
   }
   const float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   static_cast<T *>(c.out)[row * D + threadIdx.x] =
-      Pack<T>::from_float(lsum > 0.f ? total / lsum : 0.f);
+      Pack<T>::from_float(lsum > 0.f ? total * c.out_scale / lsum : 0.f);
 }
 
 // ---------------------------------------------------------------------------
@@ -462,11 +478,11 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int3
   return true;
 }
 
-template <typename T, int D, int BS, bool BIG>
+template <typename T, int D, int BS, bool BIG, bool KV8>
 pkv_status launch_grid(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
                        cudaStream_t stream) {
-  using TN = GridTune<D, BS>;
-  auto kern = paged_decode_grid_kernel<T, D, BS, TN::kWarps, TN::kStages, BIG>;
+  using TN = GridTune<D, BS, KV8 ? 1 : 2>;
+  auto kern = paged_decode_grid_kernel<T, D, BS, TN::kWarps, TN::kStages, BIG, KV8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TN::kSmem) !=
       cudaSuccess)
     return PKV_ERR_CUDA;
@@ -479,7 +495,24 @@ pkv_status launch_grid(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
 template <typename T, int D, int BS, bool BIG>
 pkv_status launch_decode(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
                          cudaStream_t stream) {
-  return launch_grid<T, D, BS, BIG>(tmk, tmv, args, stream);
+  return launch_grid<T, D, BS, BIG, false>(tmk, tmv, args, stream);
+}
+
+// 8-bit pools: head_dim 128, block_size 16, 32 or 64.
+template <typename T>
+pkv_status launch_decode_fp8(int block_size, bool big, const CUtensorMap &tmk,
+                             const CUtensorMap &tmv, const DecodeArgs &args, cudaStream_t stream) {
+#define PKV_BS8_CASE(BSV)                                                            \
+  case BSV:                                                                          \
+    return big ? launch_grid<T, 128, BSV, true, true>(tmk, tmv, args, stream)         \
+               : launch_grid<T, 128, BSV, false, true>(tmk, tmv, args, stream);
+  switch (block_size) {
+    PKV_BS8_CASE(16)
+    PKV_BS8_CASE(32)
+    PKV_BS8_CASE(64)
+  }
+#undef PKV_BS8_CASE
+  return PKV_ERR_BAD_SHAPE;
 }
 
 template <typename T, int D>
@@ -530,20 +563,31 @@ extern "C" int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t 
   return plan.part_blocks * block_size;
 }
 
-extern "C" pkv_status pkv_paged_attention_decode(
-    void *out, const void *query, const void *k_cache, const void *v_cache, pkv_cache_desc cache,
-    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
-    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
-    int32_t partition_size, void *workspace, size_t workspace_bytes, int32_t *d_status,
-    pkv_stream_t stream) {
-  using namespace pkv;
+namespace pkv {
+namespace {
+
+// Shared body of the decode entry points.  kv8: 8-bit pools with scales
+// k_scale / v_scale; act: dtype of query and out.
+pkv_status decode_impl(void *out, const void *query, pkv_dtype act, const void *k_cache,
+                       const void *v_cache, const pkv_cache_desc &cache, bool kv8,
+                       const int32_t *block_tables, int32_t max_blocks_per_seq,
+                       const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads,
+                       int32_t max_context_len, float scale, float k_scale, float v_scale,
+                       int32_t partition_size, void *workspace, size_t workspace_bytes,
+                       int32_t *d_status, pkv_stream_t stream) {
   pkv_status st = check_cache_desc(cache);
   if (st != PKV_OK) return st;
+  if (kv8 ? (cache.dtype != PKV_FP8_E4M3 || !is_16bit(act)) : !is_16bit(cache.dtype))
+    return PKV_ERR_BAD_DTYPE;
+  if (kv8 && (cache.head_dim != 128 || cache.block_size < 16)) return PKV_ERR_BAD_SHAPE;
   if (num_seqs < 0 || max_context_len < 0 || max_blocks_per_seq < 1 || num_q_heads < 1)
     return PKV_ERR_BAD_SHAPE;
   if (num_q_heads % cache.num_kv_heads != 0 || num_q_heads / cache.num_kv_heads > 16)
     return PKV_ERR_BAD_SHAPE;
   if (!(scale > 0.f) || !(scale < INFINITY)) return PKV_ERR_BAD_SHAPE;
+  if (kv8 && (!(k_scale > 0.f) || !(k_scale < INFINITY) || !(v_scale > 0.f) ||
+              !(v_scale < INFINITY)))
+    return PKV_ERR_BAD_SHAPE;
   if (partition_size < 0 || (partition_size > 0 && partition_size % cache.block_size != 0))
     return PKV_ERR_BAD_PARTITION;
   if (num_seqs == 0) return PKV_OK;
@@ -566,8 +610,13 @@ extern "C" pkv_status pkv_paged_attention_decode(
   if ((st = check_device()) != PKV_OK) return st;
 
   CUtensorMap tmk, tmv;
-  if ((st = encode_cache_map(&tmk, k_cache, cache)) != PKV_OK) return st;
-  if ((st = encode_cache_map(&tmv, v_cache, cache)) != PKV_OK) return st;
+  if (kv8) {
+    if ((st = encode_fp8_k_map(&tmk, k_cache, cache)) != PKV_OK) return st;
+    if ((st = encode_fp8_v_map(&tmv, v_cache, cache)) != PKV_OK) return st;
+  } else {
+    if ((st = encode_cache_map(&tmk, k_cache, cache)) != PKV_OK) return st;
+    if ((st = encode_cache_map(&tmv, v_cache, cache)) != PKV_OK) return st;
+  }
 
   DecodeArgs args{};
   args.query = query;
@@ -577,7 +626,7 @@ extern "C" pkv_status pkv_paged_attention_decode(
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   args.counters = reinterpret_cast<int32_t *>(ws);
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * plan.max_parts;
-  float *part = reinterpret_cast<float *>(ws + plan.ctrl_bytes);
+  float *part = plan.ws_bytes ? reinterpret_cast<float *>(ws + plan.ctrl_bytes) : nullptr;
   const bool split = plan.max_parts > 1;
   args.ws_o = split ? part : nullptr;
   args.ws_m = split ? part + rows * cache.head_dim : nullptr;
@@ -593,14 +642,18 @@ extern "C" pkv_status pkv_paged_attention_decode(
       max_context_len, static_cast<long long>(max_blocks_per_seq) * cache.block_size));
   args.part_blocks = plan.part_blocks;
   args.max_parts = plan.max_parts;
-  args.scale_log2 = scale * kLog2e;
+  args.scale_log2 = scale * kLog2e * (kv8 ? k_scale : 1.f);
+  args.out_scale = kv8 ? v_scale : 1.f;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (plan.ctrl_bytes > 0 && cudaMemsetAsync(ws, 0, plan.ctrl_bytes, s) != cudaSuccess)
     return PKV_ERR_CUDA;
   const bool big = args.group > 8;
-  const bool bf16 = cache.dtype == PKV_BF16;
-  if (cache.head_dim == 128)
+  const bool bf16 = act == PKV_BF16;
+  if (kv8)
+    st = bf16 ? launch_decode_fp8<__nv_bfloat16>(cache.block_size, big, tmk, tmv, args, s)
+              : launch_decode_fp8<__half>(cache.block_size, big, tmk, tmv, args, s);
+  else if (cache.head_dim == 128)
     st = bf16 ? launch_for_dim<__nv_bfloat16, 128>(cache.block_size, big, tmk, tmv, args, s)
               : launch_for_dim<__half, 128>(cache.block_size, big, tmk, tmv, args, s);
   else
@@ -619,9 +672,37 @@ extern "C" pkv_status pkv_paged_attention_decode(
   c.len_limit = args.len_limit;
   c.part_blocks = plan.part_blocks;
   c.max_parts = plan.max_parts;
+  c.out_scale = args.out_scale;
   if (cache.head_dim == 128)
     return bf16 ? launch_combine<__nv_bfloat16, 128>(c, num_seqs, s)
                 : launch_combine<__half, 128>(c, num_seqs, s);
   return bf16 ? launch_combine<__nv_bfloat16, 64>(c, num_seqs, s)
               : launch_combine<__half, 64>(c, num_seqs, s);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_attention_decode(
+    void *out, const void *query, const void *k_cache, const void *v_cache, pkv_cache_desc cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
+    int32_t partition_size, void *workspace, size_t workspace_bytes, int32_t *d_status,
+    pkv_stream_t stream) {
+  return pkv::decode_impl(out, query, cache.dtype, k_cache, v_cache, cache, false, block_tables,
+                          max_blocks_per_seq, context_lens, num_seqs, num_q_heads, max_context_len,
+                          scale, 1.f, 1.f, partition_size, workspace, workspace_bytes, d_status,
+                          stream);
+}
+
+extern "C" pkv_status pkv_paged_attention_decode_fp8(
+    void *out, const void *query, pkv_dtype query_dtype, const void *k_cache, const void *v_cache,
+    pkv_cache_desc cache, const int32_t *block_tables, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+    float scale, float k_scale, float v_scale, int32_t partition_size, void *workspace,
+    size_t workspace_bytes, int32_t *d_status, pkv_stream_t stream) {
+  return pkv::decode_impl(out, query, query_dtype, k_cache, v_cache, cache, true, block_tables,
+                          max_blocks_per_seq, context_lens, num_seqs, num_q_heads, max_context_len,
+                          scale, k_scale, v_scale, partition_size, workspace, workspace_bytes,
+                          d_status, stream);
 }

@@ -194,6 +194,19 @@ struct Pack<__nv_bfloat16> {
   }
 };
 
+// Two E4M3 codes (bits 0..7 and 8..15 of `pair`) to two fp16 values (exact).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
+  uint32_t out;
+  asm("{\n"
+      " .reg .b16 lo;\n"
+      " cvt.u16.u32 lo, %1;\n"
+      " cvt.rn.f16x2.e4m3x2 %0, lo;\n"
+      "}\n"
+      : "=r"(out)
+      : "r"(pair));
+  return out;
+}
+
 // 2^x with the hardware approximation (relative error about 2^-22).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

@@ -46,20 +46,51 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 }
 }  // namespace
 
-pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
+namespace {
+// Rank-4 tiled map; dims fastest first, element size esz bytes, box inner x
+// rows (the other two box extents 1).
+pkv_status encode_map(CUtensorMap *map, const void *pool, CUtensorMapDataType type, cuuint64_t esz,
+                      const cuuint64_t (&dims)[4], cuuint32_t box_inner, cuuint32_t box_rows,
+                      CUtensorMapSwizzle swizzle) {
   auto fn = encoder();
   if (fn == nullptr) return PKV_ERR_CUDA;
-  const cuuint64_t esz = 2;
-  cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
-                        static_cast<cuuint64_t>(c.num_kv_heads),
-                        static_cast<cuuint64_t>(c.num_blocks)};
-  cuuint64_t strides[3] = {dims[0] * esz, dims[0] * dims[1] * esz, dims[0] * dims[1] * dims[2] * esz};
-  cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(c.block_size), 1u, 1u};
+  cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t strides[3] = {d[0] * esz, d[0] * d[1] * esz, d[0] * d[1] * d[2] * esz};
+  cuuint32_t box[4] = {box_inner, box_rows, 1u, 1u};
   cuuint32_t estride[4] = {1u, 1u, 1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void *>(pool), dims, strides,
-                  box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, type, 4, const_cast<void *>(pool), d, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+}  // namespace
+
+pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
+                              static_cast<cuuint64_t>(c.num_kv_heads),
+                              static_cast<cuuint64_t>(c.num_blocks)};
+  return encode_map(map, pool, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, dims, 64u,
+                    static_cast<cuuint32_t>(c.block_size), CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+pkv_status encode_fp8_k_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
+                              static_cast<cuuint64_t>(c.num_kv_heads),
+                              static_cast<cuuint64_t>(c.num_blocks)};
+  return encode_map(map, pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dims,
+                    static_cast<cuuint32_t>(c.head_dim), static_cast<cuuint32_t>(c.block_size),
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+pkv_status encode_fp8_v_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.block_size), static_cast<cuuint64_t>(c.head_dim),
+                              static_cast<cuuint64_t>(c.num_kv_heads),
+                              static_cast<cuuint64_t>(c.num_blocks)};
+  const CUtensorMapSwizzle sw = c.block_size == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : c.block_size == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                     : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return encode_map(map, pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dims,
+                    static_cast<cuuint32_t>(c.block_size), static_cast<cuuint32_t>(c.head_dim), sw);
 }
 
 }  // namespace pkv
@@ -68,7 +99,7 @@ extern "C" const char *pkv_status_string(pkv_status s) {
   switch (s) {
     case PKV_OK: return "ok";
     case PKV_ERR_NULL_POINTER: return "a required pointer is NULL";
-    case PKV_ERR_BAD_DTYPE: return "dtype must be PKV_F16 or PKV_BF16";
+    case PKV_ERR_BAD_DTYPE: return "dtype not accepted here (fp16/bf16 pools, or PKV_FP8_E4M3 pools for the _fp8 calls)";
     case PKV_ERR_BAD_SHAPE: return "unsupported shape (head_dim 64/128, block_size 8/16/32/64, head counts)";
     case PKV_ERR_MISALIGNED: return "pointer or stride breaks the required alignment";
     case PKV_ERR_WORKSPACE: return "workspace missing or smaller than pkv_paged_attention_workspace_size";

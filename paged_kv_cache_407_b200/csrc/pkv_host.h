@@ -14,7 +14,11 @@ inline bool aligned(const void *p, size_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
 
-inline bool valid_dtype(pkv_dtype t) { return t == PKV_F16 || t == PKV_BF16; }
+inline bool valid_dtype(pkv_dtype t) { return t == PKV_F16 || t == PKV_BF16 || t == PKV_FP8_E4M3; }
+
+inline bool is_16bit(pkv_dtype t) { return t == PKV_F16 || t == PKV_BF16; }
+
+inline int elem_bytes(pkv_dtype t) { return t == PKV_FP8_E4M3 ? 1 : 2; }
 
 // Checks shared by every call that takes a cache descriptor.
 pkv_status check_cache_desc(const pkv_cache_desc &c);
@@ -22,9 +26,14 @@ pkv_status check_cache_desc(const pkv_cache_desc &c);
 // PKV_ERR_DEVICE unless the current device is compute capability 10.0.
 pkv_status check_device();
 
-// Encode a rank-4 tiled tensor map over one cache pool viewed as
+// Encode a rank-4 tiled tensor map over one fp16/bf16 cache pool viewed as
 // [N][Hkv][B][D] (fastest last), box = 64 elements x B rows, 128-byte swizzle.
 pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
+
+// 8-bit pools: K as [N][Hkv][B][D] bytes, box D x B, 128-byte swizzle (D = 128);
+// V as [N][Hkv][D][B] bytes, box B x D, swizzle span B bytes (none at B = 16).
+pkv_status encode_fp8_k_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
+pkv_status encode_fp8_v_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
 
 inline pkv_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;

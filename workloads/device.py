@@ -56,3 +56,34 @@ def upload(b: PagedBatch, device="cuda") -> DeviceBatch:
                                  else torch.from_numpy(b.block_tables_before_cow).to(device)),
         out=torch.empty_like(q),
     )
+
+
+@dataclass
+class DeviceFp8Batch:
+    q: torch.Tensor
+    k_cache: torch.Tensor  # uint8 [N, Hkv, B, D]
+    v_cache: torch.Tensor  # uint8 [N, Hkv, D, B]
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+    key: torch.Tensor
+    value: torch.Tensor
+    slot_mapping: torch.Tensor
+    cow_pairs: torch.Tensor
+    out: torch.Tensor
+
+
+def upload_fp8(f8, device="cuda") -> DeviceFp8Batch:
+    b = f8.base
+    q = bits_to_tensor(b.q, b.dtype, device)
+    return DeviceFp8Batch(
+        q=q,
+        k_cache=torch.from_numpy(f8.k_cache).to(device),
+        v_cache=torch.from_numpy(f8.v_cache).to(device),
+        block_tables=torch.from_numpy(b.block_tables).to(device),
+        context_lens=torch.from_numpy(b.context_lens).to(device),
+        key=bits_to_tensor(b.key, b.dtype, device),
+        value=bits_to_tensor(b.value, b.dtype, device),
+        slot_mapping=torch.from_numpy(b.slot_mapping).to(device),
+        cow_pairs=torch.from_numpy(np.ascontiguousarray(b.cow_pairs)).to(device),
+        out=torch.empty_like(q),
+    )
