@@ -39,7 +39,8 @@ import numpy as np  # noqa: E402
 METRIC = "paged decode attention KV GB/s and tokens/s on 1 B200; % of HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/paged_attention.cu",
+KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/pkv_host.cu",
+                  "paged_kv_cache_407_b200/csrc/paged_attention.cu",
                   "paged_kv_cache_407_b200/csrc/decode_core.cuh",
                   "paged_kv_cache_407_b200/csrc/pkv_device.cuh"]
 
@@ -51,6 +52,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="llama7b_mha")
+    p.add_argument("--kv-dtype", choices=["auto", "e4m3"], default="auto",
+                   help="auto: the workload's fp16/bf16 pools; e4m3: 8-bit pools (quantising write)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
@@ -75,10 +78,11 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kv_dtype: str = "f16"):
     """DRAM bytes per launch of the attention kernel from the committed ncu
     summary, if it was taken on the current kernel source; else None."""
-    path = os.path.join(PROFILE_DIR, f"paged_decode_kernel_{workload}.txt")
+    suffix = "_e4m3" if kv_dtype == "e4m3" else ""
+    path = os.path.join(PROFILE_DIR, f"paged_decode_kernel{suffix}_{workload}.txt")
     try:
         kv = {}
         with open(path, encoding="utf-8") as f:
@@ -176,13 +180,15 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- helpers
-def step_bytes(batch):
+def step_bytes(batch, kv_bytes=2):
     from paged_kv_cache_407_b200 import accounting as A
 
     att = A.decode_bytes(batch.context_lens, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
-                         batch.block_size)
-    write = A.reshape_and_cache_bytes(batch.num_tokens, batch.num_kv_heads, batch.head_dim)
-    copy = A.copy_blocks_bytes(batch.cow_pairs.shape[0], batch.num_kv_heads, batch.block_size, batch.head_dim)
+                         batch.block_size, kv_elem_bytes=kv_bytes)
+    write = A.reshape_and_cache_bytes(batch.num_tokens, batch.num_kv_heads, batch.head_dim,
+                                      cache_elem_bytes=kv_bytes)
+    copy = A.copy_blocks_bytes(batch.cow_pairs.shape[0], batch.num_kv_heads, batch.block_size, batch.head_dim,
+                               elem_bytes=kv_bytes)
     return att, write, copy
 
 
@@ -196,9 +202,10 @@ def blas_threads():
         return 1
 
 
-def oracle_sample_rate(batch, seconds: float):
-    """Time the oracle's decode over whole sequences of the batch until about
-    ``seconds`` of CPU work; returns (GB/s, description, cores)."""
+def oracle_sample_rate(batch, seconds: float, f8=None):
+    """Time the oracle's decode over whole sequences of the batch (of its 8-bit
+    variant ``f8`` when given) until about ``seconds`` of CPU work; returns
+    (GB/s, description, cores, seconds)."""
     import oracle as O
     from paged_kv_cache_407_b200 import accounting as A
 
@@ -206,12 +213,17 @@ def oracle_sample_rate(batch, seconds: float):
     done, t0 = [], time.perf_counter()
     while len(done) < len(order) and time.perf_counter() - t0 < seconds:
         s = int(order[len(done)])
-        O.decode_sequence(batch.q[s], batch.k_cache, batch.v_cache, batch.block_tables[s],
-                          int(batch.context_lens[s]), batch.block_size, batch.scale, batch.dtype)
+        if f8 is None:
+            O.decode_sequence(batch.q[s], batch.k_cache, batch.v_cache, batch.block_tables[s],
+                              int(batch.context_lens[s]), batch.block_size, batch.scale, batch.dtype)
+        else:
+            O.paged_attention_decode_fp8(batch.q, f8.k_cache, f8.v_cache, batch.block_tables, batch.context_lens,
+                                         batch.block_size, batch.scale, f8.k_scale, f8.v_scale, batch.dtype,
+                                         seqs=[s])
         done.append(s)
     dt = time.perf_counter() - t0
     b = A.decode_bytes(batch.context_lens[done], batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
-                       batch.block_size)["total"]
+                       batch.block_size, kv_elem_bytes=1 if f8 is not None else 2)["total"]
     desc = (f"oracle decode (fp64 NumPy) of {len(done)} of {batch.num_seqs} sequences of the "
             f"{batch.name} batch ({int(batch.context_lens[done].sum())} tokens), {dt:.1f} s")
     return b / dt / 1e9, desc, blas_threads(), dt
@@ -319,7 +331,16 @@ def run_ours(args):
     pkv.library()
 
     batch = build_workload(args.workload, rank)
-    db = upload(batch, dev)
+    e4m3 = args.kv_dtype == "e4m3"
+    f8 = None
+    if e4m3:
+        import workloads as W
+        from workloads.device import upload_fp8
+
+        f8 = W.fp8_variant(batch, 777 + rank)
+        db = upload_fp8(f8, dev)
+    else:
+        db = upload(batch, dev)
     ws_bytes = pkv.workspace_size(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
                                   batch.block_size, batch.max_context_len, batch.partition_size)
     workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
@@ -328,19 +349,33 @@ def run_ours(args):
     P = pkv.partition_size(batch.num_seqs, batch.num_kv_heads, batch.block_size, batch.max_context_len,
                            batch.partition_size)
     split = batch.max_context_len > P
+    nb_max = -(-batch.max_context_len // batch.block_size)
+    max_parts = -(-nb_max // (P // batch.block_size))
     has_cow = batch.cow_pairs.shape[0] > 0
-    launches_per_step = 1 + 1 + (1 if split else 0) + (1 if has_cow else 0)
+    # cache write + attention kernel (+ merge kernel for splits of more than
+    # 32 partitions) (+ block copy)
+    launches_per_step = 2 + (1 if max_parts > 32 else 0) + (1 if has_cow else 0)
 
     def step(q=db.q, out=db.out, key=db.key, value=db.value, slots=db.slot_mapping, tables=db.block_tables,
              lens=db.context_lens, ev=None):
         if has_cow:
             pkv.copy_blocks(db.k_cache, db.v_cache, db.cow_pairs, d_status=status, stream=stream)
-        pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=status, stream=stream)
+        if e4m3:
+            pkv.reshape_and_cache_fp8(key, value, db.k_cache, db.v_cache, slots, f8.k_scale, f8.v_scale,
+                                      d_status=status, stream=stream)
+        else:
+            pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=status, stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, batch.max_context_len,
-                                   batch.scale, partition_size=batch.partition_size, workspace=workspace,
-                                   d_status=status, stream=stream)
+        if e4m3:
+            pkv.paged_attention_decode_fp8(out, q, db.k_cache, db.v_cache, tables, lens, batch.max_context_len,
+                                           batch.scale, f8.k_scale, f8.v_scale,
+                                           partition_size=batch.partition_size, workspace=workspace,
+                                           d_status=status, stream=stream)
+        else:
+            pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, batch.max_context_len,
+                                       batch.scale, partition_size=batch.partition_size, workspace=workspace,
+                                       d_status=status, stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -434,7 +469,7 @@ def run_ours(args):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
 
-    att_bytes, write_bytes, copy_bytes = step_bytes(batch)
+    att_bytes, write_bytes, copy_bytes = step_bytes(batch, kv_bytes=1 if e4m3 else 2)
     att_ms_mean = float(np.mean(att_ms))
     (ms_total, att_ms_max, e2e_ms), (bytes_all, seqs_all) = reduce_across_ranks(
         [ms_total, att_ms_mean, e2e["ms"] if e2e else 0.0], [att_bytes["total"], batch.num_seqs], dev)
@@ -442,7 +477,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, cores, _ = oracle_sample_rate(batch, args.cpu_seconds)
+        rate, desc, cores, _ = oracle_sample_rate(batch, args.cpu_seconds, f8=f8)
         cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if world > 1:
@@ -455,7 +490,11 @@ def run_ours(args):
     total_att_bytes = bytes_all  # every rank's own batch, summed
     value = total_att_bytes / (ms_step * 1e-3) / 1e9
     achieved = att_bytes["total"] / (att_ms_max * 1e-3) / 1e9
-    traffic = profiled_traffic(batch.name)
+    traffic = profiled_traffic(batch.name, "e4m3" if e4m3 else "f16")
+    config = workload_config(batch, args, world)
+    config["kv_cache_dtype"] = "e4m3 (8-bit pools, fp16 MMA operands)" if e4m3 else batch.dtype
+    if e4m3:
+        config["pool_bytes"] = int(f8.k_cache.nbytes + f8.v_cache.nbytes)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -467,9 +506,9 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": batch.dtype,
+        "dtype": "f16" if e4m3 else batch.dtype,
         "data": "synthetic (seeded generator, inputs resident in HBM)",
-        "config": workload_config(batch, args, world),
+        "config": config,
         "decode_tokens_per_s": round(seqs_all / (ms_step * 1e-3), 1),
         "decode_tokens_per_s_32_layer_attention_only": round(seqs_all / (ms_step * 1e-3) / 32, 1),
         "bytes_per_step": {"attention": att_bytes["total"], "attention_kv": att_bytes["kv"],

@@ -9,8 +9,9 @@
 //   S^T = Q K^T on mma.sync with the query heads on M, scale and mask,
 //   online softmax update, O = O * 2^(m_old - m_new) + P V.
 // The score accumulator fragment is, element for element, the A fragment of
-// P V, so P never moves between lanes.  P enters the second MMA as a 16-bit
-// high part plus a 16-bit residual, which keeps it at about fp32 precision.
+// P V, so P never moves between lanes.  With bf16 operands P enters the second
+// MMA as a bf16 high part plus a bf16 residual (bf16 alone would round P by up
+// to 2^-8 relative); with fp16 operands one fp16 P (at most 2^-11) is enough.
 //
 // 8-bit pools (KV8): K tiles hold one 128-byte row of E4M3 codes per token, V
 // tiles one row of BS codes per dimension (V stored transposed).  ldmatrix on
@@ -20,7 +21,11 @@
 // 8-token column tile 2t+u are tokens {0,1,4,5,8,9,12,13} + 2u of the 16-token
 // group t, so a lane's scores are tokens 4c..4c+3 of the group (c = lane % 4);
 // the head-dimension order inside each 16-wide step is permuted the same way
-// for Q and K.  Operands are fp16 (E4M3 codes are exact in fp16).
+// for Q and K.  Operands are fp16 (E4M3 codes are exact in fp16).  The K tile
+// arrives with those eight tokens on consecutive shared-memory rows
+// (row 8t + i of tile half u = token 16t + 4(i/2) + i%2 + 2u), and the V tile
+// as rows of 128 bytes, so both ldmatrix patterns are free of bank conflicts
+// under the 128-byte swizzle.
 #pragma once
 
 #include <type_traits>
@@ -40,13 +45,12 @@ __device__ __forceinline__ uint32_t tile_off(int tok, int chunk) {
                                (((chunk & 7) ^ (tok & 7)) << 4));
 }
 
-// Byte offset of 16-byte chunk `chunk` of row `row` in an 8-bit V tile whose
-// rows are BS bytes, written by TMA with a BS-byte swizzle span (none at 16).
+// Byte offset of 16-byte chunk `chunk` of dimension row `row` (BS bytes) in an
+// 8-bit V tile moved as 128-byte rows with the 128-byte swizzle.
 template <int BS>
 __device__ __forceinline__ uint32_t v8_off(int row, int chunk) {
-  if constexpr (BS == 16) return static_cast<uint32_t>(row * 16);
-  if constexpr (BS == 32) return static_cast<uint32_t>(row * 32 + ((chunk ^ ((row >> 2) & 1)) << 4));
-  return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+  const uint32_t b = static_cast<uint32_t>(row * BS + chunk * 16);
+  return (b & ~127u) | ((((b >> 4) ^ (b >> 7)) & 7u) << 4);
 }
 
 template <typename T, int D, int BS, bool BIG, bool KV8 = false>
@@ -57,6 +61,7 @@ struct DecodeState {
   using OP = typename std::conditional<KV8, __half, T>::type;  // MMA operand type
   using MMA = Mma<OP>;
   using PK = Pack<OP>;
+  static constexpr bool kSplitP = std::is_same<OP, __nv_bfloat16>::value;
 
   uint32_t qa0[kKS], qa1[kKS], qa2[kKS], qa3[kKS];  // Q as A fragments (rows r, r + 8)
   float m0, m1, l0, l1;                             // running max / sum, rows r and r + 8
@@ -136,24 +141,24 @@ struct DecodeState {
     for (int nt = 0; nt < kNT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
     if constexpr (KV8) {
       // matrices: 0 = tile 2tp, step 2kk2; 1 = tile 2tp+1, step 2kk2; 2, 3 = step 2kk2+1
-      const int perm = (ri >> 1) * 4 + (ri & 1) + ((mi & 1) << 1);
 #pragma unroll
       for (int kk2 = 0; kk2 < kKS / 2; ++kk2) {
 #pragma unroll
         for (int tp = 0; tp < BS / 16; ++tp) {
           uint32_t r0, r1, r2, r3;
-          const int tok = tp * 16 + perm;
+          const int row = (mi & 1) * (BS / 2) + tp * 8 + ri;
           const int chunk = 2 * kk2 + (mi >> 1);
-          ldsm_x4(kb + tok * 128 + (((chunk ^ (tok & 7)) & 7) << 4), r0, r1, r2, r3);
+          ldsm_x4(kb + row * 128 + ((chunk ^ ri) << 4), r0, r1, r2, r3);
           const int k0 = 2 * kk2, k1 = 2 * kk2 + 1;
-          MMA::k16(sc[2 * tp], qa0[k0], qa1[k0], qa2[k0], qa3[k0], e4m3x2_to_f16x2(r0),
-                   e4m3x2_to_f16x2(r0 >> 16));
-          MMA::k16(sc[2 * tp + 1], qa0[k0], qa1[k0], qa2[k0], qa3[k0], e4m3x2_to_f16x2(r1),
-                   e4m3x2_to_f16x2(r1 >> 16));
-          MMA::k16(sc[2 * tp], qa0[k1], qa1[k1], qa2[k1], qa3[k1], e4m3x2_to_f16x2(r2),
-                   e4m3x2_to_f16x2(r2 >> 16));
-          MMA::k16(sc[2 * tp + 1], qa0[k1], qa1[k1], qa2[k1], qa3[k1], e4m3x2_to_f16x2(r3),
-                   e4m3x2_to_f16x2(r3 >> 16));
+          uint32_t f0, f1;
+          e4m3x4_to_f16x2x2(r0, f0, f1);
+          MMA::k16(sc[2 * tp], qa0[k0], qa1[k0], qa2[k0], qa3[k0], f0, f1);
+          e4m3x4_to_f16x2x2(r1, f0, f1);
+          MMA::k16(sc[2 * tp + 1], qa0[k0], qa1[k0], qa2[k0], qa3[k0], f0, f1);
+          e4m3x4_to_f16x2x2(r2, f0, f1);
+          MMA::k16(sc[2 * tp], qa0[k1], qa1[k1], qa2[k1], qa3[k1], f0, f1);
+          e4m3x4_to_f16x2x2(r3, f0, f1);
+          MMA::k16(sc[2 * tp + 1], qa0[k1], qa1[k1], qa2[k1], qa3[k1], f0, f1);
         }
       }
     } else if constexpr (BS >= 16) {
@@ -248,18 +253,10 @@ struct DecodeState {
         // 4c+2, 4c+3 (k-slots 2c+8, 2c+9)
         const uint32_t h0 = PK::pack(sc[2 * tp][0], sc[2 * tp][1]);
         const uint32_t h2 = PK::pack(sc[2 * tp + 1][0], sc[2 * tp + 1][1]);
-        const float2 f0 = PK::unpack(h0);
-        const float2 f2 = PK::unpack(h2);
-        const uint32_t e0 = PK::pack(sc[2 * tp][0] - f0.x, sc[2 * tp][1] - f0.y);
-        const uint32_t e2 = PK::pack(sc[2 * tp + 1][0] - f2.x, sc[2 * tp + 1][1] - f2.y);
-        uint32_t h1 = 0u, h3 = 0u, e1 = 0u, e3 = 0u;
+        uint32_t h1 = 0u, h3 = 0u;
         if constexpr (BIG) {
           h1 = PK::pack(sc[2 * tp][2], sc[2 * tp][3]);
           h3 = PK::pack(sc[2 * tp + 1][2], sc[2 * tp + 1][3]);
-          const float2 f1 = PK::unpack(h1);
-          const float2 f3 = PK::unpack(h3);
-          e1 = PK::pack(sc[2 * tp][2] - f1.x, sc[2 * tp][3] - f1.y);
-          e3 = PK::pack(sc[2 * tp + 1][2] - f3.x, sc[2 * tp + 1][3] - f3.y);
         }
         const int t0 = tp * 16 + 2 * c2;  // first of this lane's four tokens
         const bool vmask = partial && (tp * 16 + 16 > nv);
@@ -271,11 +268,9 @@ struct DecodeState {
           ldsm_x4(vb + v8_off<BS>(32 * dq + 8 * mi + ri, tp), v[0], v[1], v[2], v[3]);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint32_t vv = vmask ? (v[j] & bmask) : v[j];
-            const uint32_t b01 = e4m3x2_to_f16x2(vv);
-            const uint32_t b23 = e4m3x2_to_f16x2(vv >> 16);
+            uint32_t b01, b23;
+            e4m3x4_to_f16x2x2(vmask ? (v[j] & bmask) : v[j], b01, b23);
             MMA::k16(o[4 * dq + j], h0, h1, h2, h3, b01, b23);
-            MMA::k16(o[4 * dq + j], e0, e1, e2, e3, b01, b23);
           }
         }
       }
@@ -284,18 +279,22 @@ struct DecodeState {
       for (int tp = 0; tp < BS / 16; ++tp) {
         const uint32_t h0 = PK::pack(sc[2 * tp][0], sc[2 * tp][1]);
         const uint32_t h2 = PK::pack(sc[2 * tp + 1][0], sc[2 * tp + 1][1]);
-        const float2 f0 = PK::unpack(h0);
-        const float2 f2 = PK::unpack(h2);
-        const uint32_t e0 = PK::pack(sc[2 * tp][0] - f0.x, sc[2 * tp][1] - f0.y);
-        const uint32_t e2 = PK::pack(sc[2 * tp + 1][0] - f2.x, sc[2 * tp + 1][1] - f2.y);
-        uint32_t h1 = 0u, h3 = 0u, e1 = 0u, e3 = 0u;
+        uint32_t h1 = 0u, h3 = 0u, e0 = 0u, e1 = 0u, e2 = 0u, e3 = 0u;
         if constexpr (BIG) {
           h1 = PK::pack(sc[2 * tp][2], sc[2 * tp][3]);
           h3 = PK::pack(sc[2 * tp + 1][2], sc[2 * tp + 1][3]);
-          const float2 f1 = PK::unpack(h1);
-          const float2 f3 = PK::unpack(h3);
-          e1 = PK::pack(sc[2 * tp][2] - f1.x, sc[2 * tp][3] - f1.y);
-          e3 = PK::pack(sc[2 * tp + 1][2] - f3.x, sc[2 * tp + 1][3] - f3.y);
+        }
+        if constexpr (kSplitP) {
+          const float2 f0 = PK::unpack(h0);
+          const float2 f2 = PK::unpack(h2);
+          e0 = PK::pack(sc[2 * tp][0] - f0.x, sc[2 * tp][1] - f0.y);
+          e2 = PK::pack(sc[2 * tp + 1][0] - f2.x, sc[2 * tp + 1][1] - f2.y);
+          if constexpr (BIG) {
+            const float2 f1 = PK::unpack(h1);
+            const float2 f3 = PK::unpack(h3);
+            e1 = PK::pack(sc[2 * tp][2] - f1.x, sc[2 * tp][3] - f1.y);
+            e3 = PK::pack(sc[2 * tp + 1][2] - f3.x, sc[2 * tp + 1][3] - f3.y);
+          }
         }
         const bool vmask = partial && (tp * 16 + 16 > nv);
         const int t0 = tp * 16 + c2;
@@ -313,20 +312,24 @@ struct DecodeState {
             v3 &= mhi;
           }
           MMA::k16(o[2 * dp], h0, h1, h2, h3, v0, v1);
-          MMA::k16(o[2 * dp], e0, e1, e2, e3, v0, v1);
           MMA::k16(o[2 * dp + 1], h0, h1, h2, h3, v2, v3);
-          MMA::k16(o[2 * dp + 1], e0, e1, e2, e3, v2, v3);
+          if constexpr (kSplitP) {
+            MMA::k16(o[2 * dp], e0, e1, e2, e3, v0, v1);
+            MMA::k16(o[2 * dp + 1], e0, e1, e2, e3, v2, v3);
+          }
         }
       }
     } else {
       const uint32_t h0 = PK::pack(sc[0][0], sc[0][1]);
-      const float2 f0 = PK::unpack(h0);
-      const uint32_t e0 = PK::pack(sc[0][0] - f0.x, sc[0][1] - f0.y);
-      uint32_t h1 = 0u, e1 = 0u;
-      if constexpr (BIG) {
-        h1 = PK::pack(sc[0][2], sc[0][3]);
-        const float2 f1 = PK::unpack(h1);
-        e1 = PK::pack(sc[0][2] - f1.x, sc[0][3] - f1.y);
+      uint32_t h1 = 0u, e0 = 0u, e1 = 0u;
+      if constexpr (BIG) h1 = PK::pack(sc[0][2], sc[0][3]);
+      if constexpr (kSplitP) {
+        const float2 f0 = PK::unpack(h0);
+        e0 = PK::pack(sc[0][0] - f0.x, sc[0][1] - f0.y);
+        if constexpr (BIG) {
+          const float2 f1 = PK::unpack(h1);
+          e1 = PK::pack(sc[0][2] - f1.x, sc[0][3] - f1.y);
+        }
       }
       const uint32_t mlo = (c2 < nv ? 0x0000ffffu : 0u) | (c2 + 1 < nv ? 0xffff0000u : 0u);
 #pragma unroll
@@ -337,7 +340,7 @@ struct DecodeState {
         for (int j = 0; j < 4; ++j) {
           if (partial) v[j] &= mlo;
           MMA::k8(o[4 * dq + j], h0, h1, v[j]);
-          MMA::k8(o[4 * dq + j], e0, e1, v[j]);
+          if constexpr (kSplitP) MMA::k8(o[4 * dq + j], e0, e1, v[j]);
         }
       }
     }

@@ -131,7 +131,8 @@ __device__ __forceinline__ bool arrive_partition(const DecodeArgs &a, int s, int
 // Merge the nparts (<= 32) partials of (s, g) from the workspace into the
 // output, one warp, rows h = h0, h0 + hstep, ...: lane p reads partition p's
 // (m, l); the maximum and the weighted sum are warp reductions; the partial
-// outputs are read eight partitions at a time so their loads overlap.
+// outputs are read eight partitions at a time so their loads overlap, the
+// first eight together with (m, l).
 template <typename T, int D>
 __device__ __forceinline__ void merge_partials_warp(const DecodeArgs &a, int s, int g, int nparts,
                                                     int h0, int hstep, int lane) {
@@ -140,6 +141,14 @@ __device__ __forceinline__ void merge_partials_warp(const DecodeArgs &a, int s, 
   for (int h = h0; h < G; h += hstep) {
     const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
     const size_t base = row * a.max_parts;
+    const float *o = a.ws_o + base * D + lane * VPL;
+    // the first eight partial outputs are requested together with (m, l)
+    float v[8][VPL];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int j = 0; j < VPL; ++j)
+        v[u][j] = u < nparts ? __ldcg(o + static_cast<size_t>(u) * D + j) : 0.f;
     const float mp = lane < nparts ? __ldcg(a.ws_m + base + lane) : -INFINITY;
     const float lp = lane < nparts ? __ldcg(a.ws_l + base + lane) : 0.f;
     float M = mp;
@@ -152,14 +161,14 @@ __device__ __forceinline__ void merge_partials_warp(const DecodeArgs &a, int s, 
     float acc[VPL];
 #pragma unroll
     for (int j = 0; j < VPL; ++j) acc[j] = 0.f;
-    const float *o = a.ws_o + base * D + lane * VPL;
     for (int p0 = 0; p0 < nparts; p0 += 8) {
-      float v[8][VPL];
+      if (p0 > 0) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 8; ++u)
 #pragma unroll
-        for (int j = 0; j < VPL; ++j)
-          v[u][j] = p0 + u < nparts ? __ldcg(o + static_cast<size_t>(p0 + u) * D + j) : 0.f;
+          for (int j = 0; j < VPL; ++j)
+            v[u][j] = p0 + u < nparts ? __ldcg(o + static_cast<size_t>(p0 + u) * D + j) : 0.f;
+      }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const float wu = __shfl_sync(kFullMask, w, (p0 + u) & 31);
@@ -188,14 +197,14 @@ __device__ __forceinline__ int parts_of(int nb, int part_blocks) {
 }
 
 // Issue the TMA loads of one block of 8-bit pools (K tile of BS rows x D
-// codes, V tile of D rows x BS codes) into a stage.
+// codes, V tile of D rows x BS codes) into a stage; tile = block * Hkv + head.
 template <int D, int BS>
 __device__ __forceinline__ void load_block_fp8(uint32_t dst, const CUtensorMap *tmk,
-                                               const CUtensorMap *tmv, uint32_t bar, int g, int id,
+                                               const CUtensorMap *tmv, uint32_t bar, int tile,
                                                uint64_t policy) {
   mbar_arrive_expect_tx(bar, 2 * BS * D);
-  tma_load_4d(dst, tmk, bar, 0, 0, g, id, policy);
-  tma_load_4d(dst + BS * D, tmv, bar, 0, 0, g, id, policy);
+  tma_load_5d(dst, tmk, bar, 0, 0, 0, 0, tile, policy);
+  tma_load_3d(dst + BS * D, tmv, bar, 0, 0, tile, policy);
 }
 
 // Issue the TMA loads of one block (K and V tiles) into a stage.
@@ -224,6 +233,9 @@ struct GridTune {
   static constexpr int kWarps = kStage >= 16384 ? 2 : 4;
   static constexpr int kFit = 65536 / (kWarps * kStage);
   static constexpr int kStages = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
+  // Three CTAs per SM fit in shared memory; ask the register allocation for
+  // three as well (at most 168 registers with four warps).
+  static constexpr int kMinBlocks = 3;
   static constexpr int kRing = kWarps * kStages * kStage;
   static constexpr int kMerge = kWarps * 16 * (D + 2) * 4;
   static constexpr int kData = kRing > kMerge ? kRing : kMerge;
@@ -233,7 +245,7 @@ struct GridTune {
 };
 
 template <typename T, int D, int BS, int WARPS, int NST, bool BIG, bool KV8>
-__global__ void __launch_bounds__(WARPS * 32)
+__global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMinBlocks))
     paged_decode_grid_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
   using TN = GridTune<D, BS, KV8 ? 1 : 2>;
@@ -249,11 +261,24 @@ __global__ void __launch_bounds__(WARPS * 32)
   const int lane = threadIdx.x & 31;
   const int G = a.group;
 
+  // The length, the query rows and the first Block Table window are loaded
+  // together: none of them waits for another.
+  const int b0 = part * a.part_blocks;
+  const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + b0 + warp;
+  const int table_left = a.max_blocks_per_seq - b0 - warp;  // table entries from trow on
+  auto load_window = [&](int w) -> int {
+    const int k = (w << 5) + lane;
+    return k * WARPS < table_left ? __ldg(trow + static_cast<size_t>(k) * WARPS) : 0;
+  };
+  int win_cur = load_window(0);
+  State st_;
+  st_.load_q(static_cast<const T *>(a.query) +
+                 (static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G) * D,
+             G, lane);
   const int len = clamp_len(a, s, g == 0 && part == 0 && threadIdx.x == 0);
   const int nb = (len + BS - 1) / BS;
   const int nparts = parts_of(nb, a.part_blocks);
   if (part >= nparts) return;  // uniform over the CTA, before any barrier
-  const int b0 = part * a.part_blocks;
   const int nblk = min(nb - b0, a.part_blocks);
   const int tail_nv = len - (nb - 1) * BS;
   const int cnt = nblk > warp ? (nblk - warp + WARPS - 1) / WARPS : 0;
@@ -269,20 +294,7 @@ __global__ void __launch_bounds__(WARPS * 32)
     prefetch_tensormap(&tm_v);
   }
   __syncwarp();
-
-  State st_;
-  st_.load_q(static_cast<const T *>(a.query) +
-                 (static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G) * D,
-             G, lane);
   st_.reset();
-
-  // Block Table window: lane j holds the id of this warp's block 32*w + j.
-  const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + b0 + warp;
-  auto load_window = [&](int w) -> int {
-    const int k = (w << 5) + lane;
-    return k < cnt ? __ldg(trow + static_cast<size_t>(k) * WARPS) : 0;
-  };
-  int win_cur = load_window(0);
   int win_next = cnt > 32 ? load_window(1) : 0;
 
   const uint64_t policy = l2_evict_first_policy();
@@ -300,7 +312,8 @@ __global__ void __launch_bounds__(WARPS * 32)
         stage_nv[st] = (blk == nb - 1) ? tail_nv : BS;
         fence_proxy_async_smem();
         if constexpr (KV8)
-          load_block_fp8<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar, g, id, policy);
+          load_block_fp8<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar,
+                                id * a.num_kv_heads + g, policy);
         else
           load_block<D, BS>(ring + st * kStageBytes, &tm_k, &tm_v, bar, g, id, policy);
       } else {

@@ -105,6 +105,27 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// Rank-3 and rank-5 forms of the same load.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(bar), "l"(policy)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- ldmatrix
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                         uint32_t &r3) {
@@ -194,17 +215,16 @@ struct Pack<__nv_bfloat16> {
   }
 };
 
-// Two E4M3 codes (bits 0..7 and 8..15 of `pair`) to two fp16 values (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
-  uint32_t out;
+// Four E4M3 codes of `quad` to two fp16 pairs: bytes 0, 1 -> lo, bytes 2, 3 -> hi.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t quad, uint32_t &lo, uint32_t &hi) {
   asm("{\n"
-      " .reg .b16 lo;\n"
-      " cvt.u16.u32 lo, %1;\n"
-      " cvt.rn.f16x2.e4m3x2 %0, lo;\n"
+      " .reg .b16 a, b;\n"
+      " mov.b32 {a, b}, %2;\n"
+      " cvt.rn.f16x2.e4m3x2 %0, a;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, b;\n"
       "}\n"
-      : "=r"(out)
-      : "r"(pair));
-  return out;
+      : "=r"(lo), "=r"(hi)
+      : "r"(quad));
 }
 
 // 2^x with the hardware approximation (relative error about 2^-22).

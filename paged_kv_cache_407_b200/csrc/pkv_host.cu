@@ -73,24 +73,47 @@ pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_
                     static_cast<cuuint32_t>(c.block_size), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+namespace {
+// Byte map of `rank` dims (fastest first) with explicit byte strides of dims
+// 1.. and a full box, 128-byte swizzle.
+pkv_status encode_bytes(CUtensorMap *map, const void *pool, cuuint32_t rank, const cuuint64_t *dims,
+                        const cuuint64_t *strides, const cuuint32_t *box) {
+  auto fn = encoder();
+  if (fn == nullptr) return PKV_ERR_CUDA;
+  const cuuint32_t estride[5] = {1u, 1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(pool),
+                  const_cast<cuuint64_t *>(dims), const_cast<cuuint64_t *>(strides),
+                  const_cast<cuuint32_t *>(box), estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+}  // namespace
+
+// The K tile of (block, kv head) is B rows of D codes.  Token t = b + 2 a + 4 c
+// (b, a in {0, 1}) is addressed through dims (d, b, c, a, block*Hkv + head),
+// so the box lands in shared memory with token t on row b + 2 c + (B/2) a:
+// the eight tokens {0,1,4,5,8,9,12,13} + 2a + 16 j of one score column tile
+// sit on eight consecutive rows.
 pkv_status encode_fp8_k_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
-                              static_cast<cuuint64_t>(c.num_kv_heads),
-                              static_cast<cuuint64_t>(c.num_blocks)};
-  return encode_map(map, pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dims,
-                    static_cast<cuuint32_t>(c.head_dim), static_cast<cuuint32_t>(c.block_size),
-                    CU_TENSOR_MAP_SWIZZLE_128B);
+  const cuuint64_t D = static_cast<cuuint64_t>(c.head_dim);
+  const cuuint64_t B = static_cast<cuuint64_t>(c.block_size);
+  const cuuint64_t rows = static_cast<cuuint64_t>(c.num_blocks) * c.num_kv_heads;
+  const cuuint64_t dims[5] = {D, 2, B / 4, 2, rows};
+  const cuuint64_t strides[4] = {D, 4 * D, 2 * D, B * D};
+  const cuuint32_t box[5] = {static_cast<cuuint32_t>(D), 2u, static_cast<cuuint32_t>(B / 4), 2u, 1u};
+  return encode_bytes(map, pool, 5, dims, strides, box);
 }
 
+// The V tile of (block, kv head) is D rows of B codes, D*B contiguous bytes;
+// it is moved as (D*B)/128 rows of 128 bytes.
 pkv_status encode_fp8_v_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(c.block_size), static_cast<cuuint64_t>(c.head_dim),
-                              static_cast<cuuint64_t>(c.num_kv_heads),
-                              static_cast<cuuint64_t>(c.num_blocks)};
-  const CUtensorMapSwizzle sw = c.block_size == 64   ? CU_TENSOR_MAP_SWIZZLE_64B
-                                : c.block_size == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                                     : CU_TENSOR_MAP_SWIZZLE_NONE;
-  return encode_map(map, pool, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dims,
-                    static_cast<cuuint32_t>(c.block_size), static_cast<cuuint32_t>(c.head_dim), sw);
+  const cuuint64_t tile = static_cast<cuuint64_t>(c.head_dim) * c.block_size;
+  const cuuint64_t rows = static_cast<cuuint64_t>(c.num_blocks) * c.num_kv_heads;
+  const cuuint64_t dims[3] = {128, tile / 128, rows};
+  const cuuint64_t strides[2] = {128, tile};
+  const cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(tile / 128), 1u};
+  return encode_bytes(map, pool, 3, dims, strides, box);
 }
 
 }  // namespace pkv

@@ -30,8 +30,12 @@ pkv_status check_device();
 // [N][Hkv][B][D] (fastest last), box = 64 elements x B rows, 128-byte swizzle.
 pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
 
-// 8-bit pools: K as [N][Hkv][B][D] bytes, box D x B, 128-byte swizzle (D = 128);
-// V as [N][Hkv][D][B] bytes, box B x D, swizzle span B bytes (none at B = 16).
+// 8-bit pools (D = 128), 128-byte swizzle, one box per (block, kv head) tile
+// addressed by the row block * Hkv + head.  K [N][Hkv][B][D] bytes through a
+// rank-5 view that puts the rows of each score column tile together (the
+// token order is given with the encoder); V [N][Hkv][D][B] bytes as rows of
+// 128 bytes.
+
 pkv_status encode_fp8_k_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
 pkv_status encode_fp8_v_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
 

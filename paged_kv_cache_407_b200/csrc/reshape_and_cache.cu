@@ -78,11 +78,13 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Quantising write into 8-bit pools: one thread per 16 dimensions of one
-// (token, kv head).  Each value x is stored as e4m3(x / scale) (IEEE fp32
-// division, round to nearest even, saturated to +-448).  K codes go to the
-// token's row, V codes to the token's column of the transposed V tile.
-template <typename T>
+// Quantising write into 8-bit pools: one thread per 4 dimensions of one
+// (token, kv head), so a warp covers a 128-wide head.  Each value x is stored
+// as e4m3(x / scale) (IEEE fp32 division, round to nearest even, saturated to
+// +-448).  K codes go to the token's row (one 32-bit store per thread, a
+// coalesced 128-byte row per warp), V codes to the token's column of the
+// transposed V tile (single bytes, B apart).  VEC: 8-byte input loads.
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(256)
     reshape_and_cache_fp8_kernel(const T *__restrict__ key, const T *__restrict__ value,
                                  int64_t key_stride, int64_t value_stride,
@@ -90,8 +92,8 @@ __global__ void __launch_bounds__(256)
                                  const int64_t *__restrict__ slot_mapping, int num_tokens,
                                  int num_kv_heads, int head_dim, int block_size, int64_t num_slots,
                                  float k_scale, float v_scale, int32_t *d_status) {
-  const int chunks = head_dim / 16;
-  const int64_t per_token = static_cast<int64_t>(num_kv_heads) * chunks;
+  const int quads = head_dim / 4;
+  const int64_t per_token = static_cast<int64_t>(num_kv_heads) * quads;
   const int64_t total = per_token * num_tokens;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -103,36 +105,43 @@ __global__ void __launch_bounds__(256)
       if (r == 0) raise_flag(d_status, PKV_DEV_BAD_SLOT);
       continue;
     }
-    const int64_t h = r / chunks;
-    const int64_t d0 = (r - h * chunks) * 16;
+    const int64_t h = r / quads;
+    const int64_t d0 = (r - h * quads) * 4;
     const int64_t blk = slot / block_size;
     const int64_t pos = slot - blk * block_size;
     const T *kp = key + t * key_stride + h * head_dim + d0;
     const T *vp = value + t * value_stride + h * head_dim + d0;
-    uint32_t kw[4];
-    uint8_t vq[16];
+    T kx[4], vx[4];
+    if constexpr (VEC) {
+      *reinterpret_cast<uint2 *>(kx) = *reinterpret_cast<const uint2 *>(kp);
+      *reinterpret_cast<uint2 *>(vx) = *reinterpret_cast<const uint2 *>(vp);
+    } else {
 #pragma unroll
-    for (int j = 0; j < 16; j += 4) {
-      float2 a = make_float2(static_cast<float>(kp[j]) / k_scale, static_cast<float>(kp[j + 1]) / k_scale);
-      float2 b = make_float2(static_cast<float>(kp[j + 2]) / k_scale, static_cast<float>(kp[j + 3]) / k_scale);
-      const uint32_t lo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
-      const uint32_t hi = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
-      kw[j / 4] = lo | (hi << 16);
-      a = make_float2(static_cast<float>(vp[j]) / v_scale, static_cast<float>(vp[j + 1]) / v_scale);
-      b = make_float2(static_cast<float>(vp[j + 2]) / v_scale, static_cast<float>(vp[j + 3]) / v_scale);
-      const uint32_t vlo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
-      const uint32_t vhi = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
-      vq[j] = vlo & 0xff;
-      vq[j + 1] = vlo >> 8;
-      vq[j + 2] = vhi & 0xff;
-      vq[j + 3] = vhi >> 8;
+      for (int j = 0; j < 4; ++j) {
+        kx[j] = kp[j];
+        vx[j] = vp[j];
+      }
     }
-    const int64_t base = (blk * num_kv_heads + h);
-    *reinterpret_cast<uint4 *>(k_cache + (base * block_size + pos) * head_dim + d0) =
-        make_uint4(kw[0], kw[1], kw[2], kw[3]);
+    const uint32_t k01 = __nv_cvt_float2_to_fp8x2(
+        make_float2(static_cast<float>(kx[0]) / k_scale, static_cast<float>(kx[1]) / k_scale),
+        __NV_SATFINITE, __NV_E4M3);
+    const uint32_t k23 = __nv_cvt_float2_to_fp8x2(
+        make_float2(static_cast<float>(kx[2]) / k_scale, static_cast<float>(kx[3]) / k_scale),
+        __NV_SATFINITE, __NV_E4M3);
+    const uint32_t v01 = __nv_cvt_float2_to_fp8x2(
+        make_float2(static_cast<float>(vx[0]) / v_scale, static_cast<float>(vx[1]) / v_scale),
+        __NV_SATFINITE, __NV_E4M3);
+    const uint32_t v23 = __nv_cvt_float2_to_fp8x2(
+        make_float2(static_cast<float>(vx[2]) / v_scale, static_cast<float>(vx[3]) / v_scale),
+        __NV_SATFINITE, __NV_E4M3);
+    const int64_t base = blk * num_kv_heads + h;
+    *reinterpret_cast<uint32_t *>(k_cache + (base * block_size + pos) * head_dim + d0) =
+        (k01 & 0xffffu) | (k23 << 16);
     uint8_t *vrow = v_cache + (base * head_dim + d0) * block_size + pos;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) vrow[j * block_size] = vq[j];
+    vrow[0] = static_cast<uint8_t>(v01);
+    vrow[block_size] = static_cast<uint8_t>(v01 >> 8);
+    vrow[2 * block_size] = static_cast<uint8_t>(v23);
+    vrow[3 * block_size] = static_cast<uint8_t>(v23 >> 8);
   }
 }
 
@@ -166,21 +175,29 @@ extern "C" pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *val
   if ((st = check_device()) != PKV_OK) return st;
   const int64_t num_slots = static_cast<int64_t>(cache.num_blocks) * cache.block_size;
   const int threads = 256;
-  const int64_t items = static_cast<int64_t>(num_tokens) * cache.num_kv_heads * (cache.head_dim / 16);
+  const int64_t items = static_cast<int64_t>(num_tokens) * cache.num_kv_heads * (cache.head_dim / 4);
   const int blocks = static_cast<int>(std::min<int64_t>((items + threads - 1) / threads, 148 * 16));
+  const bool vec = aligned(key, 8) && aligned(value, 8) && key_token_stride % 4 == 0 &&
+                   value_token_stride % 4 == 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (input_dtype == PKV_BF16)
-    reshape_and_cache_fp8_kernel<__nv_bfloat16><<<blocks, threads, 0, s>>>(
-        static_cast<const __nv_bfloat16 *>(key), static_cast<const __nv_bfloat16 *>(value),
-        key_token_stride, value_token_stride, static_cast<uint8_t *>(k_cache),
-        static_cast<uint8_t *>(v_cache), slot_mapping, num_tokens, cache.num_kv_heads,
-        cache.head_dim, cache.block_size, num_slots, k_scale, v_scale, d_status);
-  else
-    reshape_and_cache_fp8_kernel<__half><<<blocks, threads, 0, s>>>(
-        static_cast<const __half *>(key), static_cast<const __half *>(value), key_token_stride,
-        value_token_stride, static_cast<uint8_t *>(k_cache), static_cast<uint8_t *>(v_cache),
-        slot_mapping, num_tokens, cache.num_kv_heads, cache.head_dim, cache.block_size,
-        num_slots, k_scale, v_scale, d_status);
+#define PKV_FP8_WRITE(T, V)                                                                   \
+  reshape_and_cache_fp8_kernel<T, V><<<blocks, threads, 0, s>>>(                              \
+      static_cast<const T *>(key), static_cast<const T *>(value), key_token_stride,           \
+      value_token_stride, static_cast<uint8_t *>(k_cache), static_cast<uint8_t *>(v_cache),   \
+      slot_mapping, num_tokens, cache.num_kv_heads, cache.head_dim, cache.block_size,         \
+      num_slots, k_scale, v_scale, d_status)
+  if (input_dtype == PKV_BF16) {
+    if (vec)
+      PKV_FP8_WRITE(__nv_bfloat16, true);
+    else
+      PKV_FP8_WRITE(__nv_bfloat16, false);
+  } else {
+    if (vec)
+      PKV_FP8_WRITE(__half, true);
+    else
+      PKV_FP8_WRITE(__half, false);
+  }
+#undef PKV_FP8_WRITE
   return launch_status();
 }
 

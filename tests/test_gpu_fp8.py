@@ -10,7 +10,7 @@ import oracle as O
 import paged_kv_cache_407_b200 as pkv
 import workloads as W
 from parity import compare, status_tensor
-from workloads.device import upload_fp8
+from workloads.device import bits_to_tensor, upload_fp8
 
 pytestmark = pytest.mark.gpu
 
@@ -68,6 +68,37 @@ def test_fp8_cache_write_bit_exact(dtype, B, Hkv, scales):
     assert np.array_equal(_u8(db.k_cache), kc)
     assert np.array_equal(_u8(db.v_cache), vc)
     assert int(st.item()) == 0
+
+
+def test_fp8_cache_write_strided_and_unaligned_inputs():
+    """Keys/values given as a slice of a fused QKV row (8-byte loads) and as
+    rows that are only 2-byte aligned (element loads); padding slots skipped."""
+    b = W.small_case(17, num_seqs=7, num_q_heads=4, num_kv_heads=4, head_dim=128, block_size=16,
+                     dtype=W.F16, max_len=50)
+    f8 = W.fp8_variant(b, 3, k_scale=0.09, v_scale=0.13)
+    slots = b.slot_mapping.copy()
+    slots[[2, 5]] = -1
+    T, H, D = b.key.shape
+    kc, vc = O.reshape_and_cache_fp8(f8.k_cache, f8.v_cache, b.key, b.value, slots, 16, f8.k_scale,
+                                     f8.v_scale, b.dtype)
+    s_dev = torch.from_numpy(slots).cuda()
+    wide_k = np.zeros((T, 3, H, D), np.uint16)
+    wide_v = np.zeros((T, 3, H, D), np.uint16)
+    wide_k[:, 1], wide_v[:, 2] = b.key, b.value
+    k_view = bits_to_tensor(wide_k, b.dtype, "cuda")[:, 1]
+    v_view = bits_to_tensor(wide_v, b.dtype, "cuda")[:, 2]
+    db = upload_fp8(f8)
+    pkv.reshape_and_cache_fp8(k_view, v_view, db.k_cache, db.v_cache, s_dev, f8.k_scale, f8.v_scale)
+    torch.cuda.synchronize()
+    assert np.array_equal(_u8(db.k_cache), kc) and np.array_equal(_u8(db.v_cache), vc)
+    flat_k = bits_to_tensor(np.concatenate([[0], b.key.ravel()]).astype(np.uint16), b.dtype, "cuda")
+    flat_v = bits_to_tensor(np.concatenate([[0], b.value.ravel()]).astype(np.uint16), b.dtype, "cuda")
+    k_odd, v_odd = flat_k[1:].view(T, H, D), flat_v[1:].view(T, H, D)
+    assert k_odd.data_ptr() % 8 != 0
+    db = upload_fp8(f8)
+    pkv.reshape_and_cache_fp8(k_odd, v_odd, db.k_cache, db.v_cache, s_dev, f8.k_scale, f8.v_scale)
+    torch.cuda.synchronize()
+    assert np.array_equal(_u8(db.k_cache), kc) and np.array_equal(_u8(db.v_cache), vc)
 
 
 FP8_CASES = [

@@ -178,6 +178,24 @@ def test_partition_size_does_not_change_the_result():
         assert np.max(np.abs(o - outs[2048])) < 4e-3, P
 
 
+def test_repeated_calls_are_bit_identical():
+    """Split partitions merged by whichever partition arrives last, the
+    separate merge kernel (> 32 partitions) and unsplit sequences: the same
+    inputs give the same bits on every call."""
+    b = W.small_case(21, num_seqs=9, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                     dtype=W.F16, max_len=1200)
+    db = run_step(b)
+    for P in (0, 32, 256):
+        outs = []
+        for _ in range(4):
+            pkv.paged_attention_decode(db.out, db.q, db.k_cache, db.v_cache, db.block_tables, db.context_lens,
+                                       b.max_context_len, b.scale, partition_size=P)
+            torch.cuda.synchronize()
+            outs.append(bits(db.out).copy())
+        assert all(np.array_equal(o, outs[0]) for o in outs), P
+        assert not np.any((outs[0] & 0x7C00) == 0x7C00), "inf/nan in output"
+
+
 def test_placement_and_padding_do_not_change_bits():
     """Moving every block elsewhere in the pool, and filling table padding
     with other blocks' ids, gives bit-identical outputs."""
