@@ -467,3 +467,151 @@ FP8_CHECKS = [
     check_fp8_decode_matches_fp16_decode,
 ]
 ALL_CHECKS += FP8_CHECKS
+
+
+# ---------------------------------------------------------------------------
+# Block manager: free pool, reference counts, append, copy-on-write, free
+# ---------------------------------------------------------------------------
+
+import oracle.block_manager as BMO  # noqa: E402
+
+
+def check_manager_append_rule_example():
+    """The append rule fixture, replayed through the manager: a request grows
+    from 0 to 33 tokens one step at a time and then finishes."""
+    fx = read_fixture(os.path.join(GOLDEN, "append_rule_example.txt"))
+    B = fx["block_size"][0]
+    m = BMO.BlockManager(16, B, 8, free_order=list(fx["free_pool"]))
+    m.add_sequence(0, 0)
+    slots = [m.append([0])[0][0] for _ in range(fx["tokens"][0])]
+    assert m.tables[0] == fx["expect_table"]
+    for t in (0, 15, 16, 31, 32):
+        assert slots[t] == fx[f"expect_slot_token_{t}"][0], t
+    m.free_sequence(0)
+    assert list(m.free) == fx["expect_free_after_finish"]
+
+
+def check_manager_copy_on_write_example():
+    fx = read_fixture(os.path.join(GOLDEN, "copy_on_write_example.txt"))
+    B, N = fx["block_size"][0], fx["num_blocks"][0]
+    m = BMO.BlockManager(N, B, 8)
+    m.add_sequence(9, fx["prompt_tokens"][0])
+    assert m.tables[9] == fx["expect_prompt_table"]
+    m.fork(9, 1)
+    m.fork(9, 2)
+    m.free_sequence(9)
+    slots, copies = m.append([1, 2])
+    assert slots == [fx["expect_slot_A"][0], fx["expect_slot_B"][0]]
+    assert copies == [tuple(fx["expect_copy"])]
+    assert m.tables[1] == fx["expect_table_A"] and m.tables[2] == fx["expect_table_B"]
+    assert list(m.free) == fx["expect_free_after_step"]
+    m.free_sequence(1)
+    assert list(m.free) == fx["expect_free_after_A"]
+    m.free_sequence(2)
+    assert list(m.free) == fx["expect_free_after_B"]
+
+
+def _paged_view(pool, table, length, B):
+    return [pool.get(table[t // B] * B + t % B) for t in range(length)]
+
+
+def check_manager_brute_force_churn():
+    """Random arrivals, forks, decode steps and finishes against the plain
+    logical model (each request is the list of its tokens).  After every
+    operation: reading each request through its Block Table gives its tokens;
+    every block's reference count is the number of tables that hold it;
+    the free pool holds exactly the unreferenced blocks, once each; a step is
+    refused exactly when the pool is short, and then changes nothing."""
+    rng = np.random.default_rng(5)
+    for trial in range(6):
+        B = int(rng.choice([2, 4, 16]))
+        N = int(rng.integers(6, 40))
+        m = BMO.BlockManager(N, B, 64)
+        pool: dict[int, int] = {}  # slot -> token value (the physical contents)
+        hist: dict[int, list[int]] = {}  # request -> its tokens (the logical model)
+        next_id, next_val = 0, 1
+        for _ in range(150):
+            op = rng.random()
+            live = sorted(hist)
+            if op < 0.2 or not live:
+                n = int(rng.integers(0, 3 * B))
+                if -(-n // B) <= len(m.free):
+                    vals = list(range(next_val, next_val + n))
+                    next_val += n
+                    for slot, v in zip(m.add_sequence(next_id, n), vals):
+                        pool[slot] = v
+                    hist[next_id] = vals
+                    next_id += 1
+            elif op < 0.3:
+                p = int(rng.choice(live))
+                m.fork(p, next_id)
+                hist[next_id] = list(hist[p])
+                next_id += 1
+            elif op < 0.45:
+                s = int(rng.choice(live))
+                m.free_sequence(s)
+                del hist[s]
+            else:
+                k = int(rng.integers(1, len(live) + 1))
+                ids = [int(x) for x in rng.permutation(live)[:k]]
+                need = m.blocks_needed(ids)
+                before = (list(m.free), list(m.ref), {s: list(t) for s, t in m.tables.items()}, dict(m.lens))
+                if need > len(m.free):
+                    try:
+                        m.append(ids)
+                        raise AssertionError("step should have been refused")
+                    except BMO.OutOfBlocks:
+                        pass
+                    assert (list(m.free), list(m.ref), m.tables, m.lens) == before
+                else:
+                    free_before = len(m.free)
+                    slots, copies = m.append(ids)
+                    assert free_before - len(m.free) == need
+                    for src, dst in copies:  # copies run before the writes
+                        for o in range(B):
+                            if src * B + o in pool:
+                                pool[dst * B + o] = pool[src * B + o]
+                    for s, slot in zip(ids, slots):
+                        pool[slot] = next_val
+                        hist[s].append(next_val)
+                        next_val += 1
+            # invariants
+            counts = [0] * N
+            for s, t in m.tables.items():
+                assert len(t) == -(-m.lens[s] // B) and m.lens[s] == len(hist[s])
+                assert _paged_view(pool, t, m.lens[s], B) == hist[s], (trial, s)
+                for b in t:
+                    counts[b] += 1
+            assert counts == m.ref
+            assert sorted(m.free) == [b for b in range(N) if counts[b] == 0]
+
+
+def check_manager_append_matches_append_rule():
+    """For requests that share nothing, the manager's slots are the append
+    rule's slots (the pinned single-table function) with the same pool."""
+    rng = np.random.default_rng(8)
+    B, N = 4, 30
+    order = [int(x) for x in rng.permutation(N)]
+    m = BMO.BlockManager(N, B, 64, free_order=list(order))
+    free = list(order)
+    tables = {0: [], 1: []}
+    lens = {0: 0, 1: 0}
+    m.add_sequence(0, 0)
+    m.add_sequence(1, 0)
+    for step in range(25):
+        ids = [0, 1] if step % 3 else [1, 0]
+        slots, copies = m.append(ids)
+        assert copies == []
+        for s, slot in zip(ids, slots):
+            assert slot == O.append_token(tables[s], lens[s], free, B)
+            lens[s] += 1
+    assert m.tables == tables and list(m.free) == free
+
+
+BM_CHECKS = [
+    check_manager_append_rule_example,
+    check_manager_copy_on_write_example,
+    check_manager_brute_force_churn,
+    check_manager_append_matches_append_rule,
+]
+ALL_CHECKS += BM_CHECKS

@@ -4,6 +4,7 @@ least one pin catches each of them."""
 import numpy as np
 import pytest
 
+import oracle.block_manager as BMO
 import oracle.paged_kv as O
 from pins import ALL_CHECKS
 
@@ -100,6 +101,45 @@ def _materialize_fp8_v_untransposed(k_cache, v_cache, table_row, length, block_s
     return np.ascontiguousarray(K.transpose(1, 0, 2)), np.ascontiguousarray(V.transpose(1, 0, 2))
 
 
+def _bm_append_in_place(self, seq_ids):
+    """Copy-on-write left out: a shared last block is written in place."""
+    seq_ids = list(seq_ids)
+    B = self.block_size
+    slots = []
+    for s in seq_ids:
+        table, L = self.tables[s], self.lens[s]
+        if L % B == 0:
+            table.append(self._take())
+        slots.append(table[-1] * B + L % B)
+        self.lens[s] = L + 1
+    return slots, []
+
+
+def _bm_free_ignores_refs(self, seq_id):
+    for b in self.tables.pop(seq_id):
+        self.ref[b] = 0
+        if b not in self.free:
+            self.free.append(b)
+    del self.lens[seq_id]
+
+
+def _bm_fork_without_refs(self, parent, child):
+    self.tables[child] = list(self.tables[parent])
+    self.lens[child] = self.lens[parent]
+
+
+def _bm_needed_counts_every_shared(self, seq_ids):
+    B = self.block_size
+    return sum(1 for s in seq_ids if self.lens[s] % B == 0 or self.ref[self.tables[s][-1]] > 1)
+
+
+BM_MUTANTS = {
+    "manager_copy_on_write_left_out": ("append", _bm_append_in_place),
+    "manager_free_ignores_refcounts": ("free_sequence", _bm_free_ignores_refs),
+    "manager_fork_takes_no_reference": ("fork", _bm_fork_without_refs),
+    "manager_step_count_ignores_earlier_copies": ("blocks_needed", _bm_needed_counts_every_shared),
+}
+
 MUTANTS = {
     "attend_drops_scale": ("attend", _attend_no_scale),
     "attend_uses_keys_as_values": ("attend", _attend_values_from_keys),
@@ -118,16 +158,20 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(BM_MUTANTS))
 def test_mutant_is_caught(name, monkeypatch):
-    attr, fn = MUTANTS[name]
-    monkeypatch.setattr(O, attr, fn)
+    if name in BM_MUTANTS:
+        attr, fn = BM_MUTANTS[name]
+        monkeypatch.setattr(BMO.BlockManager, attr, fn)
+    else:
+        attr, fn = MUTANTS[name]
+        monkeypatch.setattr(O, attr, fn)
     caught = []
     for check in ALL_CHECKS:
         try:
             check()
         except AssertionError:
             caught.append(check.__name__)
-        except (IndexError, ValueError):
+        except (IndexError, ValueError, KeyError, BMO.OutOfBlocks):
             caught.append(check.__name__ + " (raised)")
     assert caught, f"no pin catches the planted mistake {name}"
