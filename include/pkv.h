@@ -61,7 +61,9 @@ typedef enum {
   PKV_ERR_BAD_PARTITION = 6,  /* partition_size not a positive multiple of block_size */
   PKV_ERR_TOO_LARGE = 7,      /* a size exceeds what the kernels index (see each call) */
   PKV_ERR_CUDA = 8,           /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
-  PKV_ERR_DEVICE = 9          /* current device is not compute capability 10.0 (B200 / sm_100a) */
+  PKV_ERR_DEVICE = 9,         /* current device is not compute capability 10.0 (B200 / sm_100a) */
+  PKV_ERR_NO_BLOCKS = 10,     /* block manager: the free pool cannot supply the blocks asked for */
+  PKV_ERR_BAD_SEQUENCE = 11   /* block manager: unknown, repeated or already present sequence id */
 } pkv_status;
 
 /* Device-side error bits OR-ed into *d_status. */

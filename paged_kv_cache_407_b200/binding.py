@@ -21,7 +21,10 @@ STATUS_NAMES = {
     0: "PKV_OK", 1: "PKV_ERR_NULL_POINTER", 2: "PKV_ERR_BAD_DTYPE", 3: "PKV_ERR_BAD_SHAPE",
     4: "PKV_ERR_MISALIGNED", 5: "PKV_ERR_WORKSPACE", 6: "PKV_ERR_BAD_PARTITION",
     7: "PKV_ERR_TOO_LARGE", 8: "PKV_ERR_CUDA", 9: "PKV_ERR_DEVICE",
+    10: "PKV_ERR_NO_BLOCKS", 11: "PKV_ERR_BAD_SEQUENCE",
 }
+ERR_NO_BLOCKS = 10
+ERR_BAD_SEQUENCE = 11
 # device-side flags
 DEV_BAD_BLOCK = 0x1
 DEV_BAD_SLOT = 0x2
@@ -34,7 +37,7 @@ PKV_FP8_E4M3 = 2
 _DTYPES = {torch.float16: PKV_F16, torch.bfloat16: PKV_BF16}
 _FP8_DTYPES = (torch.uint8, torch.float8_e4m3fn)
 
-# Every function declared in include/pkv.h, with (restype, argtypes).
+# Every function declared in include/*.h, with (restype, argtypes).
 _c_void_p, _i32, _i64, _f32, _size_t = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 
 
@@ -71,6 +74,21 @@ SIGNATURES = {
                                                       _f32, _f32, _f32, _i32, _c_void_p, _size_t, _c_void_p,
                                                       _c_void_p]),
     "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    # include/pkv_block_manager.h (host only)
+    "pkv_bm_create": (ctypes.c_int, [_i32, _i32, _i32, ctypes.POINTER(_c_void_p)]),
+    "pkv_bm_destroy": (None, [_c_void_p]),
+    "pkv_bm_num_free_blocks": (_i32, [_c_void_p]),
+    "pkv_bm_num_sequences": (_i32, [_c_void_p]),
+    "pkv_bm_ref_count": (_i32, [_c_void_p, _i32]),
+    "pkv_bm_context_len": (_i32, [_c_void_p, _i64]),
+    "pkv_bm_add_sequence": (ctypes.c_int, [_c_void_p, _i64, _i32, _c_void_p]),
+    "pkv_bm_fork": (ctypes.c_int, [_c_void_p, _i64, _i64]),
+    "pkv_bm_free_sequence": (ctypes.c_int, [_c_void_p, _i64]),
+    "pkv_bm_blocks_needed": (_i32, [_c_void_p, _c_void_p, _i32]),
+    "pkv_bm_append": (ctypes.c_int, [_c_void_p, _c_void_p, _i32, _c_void_p, _c_void_p, _i32,
+                                     ctypes.POINTER(_i32)]),
+    "pkv_bm_block_tables": (ctypes.c_int, [_c_void_p, _c_void_p, _i32, _c_void_p, _i32, _c_void_p]),
+    "pkv_bm_free_list": (ctypes.c_int, [_c_void_p, _c_void_p, _i32, ctypes.POINTER(_i32)]),
     "pkv_version": (_i32, []),
 }
 

@@ -1,8 +1,9 @@
 """Build libpkv.so (the C-ABI CUDA library) in-tree for B200 (sm_100a).
 
 Usage: ``python -m paged_kv_cache_407_b200.build [-v]``.  Compiles every
-``csrc/*.cu`` with nvcc into ``_build/`` and links
-``paged_kv_cache_407_b200/libpkv.so`` (CUDA runtime linked statically).
+``csrc/*.cu`` with nvcc and every host-only ``csrc/*.cpp`` with the host
+compiler into ``_build/`` and links ``paged_kv_cache_407_b200/libpkv.so``
+(CUDA runtime linked statically).
 """
 
 from __future__ import annotations
@@ -27,6 +28,16 @@ NVCC_FLAGS = [
 ]
 
 
+CXX_FLAGS = ["-O2", "-std=c++17", "-fPIC", "-fvisibility=hidden", "-Wall", "-Wextra", "-I", INCLUDE, "-I", CSRC]
+
+
+def cxx_path() -> str:
+    cand = os.environ.get("CXX") or shutil.which("g++") or shutil.which("c++")
+    if not cand:
+        raise RuntimeError("no host C++ compiler found to build libpkv")
+    return cand
+
+
 def nvcc_path() -> str:
     cand = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
     if not os.path.exists(cand):
@@ -35,17 +46,20 @@ def nvcc_path() -> str:
 
 
 def sources() -> list[str]:
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cpp")))
 
 
 def _compile(src: str, verbose: bool, ptxas_info: bool) -> str:
-    obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
-    cmd = [nvcc_path(), *ARCH_FLAGS, *NVCC_FLAGS, "-c", src, "-o", obj]
-    if ptxas_info:
-        cmd += ["-Xptxas", "-v"]
+    obj = os.path.join(BUILD_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
+    if src.endswith(".cpp"):
+        cmd = [cxx_path(), *CXX_FLAGS, "-c", src, "-o", obj]
+    else:
+        cmd = [nvcc_path(), *ARCH_FLAGS, *NVCC_FLAGS, "-c", src, "-o", obj]
+        if ptxas_info:
+            cmd += ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError(f"nvcc failed on {src}:\n{res.stdout}\n{res.stderr}")
+        raise RuntimeError(f"compiling {src} failed:\n{res.stdout}\n{res.stderr}")
     if verbose and (res.stdout or res.stderr):
         sys.stderr.write(res.stdout + res.stderr)
     return obj
@@ -56,7 +70,7 @@ def _stale(objs_srcs) -> bool:
         return True
     lib_t = os.path.getmtime(LIB_PATH)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    headers.append(os.path.join(INCLUDE, "pkv.h"))
+    headers += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
     newest = max(os.path.getmtime(p) for p in [*objs_srcs, *headers, __file__])
     return newest > lib_t
 

@@ -130,6 +130,8 @@ extern "C" const char *pkv_status_string(pkv_status s) {
     case PKV_ERR_TOO_LARGE: return "a size exceeds what the kernels can index";
     case PKV_ERR_CUDA: return "a CUDA runtime or driver call failed";
     case PKV_ERR_DEVICE: return "current device is not compute capability 10.0 (B200, sm_100a)";
+    case PKV_ERR_NO_BLOCKS: return "the free block pool cannot supply the blocks asked for";
+    case PKV_ERR_BAD_SEQUENCE: return "unknown, repeated or already present sequence id";
   }
   return "unknown pkv_status";
 }

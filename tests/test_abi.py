@@ -1,4 +1,4 @@
-"""libpkv.so loads and exports the C ABI of include/pkv.h; host-side
+"""libpkv.so loads and exports the C ABI of include/*.h; host-side
 validation returns its status codes without touching a device (CPU only)."""
 
 import ctypes
@@ -10,13 +10,17 @@ import pytest
 from paged_kv_cache_407_b200 import binding as bd
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "pkv.h")
+INCLUDE = os.path.join(ROOT, "include")
 
 
 def declared_functions():
-    text = open(HEADER, encoding="utf-8").read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pkv_[a-z_0-9]+)\s*\(", text)))
+    names = set()
+    for f in sorted(os.listdir(INCLUDE)):
+        if f.endswith(".h"):
+            text = open(os.path.join(INCLUDE, f), encoding="utf-8").read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(pkv_[a-z_0-9]+)\s*\(", text))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -48,7 +52,7 @@ def test_only_declared_symbols_are_exported():
 
 
 def test_status_strings_and_version(lib):
-    for code in range(10):
+    for code in range(12):
         assert lib.pkv_status_string(code)
     assert lib.pkv_status_string(0) == b"ok"
     assert bd.version() >= 100
