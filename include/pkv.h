@@ -271,7 +271,8 @@ PKV_API pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *value,
  * pools: K and V read back as code * k_scale and code * v_scale.  query and
  * out are fp16 or bf16 (query_dtype); the products run on fp16 operands
  * (E4M3 codes are exact in fp16; bf16 queries are converted to fp16, exact
- * for magnitudes in [2^-24, 65504]) with fp32 accumulation.  cache.dtype must
+ * for zero and magnitudes in [2^-14, 65504], rounded to fp16 subnormals below
+ * that) with fp32 accumulation.  cache.dtype must
  * be PKV_FP8_E4M3.  Other arguments, the workspace and errors as
  * pkv_paged_attention_decode.
  */
@@ -283,6 +284,49 @@ PKV_API pkv_status pkv_paged_attention_decode_fp8(
     size_t workspace_bytes, int32_t *d_status, pkv_stream_t stream);
 
 /* Static English text for a status code. */
+/*
+ * pkv_paged_attention_decode_lse - decode attention over a part of each
+ * sequence, returned as an attention state for a later merge.
+ *
+ * The same computation and arguments as pkv_paged_attention_decode (16-bit
+ * pools), over the tokens that block_tables / context_lens describe, e.g. one
+ * GPU's share of a sequence split across GPUs.  Instead of the T16 output it
+ * writes, per (sequence, query head) row r = s * num_q_heads + h:
+ *   out[r][0..head_dim)  fp32 normalised output  sum_i p_i V_i,
+ *   lse[r]               fp32 ln(sum_i exp(z_i)), z_i = scale * <q, K_i>
+ *                        (-inf for a row with no tokens, whose out is 0).
+ * Split-K identity (textbook softmax; not printed on the pages): outputs over
+ * disjoint token sets merge exactly with weights exp(lse_r - max lse).
+ * out and lse are device memory, 4-byte aligned; PKV_ERR_NULL_POINTER when lse
+ * is NULL.  Workspace and errors as pkv_paged_attention_decode.
+ */
+PKV_API pkv_status pkv_paged_attention_decode_lse(
+    float *out, float *lse, const void *query, const void *k_cache, const void *v_cache,
+    pkv_cache_desc cache, const int32_t *block_tables, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+    float scale, int32_t partition_size, void *workspace, size_t workspace_bytes,
+    int32_t *d_status, pkv_stream_t stream);
+
+/*
+ * pkv_merge_attention_states - merge attention states of the same rows over
+ * disjoint token sets (the all-gathered states of a sequence split across
+ * GPUs).
+ *
+ * states (device, fp32): num_states states, state k starting at
+ *   states + k * state_stride (floats), laid out as written by
+ *   pkv_paged_attention_decode_lse into one buffer: out [num_rows][head_dim]
+ *   followed by lse [num_rows].  state_stride >= num_rows * (head_dim + 1)
+ *   when num_states > 1.
+ * out (device, out_dtype = PKV_F16 / PKV_BF16): [num_rows][head_dim],
+ *   out = sum_k w_k o_k / sum_k w_k with w_k = exp(lse_k - max_k lse_k); a row
+ *   whose every lse is -inf (no tokens anywhere) gets 0.  num_states = 0 gives
+ *   zero rows.  head_dim 64 or 128.  Asynchronous on stream.
+ */
+PKV_API pkv_status pkv_merge_attention_states(void *out, pkv_dtype out_dtype, const float *states,
+                                              int64_t state_stride, int32_t num_states,
+                                              int32_t num_rows, int32_t head_dim,
+                                              pkv_stream_t stream);
+
 PKV_API const char *pkv_status_string(pkv_status status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

@@ -15,11 +15,15 @@ from .binding import (  # noqa: F401
     copy_blocks,
     fp8_cache_desc,
     library,
+    merge_attention_states,
     paged_attention_decode,
+    paged_attention_decode_lse,
     paged_attention_decode_fp8,
     partition_size,
     reshape_and_cache,
     reshape_and_cache_fp8,
+    state_buffer,
+    state_views,
     version,
     workspace_size,
 )

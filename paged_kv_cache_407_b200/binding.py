@@ -73,6 +73,11 @@ SIGNATURES = {
                                                       CacheDesc, _c_void_p, _i32, _c_void_p, _i32, _i32, _i32,
                                                       _f32, _f32, _f32, _i32, _c_void_p, _size_t, _c_void_p,
                                                       _c_void_p]),
+    "pkv_paged_attention_decode_lse": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                                      CacheDesc, _c_void_p, _i32, _c_void_p, _i32, _i32, _i32,
+                                                      _f32, _i32, _c_void_p, _size_t, _c_void_p, _c_void_p]),
+    "pkv_merge_attention_states": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _i64, _i32, _i32, _i32,
+                                                  _c_void_p]),
     "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     # include/pkv_block_manager.h (host only)
     "pkv_bm_create": (ctypes.c_int, [_i32, _i32, _i32, ctypes.POINTER(_c_void_p)]),
@@ -207,6 +212,67 @@ def paged_attention_decode(out, query, k_cache, v_cache, block_tables, context_l
         block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
         int(partition_size), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device))
     _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_lse(out, lse, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                               scale, partition_size=0, workspace=None, d_status=None, stream=None):
+    """Decode attention over the tokens the tables describe, returned as an
+    attention state: ``out`` fp32 ``[S, Hq, D]`` (normalised) and ``lse`` fp32
+    ``[S, Hq]`` (natural log of the softmax denominator, -inf for no tokens).
+    ``out`` and ``lse`` may be views of one packed buffer (``state_buffer``)."""
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    S, Hq, D = query.shape
+    if query.dtype != k_cache.dtype or not query.is_contiguous():
+        raise ValueError("query must be a contiguous [S, Hq, head_dim] tensor in the cache dtype")
+    if out.dtype != torch.float32 or tuple(out.shape) != (S, Hq, D) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous float32 [S, Hq, head_dim] tensor")
+    if lse.dtype != torch.float32 or lse.numel() != S * Hq or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [S, Hq] tensor")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S \
+            or not block_tables.is_contiguous():
+        raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
+    if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
+        raise ValueError("context_lens must be a contiguous int32 [S] tensor")
+    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = library().pkv_paged_attention_decode_lse(
+        _ptr(out), _ptr(lse), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
+        int(partition_size), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device))
+    _check(st, "pkv_paged_attention_decode_lse")
+    return out, lse
+
+
+def state_buffer(num_rows: int, head_dim: int, num_states: int = 1, device="cuda") -> torch.Tensor:
+    """fp32 ``[num_states, num_rows * (head_dim + 1)]``: per state, the rows'
+    outputs followed by their log-sum-exps (the layout the merge reads)."""
+    return torch.empty((num_states, num_rows * (head_dim + 1)), dtype=torch.float32, device=device)
+
+
+def state_views(state: torch.Tensor, num_seqs: int, num_q_heads: int, head_dim: int):
+    """(out ``[S, Hq, D]``, lse ``[S, Hq]``) views of one state of a state buffer."""
+    rows = num_seqs * num_q_heads
+    return (state[: rows * head_dim].view(num_seqs, num_q_heads, head_dim),
+            state[rows * head_dim: rows * (head_dim + 1)].view(num_seqs, num_q_heads))
+
+
+def merge_attention_states(out, states, stream=None):
+    """Merge ``states`` (``[R, rows * (D + 1)]`` fp32, see ``state_buffer``)
+    into ``out`` (fp16/bf16 ``[..., D]`` with ``rows`` rows)."""
+    if out.dtype not in _DTYPES or not out.is_contiguous():
+        raise ValueError("out must be a contiguous fp16/bf16 tensor")
+    D = out.shape[-1]
+    rows = out.numel() // D
+    if states.dtype != torch.float32 or states.dim() != 2 or states.shape[1] < rows * (D + 1) \
+            or not states.is_contiguous():
+        raise ValueError("states must be a contiguous float32 [R, rows * (head_dim + 1)] tensor")
+    st = library().pkv_merge_attention_states(_ptr(out), _DTYPES[out.dtype], _ptr(states), states.shape[1],
+                                              states.shape[0], rows, D, _stream(stream, out.device))
+    _check(st, "pkv_merge_attention_states")
     return out
 
 

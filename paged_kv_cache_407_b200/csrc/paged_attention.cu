@@ -35,6 +35,7 @@ namespace pkv {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // Split sequences with at most this many partitions are merged inside the
 // attention kernel by the last partition to finish; longer splits use the
@@ -43,7 +44,8 @@ constexpr int kFuseMaxParts = 32;
 
 struct DecodeArgs {
   const void *query;
-  void *out;
+  void *out;          // [S][Hq][D] of T, or of float when lse is set
+  float *lse;         // NULL, or [S][Hq]: natural log of the softmax denominator
   const int32_t *block_tables;
   const int32_t *context_lens;
   float *ws_m;        // [S][Hq][max_parts]
@@ -67,6 +69,26 @@ struct DecodeArgs {
 // ---------------------------------------------------------------------------
 // Result of one work unit, shared by both kernels.
 // ---------------------------------------------------------------------------
+
+// Write one finished row: acc = unnormalised output (lane's VPL dims), M / L =
+// running max (log2 units of exp(score)) and denominator.  T output, or fp32
+// output plus the row's log-sum-exp ln(sum_i exp(z_i)) = (M + log2 L) ln 2.
+template <typename T, int D>
+__device__ __forceinline__ void write_row(const DecodeArgs &a, size_t row, const float *acc,
+                                          float M, float L, int lane) {
+  constexpr int VPL = D / 32;
+  const float inv = L > 0.f ? a.out_scale / L : 0.f;
+  if (a.lse == nullptr) {
+    uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
+#pragma unroll
+    for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
+  } else {
+    float *dst = static_cast<float *>(a.out) + row * D + lane * VPL;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) dst[j] = acc[j] * inv;
+    if (lane == 0) a.lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+  }
+}
 
 // Store the result of one unit from `nw` deposited warp states (o at
 // mo + w*G*D as [row][D] floats, m/l at mm/ml + w*G), one warp, rows
@@ -97,10 +119,7 @@ __device__ __forceinline__ void store_unit_warp(const DecodeArgs &a, const float
     }
     const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(g) * G + h;
     if (nparts == 1) {
-      const float inv = lsum > 0.f ? a.out_scale / lsum : 0.f;
-      uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
-#pragma unroll
-      for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
+      write_row<T, D>(a, row, acc, M, lsum, lane);
     } else {
       const size_t idx = row * a.max_parts + part;
       float *dst = a.ws_o + idx * D + lane * VPL;
@@ -176,10 +195,7 @@ __device__ __forceinline__ void merge_partials_warp(const DecodeArgs &a, int s, 
         for (int j = 0; j < VPL; ++j) acc[j] += wu * v[u][j];
       }
     }
-    const float inv = L > 0.f ? a.out_scale / L : 0.f;
-    uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(a.out) + row * D + lane * VPL);
-#pragma unroll
-    for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
+    write_row<T, D>(a, row, acc, M, L, lane);
   }
 }
 
@@ -368,7 +384,8 @@ __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMi
 //   M = max_p m_p,  w_p = 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p l_p.
 // ---------------------------------------------------------------------------
 struct CombineArgs {
-  void *out;
+  void *out;   // T, or float when lse is set
+  float *lse;  // NULL, or [S][Hq] log-sum-exp
   const int32_t *context_lens;
   const float *ws_m;
   const float *ws_l;
@@ -432,8 +449,52 @@ __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
     for (; p < nparts; ++p) acc[0] += fast_exp2(pm[p] - M) * po[static_cast<size_t>(p) * D];
   }
   const float total = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  static_cast<T *>(c.out)[row * D + threadIdx.x] =
-      Pack<T>::from_float(lsum > 0.f ? total * c.out_scale / lsum : 0.f);
+  const float o = lsum > 0.f ? total * c.out_scale / lsum : 0.f;
+  if (c.lse == nullptr) {
+    static_cast<T *>(c.out)[row * D + threadIdx.x] = Pack<T>::from_float(o);
+  } else {
+    static_cast<float *>(c.out)[row * D + threadIdx.x] = o;
+    if (threadIdx.x == 0) c.lse[row] = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of attention states computed over disjoint parts of the same
+// sequences (e.g. on different GPUs): state r holds, per row, the normalised
+// fp32 output o_r[D] and its log-sum-exp lse_r.  With M = max_r lse_r and
+// w_r = exp(lse_r - M): out = sum_r w_r o_r / sum_r w_r (0 when every lse_r
+// is -inf).  One warp per row.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    merge_states_kernel(void *out, const float *__restrict__ states, int64_t state_stride,
+                        int num_states, int num_rows) {
+  constexpr int VPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= num_rows) return;
+  const size_t lse_off = static_cast<size_t>(num_rows) * D;
+  float M = -INFINITY;
+  for (int r = 0; r < num_states; ++r) M = fmaxf(M, states[r * state_stride + lse_off + row]);
+  float acc[VPL];
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) acc[j] = 0.f;
+  float W = 0.f;
+  if (M != -INFINITY) {
+    for (int r = 0; r < num_states; ++r) {
+      const float *st = states + r * state_stride;
+      const float w = fast_exp2((st[lse_off + row] - M) * kLog2e);
+      W += w;
+      const float *o = st + static_cast<size_t>(row) * D + lane * VPL;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) acc[j] += w * o[j];
+    }
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<T *>(out) + static_cast<size_t>(row) * D +
+                                               lane * VPL);
+#pragma unroll
+  for (int j = 0; j < VPL; j += 2) dst[j / 2] = Pack<T>::pack(acc[j] * inv, acc[j + 1] * inv);
 }
 
 // ---------------------------------------------------------------------------
@@ -580,8 +641,9 @@ namespace pkv {
 namespace {
 
 // Shared body of the decode entry points.  kv8: 8-bit pools with scales
-// k_scale / v_scale; act: dtype of query and out.
-pkv_status decode_impl(void *out, const void *query, pkv_dtype act, const void *k_cache,
+// k_scale / v_scale; act: dtype of query (and of out unless lse is set, when
+// out is fp32 and lse receives each row's log-sum-exp).
+pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, const void *k_cache,
                        const void *v_cache, const pkv_cache_desc &cache, bool kv8,
                        const int32_t *block_tables, int32_t max_blocks_per_seq,
                        const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads,
@@ -608,7 +670,7 @@ pkv_status decode_impl(void *out, const void *query, pkv_dtype act, const void *
   if (!out || !query || !k_cache || !v_cache || !block_tables || !context_lens)
     return PKV_ERR_NULL_POINTER;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(query, 4) || !aligned(out, 4) ||
-      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(lse, 4))
     return PKV_ERR_MISALIGNED;
 
   Plan plan;
@@ -634,6 +696,7 @@ pkv_status decode_impl(void *out, const void *query, pkv_dtype act, const void *
   DecodeArgs args{};
   args.query = query;
   args.out = out;
+  args.lse = lse;
   args.block_tables = block_tables;
   args.context_lens = context_lens;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -676,6 +739,7 @@ pkv_status decode_impl(void *out, const void *query, pkv_dtype act, const void *
 
   CombineArgs c{};
   c.out = out;
+  c.lse = lse;
   c.context_lens = context_lens;
   c.ws_m = args.ws_m;
   c.ws_l = args.ws_l;
@@ -702,7 +766,7 @@ extern "C" pkv_status pkv_paged_attention_decode(
     int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
     int32_t partition_size, void *workspace, size_t workspace_bytes, int32_t *d_status,
     pkv_stream_t stream) {
-  return pkv::decode_impl(out, query, cache.dtype, k_cache, v_cache, cache, false, block_tables,
+  return pkv::decode_impl(out, nullptr, query, cache.dtype, k_cache, v_cache, cache, false, block_tables,
                           max_blocks_per_seq, context_lens, num_seqs, num_q_heads, max_context_len,
                           scale, 1.f, 1.f, partition_size, workspace, workspace_bytes, d_status,
                           stream);
@@ -714,8 +778,54 @@ extern "C" pkv_status pkv_paged_attention_decode_fp8(
     const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
     float scale, float k_scale, float v_scale, int32_t partition_size, void *workspace,
     size_t workspace_bytes, int32_t *d_status, pkv_stream_t stream) {
-  return pkv::decode_impl(out, query, query_dtype, k_cache, v_cache, cache, true, block_tables,
+  return pkv::decode_impl(out, nullptr, query, query_dtype, k_cache, v_cache, cache, true, block_tables,
                           max_blocks_per_seq, context_lens, num_seqs, num_q_heads, max_context_len,
                           scale, k_scale, v_scale, partition_size, workspace, workspace_bytes,
                           d_status, stream);
+}
+
+extern "C" pkv_status pkv_paged_attention_decode_lse(
+    float *out, float *lse, const void *query, const void *k_cache, const void *v_cache,
+    pkv_cache_desc cache, const int32_t *block_tables, int32_t max_blocks_per_seq,
+    const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len,
+    float scale, int32_t partition_size, void *workspace, size_t workspace_bytes,
+    int32_t *d_status, pkv_stream_t stream) {
+  if (lse == nullptr && num_seqs > 0) return PKV_ERR_NULL_POINTER;
+  return pkv::decode_impl(out, lse, query, cache.dtype, k_cache, v_cache, cache, false,
+                          block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                          max_context_len, scale, 1.f, 1.f, partition_size, workspace,
+                          workspace_bytes, d_status, stream);
+}
+
+extern "C" pkv_status pkv_merge_attention_states(void *out, pkv_dtype out_dtype, const float *states,
+                                                 int64_t state_stride, int32_t num_states,
+                                                 int32_t num_rows, int32_t head_dim,
+                                                 pkv_stream_t stream) {
+  using namespace pkv;
+  if (!is_16bit(out_dtype)) return PKV_ERR_BAD_DTYPE;
+  if (num_states < 0 || num_rows < 0 || (head_dim != 64 && head_dim != 128))
+    return PKV_ERR_BAD_SHAPE;
+  if (num_rows == 0) return PKV_OK;
+  if (out == nullptr || (num_states > 0 && states == nullptr)) return PKV_ERR_NULL_POINTER;
+  const int64_t need = static_cast<int64_t>(num_rows) * (head_dim + 1);
+  if (num_states > 1 && state_stride < need) return PKV_ERR_BAD_SHAPE;
+  if (!aligned(out, 4) || !aligned(states, 4)) return PKV_ERR_MISALIGNED;
+  if (num_rows > (1 << 30) / 8) return PKV_ERR_TOO_LARGE;
+  pkv_status st = check_device();
+  if (st != PKV_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>((num_rows + 7) / 8);
+  const bool bf16 = out_dtype == PKV_BF16;
+  if (head_dim == 128) {
+    if (bf16)
+      merge_states_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
+    else
+      merge_states_kernel<__half, 128><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
+  } else {
+    if (bf16)
+      merge_states_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
+    else
+      merge_states_kernel<__half, 64><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
+  }
+  return launch_status();
 }
