@@ -29,3 +29,4 @@ from .paged_kv import (  # noqa: F401
     reshape_and_cache_fp8,
     slot_location,
 )
+from .prefill import paged_prefill  # noqa: F401,E402

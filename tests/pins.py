@@ -615,3 +615,90 @@ BM_CHECKS = [
     check_manager_append_matches_append_rule,
 ]
 ALL_CHECKS += BM_CHECKS
+
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill: causal attention of a chunk of new tokens over the cache
+# ---------------------------------------------------------------------------
+
+import oracle.prefill as PO  # noqa: E402
+
+
+def _prefill_case(seed=9, dtype=W.F16, B=8, lens=(1, 9, 30, 17, 64), chunks=(1, 9, 7, 1, 20)):
+    b = W.prefill_batch(seed, dtype=dtype, num_q_heads=6, num_kv_heads=2, head_dim=16, block_size=B,
+                        context_lens=list(lens), chunk_lens=list(chunks))
+    kc, vc = O.reshape_and_cache(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, B)
+    return b, kc, vc
+
+
+def check_prefill_is_a_sequence_of_decode_steps():
+    """Token j of a chunk sits at position p = L - C + j and sees positions
+    0..p: its row equals the (pinned) decode of that sequence cut at p + 1."""
+    b, kc, vc = _prefill_case()
+    out = PO.paged_prefill(b.q, kc, vc, b.block_tables, b.query_start, b.context_lens, b.block_size, b.scale,
+                           b.dtype)
+    for s in range(b.num_seqs):
+        L, t0, t1 = int(b.context_lens[s]), int(b.query_start[s]), int(b.query_start[s + 1])
+        for j in range(t1 - t0):
+            p = L - (t1 - t0) + j
+            ref = O.decode_sequence(b.q[t0 + j], kc, vc, b.block_tables[s], p + 1, b.block_size, b.scale, b.dtype)
+            assert np.allclose(out[t0 + j], ref, rtol=0, atol=1e-12), (s, j)
+
+
+def check_prefill_against_torch_sdpa_causal():
+    """Library special case: a whole-prompt prefill is torch's causal SDPA,
+    and a chunk is SDPA with the explicit mask key position <= query
+    position, both in float64 on the materialised K/V."""
+    import torch
+    b, kc, vc = _prefill_case(seed=10, dtype=W.BF16, lens=(12, 40), chunks=(12, 15))
+    out = PO.paged_prefill(b.q, kc, vc, b.block_tables, b.query_start, b.context_lens, b.block_size, b.scale,
+                           b.dtype)
+    Hq, Hkv = b.num_q_heads, b.num_kv_heads
+    for s in range(b.num_seqs):
+        L, t0, t1 = int(b.context_lens[s]), int(b.query_start[s]), int(b.query_start[s + 1])
+        C = t1 - t0
+        K = torch.from_numpy(O.decode_bits(O.materialize(kc, b.block_tables[s], L, b.block_size), b.dtype))
+        V = torch.from_numpy(O.decode_bits(O.materialize(vc, b.block_tables[s], L, b.block_size), b.dtype))
+        q = torch.from_numpy(O.decode_bits(b.q[t0:t1], b.dtype)).transpose(0, 1)  # [Hq, C, D]
+        K = K.repeat_interleave(Hq // Hkv, dim=0)
+        V = V.repeat_interleave(Hq // Hkv, dim=0)
+        if C == L:
+            ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, is_causal=True, scale=b.scale)
+        else:
+            mask = torch.arange(L)[None, :] <= (L - C + torch.arange(C))[:, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(q, K, V, attn_mask=mask, scale=b.scale)
+        assert np.allclose(out[t0:t1], ref.transpose(0, 1).numpy(), rtol=0, atol=1e-12), s
+
+
+def check_prefill_brute_force_tiny():
+    """Pure-Python loops: per query token, per head, a table lookup per key."""
+    b, kc, vc = _prefill_case(seed=11, B=4, lens=(6, 9), chunks=(3, 9))
+    out = PO.paged_prefill(b.q, kc, vc, b.block_tables, b.query_start, b.context_lens, b.block_size, b.scale,
+                           b.dtype)
+    Hq, Hkv, D, B = b.num_q_heads, b.num_kv_heads, b.head_dim, b.block_size
+    for s in range(b.num_seqs):
+        L, t0, t1 = int(b.context_lens[s]), int(b.query_start[s]), int(b.query_start[s + 1])
+        for j in range(t1 - t0):
+            p = L - (t1 - t0) + j
+            for h in range(Hq):
+                g = h * Hkv // Hq
+                q = [float(x) for x in O.decode_bits(b.q[t0 + j, h], b.dtype)]
+                zs, vs = [], []
+                for i in range(p + 1):
+                    blk = int(b.block_tables[s][i // B])
+                    k = O.decode_bits(kc[blk, g, i % B], b.dtype)
+                    zs.append(b.scale * sum(q[d] * float(k[d]) for d in range(D)))
+                    vs.append(O.decode_bits(vc[blk, g, i % B], b.dtype))
+                m = max(zs)
+                w = [math.exp(z - m) for z in zs]
+                ref = sum(wi * vi for wi, vi in zip(w, vs)) / sum(w)
+                assert np.allclose(out[t0 + j, h], ref, rtol=0, atol=1e-12)
+
+
+PREFILL_CHECKS = [
+    check_prefill_is_a_sequence_of_decode_steps,
+    check_prefill_against_torch_sdpa_causal,
+    check_prefill_brute_force_tiny,
+]
+ALL_CHECKS += PREFILL_CHECKS

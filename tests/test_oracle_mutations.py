@@ -6,6 +6,7 @@ import pytest
 
 import oracle.block_manager as BMO
 import oracle.paged_kv as O
+import oracle.prefill as PO
 from pins import ALL_CHECKS
 
 _orig_attend = O.attend
@@ -133,6 +134,48 @@ def _bm_needed_counts_every_shared(self, seq_ids):
     return sum(1 for s in seq_ids if self.lens[s] % B == 0 or self.ref[self.tables[s][-1]] > 1)
 
 
+def _prefill_not_causal(q_bits, k_cache, v_cache, block_tables, query_start, context_lens, block_size, scale,
+                        dtype, seqs=None):
+    """Every chunk token attends over the whole sequence."""
+    T, Hq, D = q_bits.shape
+    Hkv = k_cache.shape[1]
+    out = np.full((T, Hq, D), np.nan)
+    for s in range(len(context_lens)):
+        t0, t1, L = int(query_start[s]), int(query_start[s + 1]), int(context_lens[s])
+        K = O.decode_bits(O.materialize(k_cache, block_tables[s], L, block_size), dtype)
+        V = O.decode_bits(O.materialize(v_cache, block_tables[s], L, block_size), dtype)
+        for t in range(t0, t1):
+            q = O.decode_bits(q_bits[t], dtype)
+            for h in range(Hq):
+                g = O.kv_head_of(h, Hq, Hkv)
+                out[t, h] = O.attend(q[h:h + 1], K[g], V[g], scale)[0]
+    return out
+
+
+def _prefill_excludes_itself(q_bits, k_cache, v_cache, block_tables, query_start, context_lens, block_size,
+                             scale, dtype, seqs=None):
+    """Each token sees only the positions before it (the first sees itself)."""
+    T, Hq, D = q_bits.shape
+    Hkv = k_cache.shape[1]
+    out = np.full((T, Hq, D), np.nan)
+    for s in range(len(context_lens)):
+        t0, t1, L = int(query_start[s]), int(query_start[s + 1]), int(context_lens[s])
+        K = O.decode_bits(O.materialize(k_cache, block_tables[s], L, block_size), dtype)
+        V = O.decode_bits(O.materialize(v_cache, block_tables[s], L, block_size), dtype)
+        for j, t in enumerate(range(t0, t1)):
+            p = max(1, L - (t1 - t0) + j)
+            q = O.decode_bits(q_bits[t], dtype)
+            for h in range(Hq):
+                g = O.kv_head_of(h, Hq, Hkv)
+                out[t, h] = O.attend(q[h:h + 1], K[g, :p], V[g, :p], scale)[0]
+    return out
+
+
+PREFILL_MUTANTS = {
+    "prefill_not_causal": ("paged_prefill", _prefill_not_causal),
+    "prefill_query_excludes_itself": ("paged_prefill", _prefill_excludes_itself),
+}
+
 BM_MUTANTS = {
     "manager_copy_on_write_left_out": ("append", _bm_append_in_place),
     "manager_free_ignores_refcounts": ("free_sequence", _bm_free_ignores_refs),
@@ -158,11 +201,14 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(BM_MUTANTS))
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(BM_MUTANTS) + sorted(PREFILL_MUTANTS))
 def test_mutant_is_caught(name, monkeypatch):
     if name in BM_MUTANTS:
         attr, fn = BM_MUTANTS[name]
         monkeypatch.setattr(BMO.BlockManager, attr, fn)
+    elif name in PREFILL_MUTANTS:
+        attr, fn = PREFILL_MUTANTS[name]
+        monkeypatch.setattr(PO, attr, fn)
     else:
         attr, fn = MUTANTS[name]
         monkeypatch.setattr(O, attr, fn)

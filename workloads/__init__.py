@@ -491,3 +491,101 @@ def fp8_variant(batch: PagedBatch, seed: int, k_scale: float = 0.125, v_scale: f
             kc[slot // B, :, slot % B, :] = FP8_POISON
             vc[slot // B, :, :, slot % B] = FP8_POISON
     return Fp8Batch(base=batch, k_cache=kc, v_cache=vc, k_scale=k_scale, v_scale=v_scale)
+
+
+# --------------------------------------------------------------------------
+# Chunked-prefill batches
+# --------------------------------------------------------------------------
+
+
+@dataclass
+class PrefillBatch:
+    """One prefill call: sequence s has ``context_lens[s]`` tokens, the last
+    ``chunk_lens[s]`` of which are this call's new tokens (queries ``q`` rows
+    ``query_start[s] .. query_start[s+1]``; their K/V in ``key``/``value``,
+    to be written to ``slot_mapping`` before attention).  Earlier tokens are
+    already in the pools; every other slot holds the poison value."""
+
+    name: str
+    dtype: str
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    scale: float
+    q: np.ndarray            # [T, Hq, D] bits
+    k_cache: np.ndarray      # [N, Hkv, B, D] bits
+    v_cache: np.ndarray
+    block_tables: np.ndarray  # [S, max_blocks] int32, -1 padded
+    context_lens: np.ndarray  # [S] int32
+    query_start: np.ndarray   # [S + 1] int32
+    key: np.ndarray           # [T, Hkv, D] bits
+    value: np.ndarray
+    slot_mapping: np.ndarray  # [T] int64
+    seed: int
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.q.shape[0])
+
+    @property
+    def chunk_lens(self) -> np.ndarray:
+        return np.diff(self.query_start)
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max()) if self.num_seqs else 0
+
+    @property
+    def max_query_len(self) -> int:
+        return int(self.chunk_lens.max()) if self.num_seqs else 0
+
+
+def prefill_batch(seed: int, *, dtype: str, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                  block_size: int, context_lens, chunk_lens, scale: float | None = None,
+                  pool_slack: float = 0.10, name: str | None = None) -> PrefillBatch:
+    """Sequences own disjoint blocks of a shuffled pool; q, K, V ~ N(0, 1)."""
+    assert dtype in DTYPES
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(context_lens, dtype=np.int64)
+    chunks = np.asarray(chunk_lens, dtype=np.int64)
+    assert lens.shape == chunks.shape and np.all(chunks <= lens) and np.all(chunks >= 0)
+    S, B = lens.shape[0], block_size
+    nbs = np.array([_blocks_for(L, B) for L in lens], dtype=np.int64)
+    used = int(nbs.sum())
+    N = max(1, math.ceil((1.0 + pool_slack) * used))
+    perm = rng.permutation(N).astype(np.int32)
+    tables = np.full((S, max(1, int(nbs.max()) if S else 1)), -1, dtype=np.int32)
+    off = 0
+    for s in range(S):
+        tables[s, : nbs[s]] = perm[off : off + nbs[s]]
+        off += int(nbs[s])
+    poison = POISON_BITS[dtype]
+    k_cache = np.full((N, num_kv_heads, B, head_dim), poison, dtype=np.uint16)
+    v_cache = np.full_like(k_cache, poison)
+    new_k, new_v, slots = [], [], []
+    for s in range(S):
+        L, C = int(lens[s]), int(chunks[s])
+        kb = to_bits(rng.standard_normal((L, num_kv_heads, head_dim), dtype=np.float32), dtype)
+        vb = to_bits(rng.standard_normal((L, num_kv_heads, head_dim), dtype=np.float32), dtype)
+        _place(k_cache, tables[s], kb[: L - C], B)
+        _place(v_cache, tables[s], vb[: L - C], B)
+        new_k.append(kb[L - C:])
+        new_v.append(vb[L - C:])
+        slots += [_slot(tables[s], p, B) for p in range(L - C, L)]
+    T = int(chunks.sum())
+    q = to_bits(rng.standard_normal((T, num_q_heads, head_dim), dtype=np.float32), dtype)
+    shape0 = (0, num_kv_heads, head_dim)
+    return PrefillBatch(
+        name=name or f"prefill_{seed}", dtype=dtype, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+        head_dim=head_dim, block_size=B, scale=float(scale if scale is not None else 1.0 / math.sqrt(head_dim)),
+        q=q, k_cache=k_cache, v_cache=v_cache, block_tables=tables, context_lens=lens.astype(np.int32),
+        query_start=np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32),
+        key=np.concatenate(new_k) if T else np.zeros(shape0, np.uint16),
+        value=np.concatenate(new_v) if T else np.zeros(shape0, np.uint16),
+        slot_mapping=np.asarray(slots, dtype=np.int64), seed=seed,
+    )
