@@ -283,6 +283,45 @@ PKV_API pkv_status pkv_paged_attention_decode_fp8(
     float scale, float k_scale, float v_scale, int32_t partition_size, void *workspace,
     size_t workspace_bytes, int32_t *d_status, pkv_stream_t stream);
 
+/*
+ * pkv_paged_prefill - causal attention of chunks of new tokens over their
+ * sequences' paged K/V (prompt prefill, or one chunk of a long prompt).
+ *
+ * lshu.cn/news/11644 (vLLM architecture analysis), sections "整体架构" (a
+ * prompt is prefilled, a long one in chunks over several iterations) and
+ * "性能关键路径与瓶颈" (prefill is compute-bound on the tensor cores).
+ * Sequence s has context_lens[s] = L tokens, the last C = query_start[s+1] -
+ * query_start[s] of which are this call's: rows query_start[s] ..
+ * query_start[s+1] of query / out.  Their K/V must already be in the pools
+ * (pkv_reshape_and_cache of the chunk, as in decode).  The chunk's token at
+ * position p = L - C + j attends over positions 0 .. p of its own sequence:
+ *   out[t][h] = sum_{i<=p} softmax_i(scale * <query[t][h], K_g[i]>) V_g[i],
+ *   g = h / (num_q_heads / num_kv_heads).
+ *
+ * query, out : [num_tokens][num_q_heads][128] in the cache dtype (fp16/bf16),
+ *              16-byte aligned device memory.
+ * query_start: int32 [num_seqs + 1] device, non-decreasing, query_start[0] >= 0,
+ *              query_start[num_seqs] <= num_tokens; rows outside every chunk
+ *              are not written.
+ * context_lens: int32 [num_seqs] device, C <= L <= max_blocks_per_seq * B.
+ * block_tables: as for decode.  max_query_len >= every C (host value; it
+ *              sizes the grid).
+ * head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
+ * Runs on tcgen05 tensor cores: 128-row query tiles x 128-token K/V tiles,
+ * fp32 accumulation in tensor memory.
+ * Device-detected errors: a sequence whose lengths break the rules above is
+ * skipped with PKV_DEV_BAD_LEN; a block id outside the pool raises
+ * PKV_DEV_BAD_BLOCK (that block's tokens are garbage); a wait past ~1 s
+ * raises PKV_DEV_TIMEOUT.
+ */
+PKV_API pkv_status pkv_paged_prefill(void *out, const void *query, const void *k_cache,
+                                     const void *v_cache, pkv_cache_desc cache,
+                                     const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                     const int32_t *query_start, const int32_t *context_lens,
+                                     int32_t num_seqs, int32_t num_tokens, int32_t max_query_len,
+                                     int32_t num_q_heads, float scale, int32_t *d_status,
+                                     pkv_stream_t stream);
+
 /* Static English text for a status code. */
 /*
  * pkv_paged_attention_decode_lse - decode attention over a part of each

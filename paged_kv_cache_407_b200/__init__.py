@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     merge_attention_states,
     paged_attention_decode,
     paged_attention_decode_lse,
+    paged_prefill,
     paged_attention_decode_fp8,
     partition_size,
     reshape_and_cache,

@@ -78,6 +78,9 @@ SIGNATURES = {
                                                       _f32, _i32, _c_void_p, _size_t, _c_void_p, _c_void_p]),
     "pkv_merge_attention_states": (ctypes.c_int, [_c_void_p, ctypes.c_int, _c_void_p, _i64, _i32, _i32, _i32,
                                                   _c_void_p]),
+    "pkv_paged_prefill": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc, _c_void_p, _i32,
+                                         _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _f32, _c_void_p,
+                                         _c_void_p]),
     "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     # include/pkv_block_manager.h (host only)
     "pkv_bm_create": (ctypes.c_int, [_i32, _i32, _i32, ctypes.POINTER(_c_void_p)]),
@@ -273,6 +276,34 @@ def merge_attention_states(out, states, stream=None):
     st = library().pkv_merge_attention_states(_ptr(out), _DTYPES[out.dtype], _ptr(states), states.shape[1],
                                               states.shape[0], rows, D, _stream(stream, out.device))
     _check(st, "pkv_merge_attention_states")
+    return out
+
+
+def paged_prefill(out, query, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len, scale,
+                  d_status=None, stream=None):
+    """Causal attention of chunks of new tokens over their sequences' paged
+    K/V: ``query``/``out`` ``[T, Hq, 128]``; sequence s owns rows
+    ``query_start[s] .. query_start[s+1]`` (its last tokens, already written
+    to the cache); ``context_lens`` counts them."""
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    T, Hq, D = query.shape
+    if out.shape != query.shape or out.dtype != k_cache.dtype or query.dtype != k_cache.dtype:
+        raise ValueError("query/out must be [T, Hq, head_dim] in the cache dtype")
+    if not (query.is_contiguous() and out.is_contiguous()):
+        raise ValueError("query/out must be contiguous")
+    S = context_lens.numel()
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != S \
+            or not block_tables.is_contiguous():
+        raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
+    for t, n in ((query_start, S + 1), (context_lens, S)):
+        if t.dtype != torch.int32 or t.numel() != n or not t.is_contiguous():
+            raise ValueError("query_start / context_lens must be contiguous int32 [S + 1] / [S] tensors")
+    st = library().pkv_paged_prefill(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables), block_tables.shape[1],
+        _ptr(query_start), _ptr(context_lens), S, T, int(max_query_len), Hq, float(scale), _ptr(d_status),
+        _stream(stream, query.device))
+    _check(st, "pkv_paged_prefill")
     return out
 
 

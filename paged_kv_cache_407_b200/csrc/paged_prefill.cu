@@ -1,0 +1,459 @@
+// Paged (chunked) prefill attention on the fifth-generation tensor cores.
+//
+// lshu.cn/news/11644 (vLLM architecture analysis): "整体架构" (a new request's
+// prompt is prefilled, a long prompt in chunks over several iterations) and
+// "性能关键路径与瓶颈" (prefill is compute-bound on the tensor cores).  For each
+// sequence, the chunk's token at position p = L - C + j (its K/V already
+// written to the cache) attends over positions 0..p through the Block Table.
+//
+// One CTA per (128-row query tile, kv head, sequence); a tile row is one
+// (token, query head of the group) pair, so 128 / G tokens per tile.
+//   Q tile  [128 rows][128] by TMA (rank-3 map over [T][Hq][D]);
+//   K, V    128-token tiles gathered block by block through the Block Table
+//           (TMA, rank-4 map over [N][Hkv][B][D]), two stages;
+//   S = Q K^T   tcgen05.mma 128x128x128 into tensor memory (columns 0..127);
+//   softmax     one thread per row (tcgen05.ld of its TMEM lane), causal
+//               mask, running max with lazy rescaling (the reference max
+//               moves only when the row max grows by more than 2^8);
+//   P           written to shared memory (fp16, or bf16 high + bf16 residual
+//               for bf16 operands, which alone would round P by 2^-9);
+//   O += P V    tcgen05.mma 128x128x128 into tensor memory (columns
+//               128..255), V as an MN-major operand.
+// Every wait is bounded; on a timeout the CTA raises PKV_DEV_TIMEOUT, waits
+// (bounded) for its outstanding tensor-core work and frees its TMEM.
+#include <type_traits>
+
+#include "pkv_device.cuh"
+#include "pkv_host.h"
+#include "tcgen05.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kRows = 128;    // query rows per tile (MMA M)
+constexpr int kKv = 128;      // tokens per K/V tile
+constexpr int kDim = 128;     // head_dim
+constexpr int kThreads = 128;
+constexpr uint32_t kChunk = 128u * 128u;  // [128 rows][64 elements] of 16-bit: 16 KB
+constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
+constexpr uint32_t kQOff = 0;
+constexpr uint32_t kStageOff = kTile;             // stage st: K at + 2 st kTile, V after it
+constexpr uint32_t kPOff = kStageOff + 4u * kTile;  // P high, then P residual (bf16)
+constexpr uint32_t kTmemCols = 256;               // S: columns [0, 128), O: [128, 256)
+constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
+constexpr uint32_t kFullMask = 0xffffffffu;
+
+template <typename T>
+struct PrefillTune {
+  static constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
+  static constexpr uint32_t kBarOff = kPOff + (kSplit ? 2u : 1u) * kTile;
+  static constexpr uint32_t kSmem = kBarOff + 64u + 1024u;
+};
+
+struct PrefillArgs {
+  void *out;
+  const int32_t *block_tables;
+  const int32_t *query_start;
+  const int32_t *context_lens;
+  int32_t *d_status;
+  int num_tokens;
+  int max_blocks_per_seq;
+  int num_q_heads;
+  int group;
+  int num_blocks;
+  float scale_log2;
+};
+
+// Bounded wait by every thread, made uniform over the CTA.
+__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity) {
+  return __syncthreads_and(mbar_wait(bar, parity) ? 1 : 0) != 0;
+}
+
+template <typename T, int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+  using TN = PrefillTune<T>;
+  constexpr bool kSplit = TN::kSplit;
+  constexpr int kBlocksPerTile = kKv / BS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_addr(smem);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int qt = blockIdx.x;
+  const int g = blockIdx.y;
+  const int s = blockIdx.z;
+  const int G = a.group;
+  const int tok_per_tile = kRows / G;
+
+  // ---- geometry of this tile (uniform over the CTA) ----------------------
+  const int t_begin = a.query_start[s];
+  const int t_end = a.query_start[s + 1];
+  const int C = t_end - t_begin;
+  const int L = a.context_lens[s];
+  if (C < 0 || t_begin < 0 || t_end > a.num_tokens || L < C ||
+      static_cast<long long>(L) > static_cast<long long>(a.max_blocks_per_seq) * BS) {
+    if (tid == 0 && g == 0 && qt == 0) raise_flag(a.d_status, PKV_DEV_BAD_LEN);
+    return;
+  }
+  const int tok0 = qt * tok_per_tile;
+  if (tok0 >= C) return;
+  const int last_tok = min(tok0 + tok_per_tile, C) - 1;
+  const int p_max = L - C + last_tok;             // largest position among the tile's rows
+  const int ntiles = (p_max + kKv) / kKv;         // K/V tiles to visit (>= 1)
+  const int nb = (L + BS - 1) / BS;
+
+  // this thread's row (= TMEM lane)
+  const int t_row = tok0 + tid / G;  // chunk token of the row
+  const int h_row = tid % G;
+  const bool row_valid = t_row < C;
+  const int p_row = L - C + t_row;  // >= L for rows past the chunk
+
+  const uint32_t bar_q = sb + TN::kBarOff;
+  const uint32_t bar_kv0 = bar_q + 8;
+  const uint32_t bar_s = bar_q + 24;
+  const uint32_t bar_o = bar_q + 32;
+  const uint32_t bar_done = bar_q + 40;
+  const uint32_t holder = bar_q + 48;
+  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 48);
+
+  if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
+  if (tid == 0) {
+    mbar_init(bar_q, 1);
+    mbar_init(bar_kv0, 1);
+    mbar_init(bar_kv0 + 8, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_o, 1);
+    mbar_init(bar_done, 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *holder_ptr;
+  const uint32_t tS = tmem;
+  const uint32_t tO = tmem + 128;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+
+  const uint64_t policy = l2_evict_first_policy();
+  const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
+  // Block ids of K/V tile j: lane i of warp 0 holds block i of the tile.
+  auto tile_ids = [&](int j) -> int {
+    const int lb = j * kBlocksPerTile + lane;
+    return (lane < kBlocksPerTile && lb < nb) ? __ldg(trow + lb) : -1;
+  };
+  // Warp 0: issue the TMA loads of K/V tile j into stage st.
+  auto issue_tile = [&](int j, int st, int ids) {
+    const uint32_t kdst = sb + kStageOff + 2u * st * kTile;
+    const uint32_t vdst = kdst + kTile;
+    const uint32_t bar = bar_kv0 + 8u * st;
+    uint32_t bytes = 0;
+    int idv[kBlocksPerTile];
+#pragma unroll
+    for (int bi = 0; bi < kBlocksPerTile; ++bi) {
+      idv[bi] = __shfl_sync(kFullMask, ids, bi);
+      const int lb = j * kBlocksPerTile + bi;
+      if (lb < nb) {
+        if (static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
+          bytes += 4u * 64u * BS * 2u;
+        else if (lane == 0)
+          raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
+      }
+    }
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      if (bytes == 0) {
+        mbar_arrive(bar);
+      } else {
+        mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+        for (int bi = 0; bi < kBlocksPerTile; ++bi) {
+          const int id = idv[bi];
+          const int lb = j * kBlocksPerTile + bi;
+          if (lb < nb && static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks)) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const uint32_t off = c * kChunk + bi * BS * 128u;
+              tma_load_4d(kdst + off, &tm_k, bar, c * 64, 0, g, id, policy);
+              tma_load_4d(vdst + off, &tm_v, bar, c * 64, 0, g, id, policy);
+            }
+          }
+        }
+      }
+    }
+  };
+
+  // ---- prologue: Q tile, K/V tiles 0 and 1 --------------------------------
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, kTile);
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+        tma_load_3d(sb + kQOff + c * kChunk, &tm_q, bar_q, c * 64, g * G, t_begin + tok0, policy);
+    }
+    const int ids0 = tile_ids(0);
+    issue_tile(0, 0, ids0);
+    if (ntiles > 1) issue_tile(1, 1, tile_ids(1));
+  }
+  int next_ids = (warp == 0 && ntiles > 2) ? tile_ids(2) : -1;
+  int issued = ntiles > 1 ? 2 : 1;  // K/V tiles whose loads were issued (uniform)
+
+  constexpr uint32_t kIdescS = tc::idesc_f16(std::is_same<T, __nv_bfloat16>::value, false, 128, 128);
+  constexpr uint32_t kIdescO = tc::idesc_f16(std::is_same<T, __nv_bfloat16>::value, true, 128, 128);
+
+  float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
+  float l_sum = 0.f;
+  bool ok = cta_wait(bar_q, 0);
+  int j = 0;
+  int o_issued = 0;  // PV products issued (for the final / error waits)
+  for (; ok && j < ntiles; ++j) {
+    const int st = j & 1;
+    const uint32_t kbase = sb + kStageOff + 2u * st * kTile;
+    const uint32_t vbase = kbase + kTile;
+    if (!(ok = cta_wait(bar_kv0 + 8u * st, (j >> 1) & 1))) break;
+    // Tokens past the context in this tile: zero their V rows, so that P = 0
+    // never meets a NaN in stale shared memory.
+    const int valid_tok = min(kKv, L - j * kKv);
+    if (valid_tok < kKv) {
+      uint4 *v4 = reinterpret_cast<uint4 *>(smem + (vbase - sb));
+      const int first = valid_tok * 8;  // 16-byte units per 128-byte row: 8
+      for (int u = first + tid; u < kKv * 8; u += kThreads) {
+        v4[u] = make_uint4(0u, 0u, 0u, 0u);
+        v4[kChunk / 16 + u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- S = Q K^T ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int k = 0; k < kDim / 16; ++k) {
+        const uint32_t koff = (k >> 2) * kChunk + (k & 3) * 32u;
+        tc::mma_f16_ss(tS, tc::smem_desc_sw128(sb + kQOff + koff, 16u, 1024u),
+                       tc::smem_desc_sw128(kbase + koff, 16u, 1024u), kIdescS, k > 0 ? 1u : 0u);
+      }
+      tc::commit(bar_s);
+    }
+    if (!(ok = cta_wait(bar_s, j & 1))) break;
+    tc::fence_after_sync();
+    // ---- softmax on this thread's row ----
+    float x[kKv];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t r[32];
+      tc::ld_32x32b_x32(tS + lane_off + cc * 32, r);
+      tc::wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]);
+    }
+    const int kpos0 = j * kKv;
+    const int lim = min(p_row + 1, L) - kpos0;  // columns < lim are visible
+    float mt = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kKv; ++c) {
+      x[c] = c < lim ? x[c] * a.scale_log2 : -INFINITY;
+      mt = fmaxf(mt, x[c]);
+    }
+    // previous P.V done: P memory and O are free
+    if (j > 0) {
+      if (!(ok = cta_wait(bar_o, (j - 1) & 1))) break;
+      tc::fence_after_sync();
+    }
+    if (j >= 1 && j + 1 < ntiles) {
+      if (warp == 0) {
+        issue_tile(j + 1, (j + 1) & 1, next_ids);
+        next_ids = j + 2 < ntiles ? tile_ids(j + 2) : -1;
+      }
+      ++issued;
+    }
+    const bool move = mt > m_ref + kLazyRescale;
+    float alpha = 1.f;
+    if (move) {
+      alpha = fast_exp2(m_ref - mt);  // 0 while m_ref is -inf
+      m_ref = mt;
+      l_sum *= alpha;
+    }
+    if (j > 0 && __any_sync(kFullMask, move)) {
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tc::ld_32x32b_x32(tO + lane_off + cc * 32, r);
+        tc::wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        tc::st_32x32b_x32(tO + lane_off + cc * 32, r);
+      }
+      tc::wait_st();
+    }
+    // ---- P to shared memory (K-major, 128-byte swizzle) ----
+    {
+      uint8_t *prow = smem + kPOff + tid * 128;
+#pragma unroll
+      for (int u = 0; u < kKv / 8; ++u) {  // 16 units of 8 tokens
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = fast_exp2(x[u * 8 + 2 * e] - m_ref);
+          const float p1 = fast_exp2(x[u * 8 + 2 * e + 1] - m_ref);
+          l_sum += p0 + p1;
+          hi[e] = Pack<T>::pack(p0, p1);
+          if constexpr (kSplit) {
+            const float2 f = Pack<T>::unpack(hi[e]);
+            lo[e] = Pack<T>::pack(p0 - f.x, p1 - f.y);
+          }
+        }
+        const uint32_t off = (u >> 3) * kChunk + ((((u & 7) ^ (tid & 7))) << 4);
+        *reinterpret_cast<uint4 *>(prow + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        if constexpr (kSplit)
+          *reinterpret_cast<uint4 *>(prow + kTile + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- O += P V ----
+    if (tid == 0) {
+      tc::fence_after_sync();
+#pragma unroll
+      for (int k = 0; k < kKv / 16; ++k) {
+        const uint32_t poff = (k >> 2) * kChunk + (k & 3) * 32u;
+        const uint64_t vdesc = tc::smem_desc_sw128(vbase + k * 2048u, kChunk, 1024u);
+        tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + poff, 16u, 1024u), vdesc, kIdescO,
+                       (j > 0 || k > 0) ? 1u : 0u);
+        if constexpr (kSplit)
+          tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + kTile + poff, 16u, 1024u), vdesc,
+                         kIdescO, 1u);
+      }
+      tc::commit(bar_o);
+    }
+    ++o_issued;
+  }
+
+  if (ok && o_issued > 0) ok = cta_wait(bar_o, (o_issued - 1) & 1);
+  if (ok) {
+    tc::fence_after_sync();
+    const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+    T *orow = static_cast<T *>(a.out) +
+              (static_cast<size_t>(t_begin + t_row) * a.num_q_heads + g * G + h_row) * kDim;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t r[32];
+      tc::ld_32x32b_x32(tO + lane_off + cc * 32, r);
+      tc::wait_ld();
+      if (row_valid) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 v;
+          v.x = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 0]) * inv, __uint_as_float(r[q4 * 8 + 1]) * inv);
+          v.y = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 2]) * inv, __uint_as_float(r[q4 * 8 + 3]) * inv);
+          v.z = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 4]) * inv, __uint_as_float(r[q4 * 8 + 5]) * inv);
+          v.w = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 6]) * inv, __uint_as_float(r[q4 * 8 + 7]) * inv);
+          *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) = v;
+        }
+      }
+    }
+  } else {
+    if (tid == 0) {
+      raise_flag(a.d_status, PKV_DEV_TIMEOUT);
+      tc::commit(bar_done);  // arrives once all issued tensor-core work is done
+    }
+    (void)mbar_wait(bar_done, 0);
+    // and the K/V loads still in flight land before shared memory is released
+    for (int t = j; t < issued; ++t) (void)mbar_wait(bar_kv0 + 8u * (t & 1), (t >> 1) & 1);
+    (void)mbar_wait(bar_q, 0);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <typename T>
+pkv_status launch_prefill_bs(int block_size, dim3 grid, const CUtensorMap &tq, const CUtensorMap &tk,
+                             const CUtensorMap &tv, const PrefillArgs &args, cudaStream_t stream) {
+#define PKV_PREFILL_CASE(BSV)                                                               \
+  case BSV: {                                                                               \
+    auto kern = paged_prefill_kernel<T, BSV>;                                               \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
+                             PrefillTune<T>::kSmem) != cudaSuccess)                         \
+      return PKV_ERR_CUDA;                                                                  \
+    kern<<<grid, kThreads, PrefillTune<T>::kSmem, stream>>>(tq, tk, tv, args);              \
+    return launch_status();                                                                 \
+  }
+  switch (block_size) {
+    PKV_PREFILL_CASE(8)
+    PKV_PREFILL_CASE(16)
+    PKV_PREFILL_CASE(32)
+    PKV_PREFILL_CASE(64)
+  }
+#undef PKV_PREFILL_CASE
+  return PKV_ERR_BAD_SHAPE;
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void *k_cache,
+                                        const void *v_cache, pkv_cache_desc cache,
+                                        const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                        const int32_t *query_start, const int32_t *context_lens,
+                                        int32_t num_seqs, int32_t num_tokens,
+                                        int32_t max_query_len, int32_t num_q_heads, float scale,
+                                        int32_t *d_status, pkv_stream_t stream) {
+  using namespace pkv;
+  pkv_status st = check_cache_desc(cache);
+  if (st != PKV_OK) return st;
+  if (!is_16bit(cache.dtype)) return PKV_ERR_BAD_DTYPE;
+  if (cache.head_dim != kDim) return PKV_ERR_BAD_SHAPE;
+  if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_q_heads < 1 ||
+      max_blocks_per_seq < 1)
+    return PKV_ERR_BAD_SHAPE;
+  if (num_q_heads % cache.num_kv_heads != 0) return PKV_ERR_BAD_SHAPE;
+  const int G = num_q_heads / cache.num_kv_heads;
+  if (G > 16 || (kRows % G) != 0) return PKV_ERR_BAD_SHAPE;
+  if (!(scale > 0.f) || !(scale < INFINITY)) return PKV_ERR_BAD_SHAPE;
+  if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
+  if (num_seqs > 65535 || cache.num_kv_heads > 65535) return PKV_ERR_TOO_LARGE;
+  if (!out || !query || !k_cache || !v_cache || !block_tables || !query_start || !context_lens)
+    return PKV_ERR_NULL_POINTER;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(query, 16) || !aligned(out, 16) ||
+      !aligned(block_tables, 4) || !aligned(query_start, 4) || !aligned(context_lens, 4))
+    return PKV_ERR_MISALIGNED;
+  const long long qtiles = (static_cast<long long>(max_query_len) * G + kRows - 1) / kRows;
+  if (qtiles > 2147483647ll) return PKV_ERR_TOO_LARGE;
+  if ((st = check_device()) != PKV_OK) return st;
+
+  CUtensorMap tq, tk, tv;
+  if ((st = encode_query_map(&tq, query, num_tokens, num_q_heads, kDim, G)) != PKV_OK) return st;
+  if ((st = encode_cache_map(&tk, k_cache, cache)) != PKV_OK) return st;
+  if ((st = encode_cache_map(&tv, v_cache, cache)) != PKV_OK) return st;
+
+  PrefillArgs args{};
+  args.out = out;
+  args.block_tables = block_tables;
+  args.query_start = query_start;
+  args.context_lens = context_lens;
+  args.d_status = d_status;
+  args.num_tokens = num_tokens;
+  args.max_blocks_per_seq = max_blocks_per_seq;
+  args.num_q_heads = num_q_heads;
+  args.group = G;
+  args.num_blocks = cache.num_blocks;
+  args.scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid(static_cast<unsigned>(qtiles), static_cast<unsigned>(cache.num_kv_heads),
+            static_cast<unsigned>(num_seqs));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return cache.dtype == PKV_BF16 ? launch_prefill_bs<__nv_bfloat16>(cache.block_size, grid, tq, tk, tv, args, s)
+                                 : launch_prefill_bs<__half>(cache.block_size, grid, tq, tk, tv, args, s);
+}

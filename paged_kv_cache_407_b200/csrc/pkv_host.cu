@@ -90,6 +90,22 @@ pkv_status encode_bytes(CUtensorMap *map, const void *pool, cuuint32_t rank, con
 }
 }  // namespace
 
+pkv_status encode_query_map(CUtensorMap *map, const void *query, int num_tokens, int num_q_heads,
+                            int head_dim, int group) {
+  auto fn = encoder();
+  if (fn == nullptr) return PKV_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(num_tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(head_dim) * num_q_heads * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  cuuint32_t estride[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void *>(query), dims, strides, box,
+                  estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
+}
+
 // The K tile of (block, kv head) is B rows of D codes.  Token t = b + 2 a + 4 c
 // (b, a in {0, 1}) is addressed through dims (d, b, c, a, block*Hkv + head),
 // so the box lands in shared memory with token t on row b + 2 c + (B/2) a:

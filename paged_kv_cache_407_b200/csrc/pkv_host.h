@@ -39,6 +39,12 @@ pkv_status encode_cache_map(CUtensorMap *map, const void *pool, const pkv_cache_
 pkv_status encode_fp8_k_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
 pkv_status encode_fp8_v_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c);
 
+// Rank-3 tiled map over the queries [T][Hq][D] (16-bit), box 64 x G heads x
+// (128 / G) tokens, 128-byte swizzle: one box is 64 columns of a 128-row tile
+// whose row t * G + h is query head g * G + h of token t.
+pkv_status encode_query_map(CUtensorMap *map, const void *query, int num_tokens, int num_q_heads,
+                            int head_dim, int group);
+
 inline pkv_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }

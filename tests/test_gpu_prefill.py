@@ -1,0 +1,86 @@
+"""Paged (chunked) prefill attention on tcgen05 against the oracle (B200
+only): chunks of new tokens are written to the cache, then attend causally
+over their sequences' blocks; every output element is compared with the
+float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.prefill as PO
+import oracle as O
+import paged_kv_cache_407_b200 as pkv
+import workloads as W
+from parity import bits, compare, status_tensor
+from workloads.device import upload_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    assert torch.cuda.is_available(), "these tests need a CUDA device"
+    from paged_kv_cache_407_b200.build import build
+    build()
+    pkv.library()
+
+
+def _run(b, pad_rows=0):
+    db = upload_prefill(b)
+    st = status_tensor()
+    if b.num_tokens:
+        pkv.reshape_and_cache(db.key, db.value, db.k_cache, db.v_cache, db.slot_mapping, d_status=st)
+    q = db.q
+    out = torch.empty_like(q)
+    if pad_rows:
+        q = torch.cat([q, torch.zeros((pad_rows,) + tuple(q.shape[1:]), dtype=q.dtype, device=q.device)])
+        out = torch.full_like(q, 3.0)
+    pkv.paged_prefill(out, q, db.k_cache, db.v_cache, db.block_tables, db.query_start, db.context_lens,
+                      b.max_query_len, b.scale, d_status=st)
+    torch.cuda.synchronize()
+    return out, int(st.item())
+
+
+def _oracle(b):
+    kc, vc = O.reshape_and_cache(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, b.block_size)
+    return PO.paged_prefill(b.q, kc, vc, b.block_tables, b.query_start, b.context_lens, b.block_size, b.scale,
+                            b.dtype)
+
+
+CASES = [
+    # dtype, B, Hq, Hkv, context lengths, chunk lengths
+    (W.F16, 16, 8, 8, [300, 129, 1, 200], [300, 40, 1, 77]),
+    (W.BF16, 32, 32, 8, [700, 260], [200, 260]),
+    (W.F16, 8, 16, 1, [333], [100]),
+    (W.BF16, 64, 16, 8, [1000, 5, 70], [0, 5, 64]),
+    (W.F16, 16, 4, 2, [128, 256, 129], [128, 128, 1]),
+]
+
+
+@pytest.mark.parametrize("dtype,B,Hq,Hkv,lens,chunks", CASES)
+def test_prefill_parity(dtype, B, Hq, Hkv, lens, chunks):
+    b = W.prefill_batch(900 + B + Hq, dtype=dtype, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128, block_size=B,
+                        context_lens=lens, chunk_lens=chunks)
+    out, st = _run(b)
+    assert st == 0
+    compare(bits(out), _oracle(b), dtype, f"prefill {dtype} B{B} {Hq}/{Hkv}")
+
+
+def test_rows_outside_every_chunk_are_not_written():
+    b = W.prefill_batch(77, dtype=W.F16, num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                        context_lens=[90, 40], chunk_lens=[30, 40])
+    out, st = _run(b, pad_rows=5)
+    assert st == 0
+    tail = out[b.num_tokens:].float().cpu().numpy()
+    assert np.all(tail == 3.0)
+    compare(bits(out[: b.num_tokens].contiguous()), _oracle(b), W.F16, "prefill with padding rows")
+
+
+def test_chunk_of_one_token_matches_decode():
+    """A one-token chunk is a decode step: same result as the decode kernel
+    within the tolerance of each against the oracle."""
+    b = W.prefill_batch(78, dtype=W.BF16, num_q_heads=16, num_kv_heads=4, head_dim=128, block_size=16,
+                        context_lens=[513, 64, 1000], chunk_lens=[1, 1, 1])
+    out, st = _run(b)
+    assert st == 0
+    compare(bits(out), _oracle(b), W.BF16, "one-token chunks")

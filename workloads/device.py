@@ -87,3 +87,33 @@ def upload_fp8(f8, device="cuda") -> DeviceFp8Batch:
         cow_pairs=torch.from_numpy(np.ascontiguousarray(b.cow_pairs)).to(device),
         out=torch.empty_like(q),
     )
+
+
+@dataclass
+class DevicePrefillBatch:
+    q: torch.Tensor
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    block_tables: torch.Tensor
+    context_lens: torch.Tensor
+    query_start: torch.Tensor
+    key: torch.Tensor
+    value: torch.Tensor
+    slot_mapping: torch.Tensor
+    out: torch.Tensor
+
+
+def upload_prefill(b, device="cuda") -> DevicePrefillBatch:
+    q = bits_to_tensor(b.q, b.dtype, device)
+    return DevicePrefillBatch(
+        q=q,
+        k_cache=bits_to_tensor(b.k_cache, b.dtype, device),
+        v_cache=bits_to_tensor(b.v_cache, b.dtype, device),
+        block_tables=torch.from_numpy(b.block_tables).to(device),
+        context_lens=torch.from_numpy(b.context_lens).to(device),
+        query_start=torch.from_numpy(b.query_start).to(device),
+        key=bits_to_tensor(b.key, b.dtype, device),
+        value=bits_to_tensor(b.value, b.dtype, device),
+        slot_mapping=torch.from_numpy(b.slot_mapping).to(device),
+        out=torch.empty_like(q),
+    )
