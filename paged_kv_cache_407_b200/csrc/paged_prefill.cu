@@ -7,20 +7,25 @@
 // written to the cache) attends over positions 0..p through the Block Table.
 //
 // One CTA per (128-row query tile, kv head, sequence); a tile row is one
-// (token, query head of the group) pair, so 128 / G tokens per tile.
-//   Q tile  [128 rows][128] by TMA (rank-3 map over [T][Hq][D]);
-//   K, V    128-token tiles gathered block by block through the Block Table
-//           (TMA, rank-4 map over [N][Hkv][B][D]), two stages;
-//   S = Q K^T   tcgen05.mma 128x128x128 into tensor memory (columns 0..127);
-//   softmax     one thread per row (tcgen05.ld of its TMEM lane), causal
-//               mask, running max with lazy rescaling (the reference max
-//               moves only when the row max grows by more than 2^8);
-//   P           written to shared memory (fp16, or bf16 high + bf16 residual
-//               for bf16 operands, which alone would round P by 2^-9);
-//   O += P V    tcgen05.mma 128x128x128 into tensor memory (columns
-//               128..255), V as an MN-major operand.
-// Every wait is bounded; on a timeout the CTA raises PKV_DEV_TIMEOUT, waits
-// (bounded) for its outstanding tensor-core work and frees its TMEM.
+// (token, query head of the group) pair, so 128 / G tokens per tile.  Roles
+// (warp-specialised, synchronised only through mbarriers):
+//   warps 0-3  softmax, one thread per row: tcgen05.ld of its TMEM lane of S,
+//              causal mask, running max with lazy rescaling (the reference
+//              max moves only when the row max grows by more than 2^8; then
+//              the row of O in TMEM is rescaled), P to shared memory (fp16,
+//              or bf16 high + bf16 residual, since bf16 alone would round P
+//              by 2^-9), finally O / l to the output;
+//   warp 4     TMA: the Q tile (rank-3 map over [T][Hq][D]) and the K tiles,
+//              128 tokens gathered block by block through the Block Table
+//              (rank-4 map over [N][Hkv][B][D]), two stages;
+//   warp 5     TMA: the V tiles, two stages;
+//   warp 6     tcgen05.mma, one thread: S(j) = Q K(j)^T (128x128x128) into
+//              one of two TMEM buffers, O += P(j) V(j) (V MN-major) into TMEM,
+//              in the order S(0), S(1), PV(0), S(2), PV(1), ... so that S(j+1)
+//              and P V(j-1) run on the tensor cores during softmax(j).
+// Every wait is bounded; after a timeout every role stops, PKV_DEV_TIMEOUT is
+// raised, outstanding tensor-core work and loads are drained (bounded) and
+// TMEM is freed.
 #include <type_traits>
 
 #include "pkv_device.cuh"
@@ -33,13 +38,19 @@ namespace {
 constexpr int kRows = 128;    // query rows per tile (MMA M)
 constexpr int kKv = 128;      // tokens per K/V tile
 constexpr int kDim = 128;     // head_dim
-constexpr int kThreads = 128;
+constexpr int kSoftmaxWarps = 4;  // warps 0-3: one thread per query row
+constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
+constexpr int kLoadKWarp = 4;     // TMA loads of K tiles (and Q)
+constexpr int kLoadVWarp = 5;     // TMA loads of V tiles
+constexpr int kMmaWarp = 6;       // issues every tcgen05.mma
+constexpr int kThreads = 32 * 7;
 constexpr uint32_t kChunk = 128u * 128u;  // [128 rows][64 elements] of 16-bit: 16 KB
 constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
 constexpr uint32_t kQOff = 0;
-constexpr uint32_t kStageOff = kTile;             // stage st: K at + 2 st kTile, V after it
-constexpr uint32_t kPOff = kStageOff + 4u * kTile;  // P high, then P residual (bf16)
-constexpr uint32_t kTmemCols = 256;               // S: columns [0, 128), O: [128, 256)
+constexpr uint32_t kKOff = kTile;            // two K stages
+constexpr uint32_t kVOff = 3u * kTile;       // two V stages
+constexpr uint32_t kPOff = 5u * kTile;       // P high, then P residual (bf16)
+constexpr uint32_t kTmemCols = 512;          // S buffers: columns [0, 256), O: [256, 384)
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
 
@@ -47,7 +58,7 @@ template <typename T>
 struct PrefillTune {
   static constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
   static constexpr uint32_t kBarOff = kPOff + (kSplit ? 2u : 1u) * kTile;
-  static constexpr uint32_t kSmem = kBarOff + 64u + 1024u;
+  static constexpr uint32_t kSmem = kBarOff + 192u + 1024u;
 };
 
 struct PrefillArgs {
@@ -76,6 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
   using TN = PrefillTune<T>;
   constexpr bool kSplit = TN::kSplit;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int kBlocksPerTile = kKv / BS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -103,199 +115,229 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tok0 = qt * tok_per_tile;
   if (tok0 >= C) return;
   const int last_tok = min(tok0 + tok_per_tile, C) - 1;
-  const int p_max = L - C + last_tok;             // largest position among the tile's rows
-  const int ntiles = (p_max + kKv) / kKv;         // K/V tiles to visit (>= 1)
+  const int p_max = L - C + last_tok;      // largest position among the tile's rows
+  const int ntiles = (p_max + kKv) / kKv;  // K/V tiles to visit (>= 1)
   const int nb = (L + BS - 1) / BS;
 
-  // this thread's row (= TMEM lane)
-  const int t_row = tok0 + tid / G;  // chunk token of the row
-  const int h_row = tid % G;
-  const bool row_valid = t_row < C;
-  const int p_row = L - C + t_row;  // >= L for rows past the chunk
-
-  const uint32_t bar_q = sb + TN::kBarOff;
-  const uint32_t bar_kv0 = bar_q + 8;
-  const uint32_t bar_s = bar_q + 24;
-  const uint32_t bar_o = bar_q + 32;
-  const uint32_t bar_done = bar_q + 40;
-  const uint32_t holder = bar_q + 48;
-  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 48);
+  // ---- barriers (see the role loops for who arrives on which) ------------
+  const uint32_t bars = sb + TN::kBarOff;
+  const uint32_t bar_q = bars;
+  const uint32_t bar_k = bars + 8;        // [2] K stage loaded (TMA bytes)
+  const uint32_t bar_kfree = bars + 24;   // [2] K stage read by S (MMA commit)
+  const uint32_t bar_v = bars + 40;       // [2] V stage loaded
+  const uint32_t bar_vfree = bars + 56;   // [2] V stage read by P V
+  const uint32_t bar_s = bars + 72;       // [2] S buffer written (MMA commit)
+  const uint32_t bar_sfree = bars + 88;   // [2] S buffer read by the 128 softmax threads
+  const uint32_t bar_p = bars + 104;      // P in shared memory, O rescaled (128 threads)
+  const uint32_t bar_o = bars + 112;      // P V done (MMA commit)
+  const uint32_t bar_done = bars + 120;   // drain on the error path
+  const uint32_t holder = bars + 128;
+  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 128);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 132);
 
   if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    mbar_init(bar_kv0, 1);
-    mbar_init(bar_kv0 + 8, 1);
-    mbar_init(bar_s, 1);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_k + 8 * i, 1);
+      mbar_init(bar_kfree + 8 * i, 1);
+      mbar_init(bar_v + 8 * i, 1);
+      mbar_init(bar_vfree + 8 * i, 1);
+      mbar_init(bar_s + 8 * i, 1);
+      mbar_init(bar_sfree + 8 * i, kSoftmaxThreads);
+    }
+    mbar_init(bar_p, kSoftmaxThreads);
     mbar_init(bar_o, 1);
     mbar_init(bar_done, 1);
+    *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tensormap(&tm_q);
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *holder_ptr;
-  const uint32_t tS = tmem;
-  const uint32_t tO = tmem + 128;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tO = tmem + 2 * kKv;
 
-  const uint64_t policy = l2_evict_first_policy();
-  const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
-  // Block ids of K/V tile j: lane i of warp 0 holds block i of the tile.
-  auto tile_ids = [&](int j) -> int {
-    const int lb = j * kBlocksPerTile + lane;
-    return (lane < kBlocksPerTile && lb < nb) ? __ldg(trow + lb) : -1;
+  // A wait that gives up after ~1 s (then every role stops).
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(bar, parity)) return true;
+    *abort_flag = 1;
+    return false;
   };
-  // Warp 0: issue the TMA loads of K/V tile j into stage st.
-  auto issue_tile = [&](int j, int st, int ids) {
-    const uint32_t kdst = sb + kStageOff + 2u * st * kTile;
-    const uint32_t vdst = kdst + kTile;
-    const uint32_t bar = bar_kv0 + 8u * st;
-    uint32_t bytes = 0;
-    int idv[kBlocksPerTile];
+
+  if (warp == kLoadKWarp || warp == kLoadVWarp) {
+    // ---------------------------------------------------------- producers
+    const bool is_k = warp == kLoadKWarp;
+    const CUtensorMap *map = is_k ? &tm_k : &tm_v;
+    if (lane == 0) prefetch_tensormap(map);
+    if (is_k && lane == 0) {
+      prefetch_tensormap(&tm_q);
+      mbar_arrive_expect_tx(bar_q, kTile);
 #pragma unroll
-    for (int bi = 0; bi < kBlocksPerTile; ++bi) {
-      idv[bi] = __shfl_sync(kFullMask, ids, bi);
-      const int lb = j * kBlocksPerTile + bi;
-      if (lb < nb) {
-        if (static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
-          bytes += 4u * 64u * BS * 2u;
-        else if (lane == 0)
-          raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
-      }
+      for (int c = 0; c < 2; ++c)
+        tma_load_3d(sb + kQOff + c * kChunk, &tm_q, bar_q, c * 64, g * G, t_begin + tok0,
+                    l2_evict_first_policy());
     }
-    if (lane == 0) {
-      fence_proxy_async_smem();
-      if (bytes == 0) {
-        mbar_arrive(bar);
-      } else {
-        mbar_arrive_expect_tx(bar, bytes);
+    const uint64_t policy = l2_evict_first_policy();
+    const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
+    const uint32_t full = is_k ? bar_k : bar_v;
+    const uint32_t empty = is_k ? bar_kfree : bar_vfree;
+    const uint32_t stage0 = sb + (is_k ? kKOff : kVOff);
+    auto ids_of = [&](int j) -> int {
+      const int lb = j * kBlocksPerTile + lane;
+      return (j < ntiles && lane < kBlocksPerTile && lb < nb) ? __ldg(trow + lb) : -1;
+    };
+    int ids = ids_of(0);
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j & 1;
+      const int next = ids_of(j + 1);  // in flight while this tile is issued
+      if (j >= 2 && !wait(empty + 8 * st, ((j - 2) >> 1) & 1)) break;
+      uint32_t bytes = 0;
+      int idv[kBlocksPerTile];
 #pragma unroll
-        for (int bi = 0; bi < kBlocksPerTile; ++bi) {
-          const int id = idv[bi];
-          const int lb = j * kBlocksPerTile + bi;
-          if (lb < nb && static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks)) {
+      for (int bi = 0; bi < kBlocksPerTile; ++bi) {
+        idv[bi] = __shfl_sync(kFullMask, ids, bi);
+        const int lb = j * kBlocksPerTile + bi;
+        if (lb < nb) {
+          if (static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
+            bytes += 2u * 64u * BS * 2u;
+          else if (lane == 0)
+            raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
+        }
+      }
+      if (lane == 0) {
+        const uint32_t bar = full + 8 * st;
+        const uint32_t dst = stage0 + st * kTile;
+        fence_proxy_async_smem();
+        if (bytes == 0) {
+          mbar_arrive(bar);
+        } else {
+          mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              const uint32_t off = c * kChunk + bi * BS * 128u;
-              tma_load_4d(kdst + off, &tm_k, bar, c * 64, 0, g, id, policy);
-              tma_load_4d(vdst + off, &tm_v, bar, c * 64, 0, g, id, policy);
+          for (int bi = 0; bi < kBlocksPerTile; ++bi) {
+            const int lb = j * kBlocksPerTile + bi;
+            if (lb < nb && static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks)) {
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d(dst + c * kChunk + bi * BS * 128u, map, bar, c * 64, 0, g, idv[bi], policy);
             }
           }
         }
       }
+      ids = next;
     }
-  };
-
-  // ---- prologue: Q tile, K/V tiles 0 and 1 --------------------------------
-  if (warp == 0) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, kTile);
+  } else if (warp == kMmaWarp) {
+    // --------------------------------------------------------- MMA issuer
+    constexpr uint32_t kIdescS = tc::idesc_f16(kBf16, false, 128, 128);
+    constexpr uint32_t kIdescO = tc::idesc_f16(kBf16, true, 128, 128);
+    auto issue_s = [&](int j) -> bool {
+      const int b = j & 1;
+      if (!wait(bar_k + 8 * b, (j >> 1) & 1)) return false;
+      if (j >= 2 && !wait(bar_sfree + 8 * b, ((j - 2) >> 1) & 1)) return false;
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint32_t kb = sb + kKOff + b * kTile;
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-        tma_load_3d(sb + kQOff + c * kChunk, &tm_q, bar_q, c * 64, g * G, t_begin + tok0, policy);
-    }
-    const int ids0 = tile_ids(0);
-    issue_tile(0, 0, ids0);
-    if (ntiles > 1) issue_tile(1, 1, tile_ids(1));
-  }
-  int next_ids = (warp == 0 && ntiles > 2) ? tile_ids(2) : -1;
-  int issued = ntiles > 1 ? 2 : 1;  // K/V tiles whose loads were issued (uniform)
-
-  constexpr uint32_t kIdescS = tc::idesc_f16(std::is_same<T, __nv_bfloat16>::value, false, 128, 128);
-  constexpr uint32_t kIdescO = tc::idesc_f16(std::is_same<T, __nv_bfloat16>::value, true, 128, 128);
-
-  float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
-  float l_sum = 0.f;
-  bool ok = cta_wait(bar_q, 0);
-  int j = 0;
-  int o_issued = 0;  // PV products issued (for the final / error waits)
-  for (; ok && j < ntiles; ++j) {
-    const int st = j & 1;
-    const uint32_t kbase = sb + kStageOff + 2u * st * kTile;
-    const uint32_t vbase = kbase + kTile;
-    if (!(ok = cta_wait(bar_kv0 + 8u * st, (j >> 1) & 1))) break;
-    // Tokens past the context in this tile: zero their V rows, so that P = 0
-    // never meets a NaN in stale shared memory.
-    const int valid_tok = min(kKv, L - j * kKv);
-    if (valid_tok < kKv) {
-      uint4 *v4 = reinterpret_cast<uint4 *>(smem + (vbase - sb));
-      const int first = valid_tok * 8;  // 16-byte units per 128-byte row: 8
-      for (int u = first + tid; u < kKv * 8; u += kThreads) {
-        v4[u] = make_uint4(0u, 0u, 0u, 0u);
-        v4[kChunk / 16 + u] = make_uint4(0u, 0u, 0u, 0u);
+        for (int k = 0; k < kDim / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kChunk + (k & 3) * 32u;
+          tc::mma_f16_ss(tmem + b * kKv, tc::smem_desc_sw128(sb + kQOff + koff, 16u, 1024u),
+                         tc::smem_desc_sw128(kb + koff, 16u, 1024u), kIdescS, k > 0 ? 1u : 0u);
+        }
+        tc::commit(bar_s + 8 * b);
+        tc::commit(bar_kfree + 8 * b);
       }
-      fence_proxy_async_smem();
+      __syncwarp();
+      return true;
+    };
+    auto issue_pv = [&](int j) -> bool {
+      const int b = j & 1;
+      if (!wait(bar_v + 8 * b, (j >> 1) & 1)) return false;
+      if (!wait(bar_p, j & 1)) return false;
+      if (lane == 0) {
+        tc::fence_after_sync();
+        const uint32_t vb = sb + kVOff + b * kTile;
+#pragma unroll
+        for (int k = 0; k < kKv / 16; ++k) {
+          const uint32_t poff = (k >> 2) * kChunk + (k & 3) * 32u;
+          const uint64_t vdesc = tc::smem_desc_sw128(vb + k * 2048u, kChunk, 1024u);
+          tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + poff, 16u, 1024u), vdesc, kIdescO,
+                         (j > 0 || k > 0) ? 1u : 0u);
+          if constexpr (kSplit)
+            tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + kTile + poff, 16u, 1024u), vdesc,
+                           kIdescO, 1u);
+        }
+        tc::commit(bar_o);
+        tc::commit(bar_vfree + 8 * b);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool run = wait(bar_q, 0);
+    // order on the tensor pipe: S(0), S(1), PV(0), S(2), PV(1), ...
+    for (int j = 0; run && j < ntiles; ++j) {
+      run = issue_s(j);
+      if (run && j >= 1) run = issue_pv(j - 1);
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    // ---- S = Q K^T ----
-    if (tid == 0) {
+    if (run) issue_pv(ntiles - 1);
+  } else if (warp < kSoftmaxWarps) {
+    // ------------------------------------------------- softmax, row = tid
+    const int t_row = tok0 + tid / G;  // chunk token of the row
+    const int h_row = tid % G;
+    const bool row_valid = t_row < C;
+    const int p_row = L - C + t_row;  // >= L for rows past the chunk
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
+    float l_sum = 0.f;
+    bool run = true;
+    for (int j = 0; run && j < ntiles; ++j) {
+      const int b = j & 1;
+      if (!(run = wait(bar_s + 8 * b, (j >> 1) & 1))) break;
       tc::fence_after_sync();
-#pragma unroll
-      for (int k = 0; k < kDim / 16; ++k) {
-        const uint32_t koff = (k >> 2) * kChunk + (k & 3) * 32u;
-        tc::mma_f16_ss(tS, tc::smem_desc_sw128(sb + kQOff + koff, 16u, 1024u),
-                       tc::smem_desc_sw128(kbase + koff, 16u, 1024u), kIdescS, k > 0 ? 1u : 0u);
-      }
-      tc::commit(bar_s);
-    }
-    if (!(ok = cta_wait(bar_s, j & 1))) break;
-    tc::fence_after_sync();
-    // ---- softmax on this thread's row ----
-    float x[kKv];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t r[32];
-      tc::ld_32x32b_x32(tS + lane_off + cc * 32, r);
-      tc::wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]);
-    }
-    const int kpos0 = j * kKv;
-    const int lim = min(p_row + 1, L) - kpos0;  // columns < lim are visible
-    float mt = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < kKv; ++c) {
-      x[c] = c < lim ? x[c] * a.scale_log2 : -INFINITY;
-      mt = fmaxf(mt, x[c]);
-    }
-    // previous P.V done: P memory and O are free
-    if (j > 0) {
-      if (!(ok = cta_wait(bar_o, (j - 1) & 1))) break;
-      tc::fence_after_sync();
-    }
-    if (j >= 1 && j + 1 < ntiles) {
-      if (warp == 0) {
-        issue_tile(j + 1, (j + 1) & 1, next_ids);
-        next_ids = j + 2 < ntiles ? tile_ids(j + 2) : -1;
-      }
-      ++issued;
-    }
-    const bool move = mt > m_ref + kLazyRescale;
-    float alpha = 1.f;
-    if (move) {
-      alpha = fast_exp2(m_ref - mt);  // 0 while m_ref is -inf
-      m_ref = mt;
-      l_sum *= alpha;
-    }
-    if (j > 0 && __any_sync(kFullMask, move)) {
+      float x[kKv];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t r[32];
-        tc::ld_32x32b_x32(tO + lane_off + cc * 32, r);
+        tc::ld_32x32b_x32(tmem + b * kKv + (lane_off | static_cast<uint32_t>(cc * 32)), r);
         tc::wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-        tc::st_32x32b_x32(tO + lane_off + cc * 32, r);
+        for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]);
       }
-      tc::wait_st();
-    }
-    // ---- P to shared memory (K-major, 128-byte swizzle) ----
-    {
+      tc::fence_before_sync();
+      mbar_arrive(bar_sfree + 8 * b);
+      const int lim = min(p_row + 1, L) - j * kKv;  // columns < lim are visible
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kKv; ++c) {
+        x[c] = c < lim ? x[c] * a.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, x[c]);
+      }
+      // previous P V done: P memory and O are free
+      if (j > 0) {
+        if (!(run = wait(bar_o, (j - 1) & 1))) break;
+        tc::fence_after_sync();
+      }
+      const bool move = mt > m_ref + kLazyRescale;
+      float alpha = 1.f;
+      if (move) {
+        alpha = fast_exp2(m_ref - mt);  // 0 while m_ref is -inf
+        m_ref = mt;
+        l_sum *= alpha;
+      }
+      if (j > 0 && __any_sync(kFullMask, move)) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[32];
+          tc::ld_32x32b_x32(tO + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+          tc::wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tc::st_32x32b_x32(tO + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+        }
+        tc::wait_st();
+      }
+      // P to shared memory (K-major, 128-byte swizzle)
       uint8_t *prow = smem + kPOff + tid * 128;
 #pragma unroll
       for (int u = 0; u < kKv / 8; ++u) {  // 16 units of 8 tokens
@@ -316,63 +358,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (kSplit)
           *reinterpret_cast<uint4 *>(prow + kTile + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-    }
-    fence_proxy_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    // ---- O += P V ----
-    if (tid == 0) {
-      tc::fence_after_sync();
-#pragma unroll
-      for (int k = 0; k < kKv / 16; ++k) {
-        const uint32_t poff = (k >> 2) * kChunk + (k & 3) * 32u;
-        const uint64_t vdesc = tc::smem_desc_sw128(vbase + k * 2048u, kChunk, 1024u);
-        tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + poff, 16u, 1024u), vdesc, kIdescO,
-                       (j > 0 || k > 0) ? 1u : 0u);
-        if constexpr (kSplit)
-          tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + kTile + poff, 16u, 1024u), vdesc,
-                         kIdescO, 1u);
+      // V(j) landed; tokens past the context get zero rows, so that P = 0
+      // never meets a NaN in stale shared memory
+      const int valid_tok = min(kKv, L - j * kKv);
+      if (valid_tok < kKv) {
+        if (!(run = wait(bar_v + 8 * b, (j >> 1) & 1))) break;
+        uint4 *v4 = reinterpret_cast<uint4 *>(smem + kVOff + b * kTile);
+        for (int u = valid_tok * 8 + tid; u < kKv * 8; u += kSoftmaxThreads) {
+          v4[u] = make_uint4(0u, 0u, 0u, 0u);
+          v4[kChunk / 16 + u] = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
-      tc::commit(bar_o);
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(bar_p);
     }
-    ++o_issued;
-  }
-
-  if (ok && o_issued > 0) ok = cta_wait(bar_o, (o_issued - 1) & 1);
-  if (ok) {
-    tc::fence_after_sync();
-    const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    T *orow = static_cast<T *>(a.out) +
-              (static_cast<size_t>(t_begin + t_row) * a.num_q_heads + g * G + h_row) * kDim;
+    if (run) run = wait(bar_o, (ntiles - 1) & 1);
+    if (run) {
+      tc::fence_after_sync();
+      const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      T *orow = static_cast<T *>(a.out) +
+                (static_cast<size_t>(t_begin + t_row) * a.num_q_heads + g * G + h_row) * kDim;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t r[32];
-      tc::ld_32x32b_x32(tO + lane_off + cc * 32, r);
-      tc::wait_ld();
-      if (row_valid) {
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        tc::ld_32x32b_x32(tO + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+        tc::wait_ld();
+        if (row_valid) {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 v;
-          v.x = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 0]) * inv, __uint_as_float(r[q4 * 8 + 1]) * inv);
-          v.y = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 2]) * inv, __uint_as_float(r[q4 * 8 + 3]) * inv);
-          v.z = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 4]) * inv, __uint_as_float(r[q4 * 8 + 5]) * inv);
-          v.w = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 6]) * inv, __uint_as_float(r[q4 * 8 + 7]) * inv);
-          *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) = v;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 v;
+            v.x = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 0]) * inv, __uint_as_float(r[q4 * 8 + 1]) * inv);
+            v.y = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 2]) * inv, __uint_as_float(r[q4 * 8 + 3]) * inv);
+            v.z = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 4]) * inv, __uint_as_float(r[q4 * 8 + 5]) * inv);
+            v.w = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 6]) * inv, __uint_as_float(r[q4 * 8 + 7]) * inv);
+            *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) = v;
+          }
         }
       }
     }
-  } else {
-    if (tid == 0) {
-      raise_flag(a.d_status, PKV_DEV_TIMEOUT);
-      tc::commit(bar_done);  // arrives once all issued tensor-core work is done
-    }
-    (void)mbar_wait(bar_done, 0);
-    // and the K/V loads still in flight land before shared memory is released
-    for (int t = j; t < issued; ++t) (void)mbar_wait(bar_kv0 + 8u * (t & 1), (t >> 1) & 1);
-    (void)mbar_wait(bar_q, 0);
   }
+
+  // ---- teardown -----------------------------------------------------------
   tc::fence_before_sync();
   __syncthreads();
+  if (*abort_flag) {
+    // A wait ran out: report it, let the issued tensor-core work and the
+    // loads still in flight finish (bounded) before TMEM and shared memory
+    // are released.
+    if (tid == 0) raise_flag(a.d_status, PKV_DEV_TIMEOUT);
+    if (warp == kMmaWarp && lane == 0) tc::commit(bar_done);
+    (void)mbar_wait(bar_done, 0);
+    for (int i = 0; i < 2; ++i) {
+      (void)mbar_wait(bar_k + 8 * i, 0);
+      (void)mbar_wait(bar_k + 8 * i, 1);
+      (void)mbar_wait(bar_v + 8 * i, 0);
+      (void)mbar_wait(bar_v + 8 * i, 1);
+    }
+    __syncthreads();
+  }
   if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
