@@ -11,7 +11,11 @@ Default workload: Llama-7B-shaped multi-head decode layer (64 sequences,
 uniform on [128, 2048], pool = needed blocks + 10 %, shuffled).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--kv-dtype auto|e4m3]
+
+Workloads prefill_llama7b and prefill_gqa_chunked time the chunked-prefill
+path instead (cache write of the chunks + tcgen05 prefill attention; metric
+TFLOP/s against the measured bf16 tensor peak).
 
 Under torchrun every rank runs its own batch (weak scaling, seed + rank);
 ranks share no data and the only collectives are the barrier and the max of
@@ -37,7 +41,9 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 
 METRIC = "paged decode attention KV GB/s and tokens/s on 1 B200; % of HBM roofline"
+PREFILL_METRIC = "paged prefill attention TFLOP/s (causal, algorithmic FLOPs) on 1 B200; % of tensor roofline"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/pkv_host.cu",
                   "paged_kv_cache_407_b200/csrc/paged_attention.cu",
@@ -68,14 +74,14 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_peak():
+def measured_peak(key: str = "hbm_gbs"):
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d[key]), "measured"
     except (OSError, KeyError, ValueError):
-        return FALLBACK_HBM_GBS, "fallback"
+        return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
 def profiled_traffic(workload: str, kv_dtype: str = "f16"):
@@ -229,6 +235,45 @@ def oracle_sample_rate(batch, seconds: float, f8=None):
     return b / dt / 1e9, desc, blas_threads(), dt
 
 
+def is_prefill(name: str) -> bool:
+    import workloads as W
+
+    return name in W.PREFILL_WORKLOADS
+
+
+def build_prefill(name: str, rank: int):
+    import workloads as W
+
+    base = {"prefill_llama7b": 6, "prefill_gqa_chunked": 7}[name]
+    return W.PREFILL_WORKLOADS[name](seed=base + 1000 * rank)
+
+
+def oracle_prefill_rate(b, seconds: float):
+    """Time the oracle's prefill on growing samples of one sequence's chunk
+    (its last k tokens) until about ``seconds`` of CPU work; returns
+    (TFLOP/s, description, cores, seconds)."""
+    import oracle.prefill as PO
+    import workloads as W
+    from paged_kv_cache_407_b200 import accounting as A
+
+    L = int(b.context_lens[0])
+    k, spent, flop, done = 1, 0.0, 0.0, 0
+    while spent < seconds and k <= int(b.chunk_lens[0]):
+        sub = W.PrefillBatch(**{**b.__dict__, "q": b.q[b.query_start[1] - k: b.query_start[1]],
+                                "context_lens": b.context_lens[:1], "block_tables": b.block_tables[:1],
+                                "query_start": np.array([0, k], np.int32)})
+        t0 = time.perf_counter()
+        PO.paged_prefill(sub.q, b.k_cache, b.v_cache, sub.block_tables, sub.query_start, sub.context_lens,
+                         b.block_size, b.scale, b.dtype)
+        spent += time.perf_counter() - t0
+        flop += A.prefill_flops([L], [k], b.num_q_heads, b.head_dim)
+        done += k
+        k *= 2
+    desc = (f"oracle prefill (fp64 NumPy) of the last {done} query tokens (in growing slices) of sequence 0 "
+            f"of the {b.name} batch (context {L}), {spent:.1f} s")
+    return flop / spent / 1e12, desc, blas_threads(), spent
+
+
 def build_workload(name: str, rank: int):
     import workloads as W
 
@@ -277,6 +322,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0  # the reference arm runs on rank 0 only
+    if is_prefill(args.workload):
+        return run_reference_prefill(args)
     batch = build_workload(args.workload, 0)
     per_step = max(0.5, args.cpu_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
@@ -301,6 +348,195 @@ def run_reference(args):
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "decode_tokens_per_s": round(value * 1e9 / att["total"] * batch.num_seqs, 2),
     }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def prefill_config(b, n_gpus):
+    return {
+        "workload": b.name, "num_seqs_per_gpu": b.num_seqs, "global_batch": b.num_seqs * n_gpus,
+        "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim,
+        "block_size": b.block_size, "context_len_max": b.max_context_len,
+        "chunk_tokens_per_seq": int(b.max_query_len), "query_tokens_per_step": b.num_tokens,
+        "pool_blocks": int(b.k_cache.shape[0]), "pool_bytes": int(b.k_cache.nbytes * 2),
+        "parallelism": f"dp{n_gpus} (independent sequences per GPU)",
+        "l2": "compute-bound; K/V of a sequence are re-read from L2 by its query tiles",
+    }
+
+
+def run_reference_prefill(args):
+    b = build_prefill(args.workload, 0)
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_prefill_rate(b, per_step)
+    rates, secs, desc, cores = [], 0.0, "", 1
+    for _ in range(args.steps):
+        r, desc, cores, dt = oracle_prefill_rate(b, per_step)
+        rates.append(r)
+        secs += dt
+    value = float(statistics.median(rates))
+    line = {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "config": prefill_config(b, 1),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc + "; each step a bounded sample of this workload"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_prefill(args):
+    """Chunked prefill step: write the chunks' K/V (reshape_and_cache), then
+    paged_prefill; the metric is causal attention FLOPs per second."""
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_407_b200 as pkv
+    from paged_kv_cache_407_b200 import accounting as A
+    from paged_kv_cache_407_b200.build import build
+    from workloads.device import upload_prefill
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    pkv.library()
+    b = build_prefill(args.workload, rank)
+    db = upload_prefill(b, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(q=db.q, out=db.out, key=db.key, value=db.value, slots=db.slot_mapping, tables=db.block_tables,
+             qs=db.query_start, lens=db.context_lens, ev=None):
+        pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=status, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        pkv.paged_prefill(out, q, db.k_cache, db.v_cache, tables, qs, lens, b.max_query_len, b.scale,
+                          d_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        pass
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        wall0 = time.time()
+        t0.record(stream)
+        for i in range(K):
+            step(ev=evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks.mark(wall0, time.time())
+        if world > 1:
+            dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    pre_ms = float(np.mean([x.elapsed_time(y) for x, y in evs]))
+    clock = clocks.summary()
+
+    e2e = None
+    if not args.no_e2e:  # inputs from pinned host memory, output back, every step
+        names = ("q", "key", "value", "slots", "tables", "qs", "lens")
+        srcs = (db.q, db.key, db.value, db.slot_mapping, db.block_tables, db.query_start, db.context_lens)
+        h_in = {n: t.detach().cpu().pin_memory() for n, t in zip(names, srcs)}
+        d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
+        h_out = torch.empty(db.out.shape, dtype=db.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            for n in names:
+                d_in[n].copy_(h_in[n], non_blocking=True)
+            step(q=d_in["q"], out=db.out, key=d_in["key"], value=d_in["value"], slots=d_in["slots"],
+                 tables=d_in["tables"], qs=d_in["qs"], lens=d_in["lens"])
+            h_out.copy_(db.out, non_blocking=True)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = {"ms": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h}
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+    flop = A.prefill_flops(b.context_lens, b.chunk_lens, b.num_q_heads, b.head_dim)
+    (ms_total, pre_max, e2e_ms), (flop_all,) = reduce_across_ranks(
+        [ms_total, pre_ms, e2e["ms"] if e2e else 0.0], [flop], dev)
+    ms_step = ms_total / K
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, cores, _ = oracle_prefill_rate(b, args.cpu_seconds)
+        cpu = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peak("bf16_tflops")
+    achieved = flop / (pre_max * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": round(flop_all / (ms_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": b.dtype,
+        "data": "synthetic (seeded generator, inputs resident in HBM)",
+        "config": prefill_config(b, world),
+        "prefill_tokens_per_s": round(b.num_tokens * world / (ms_step * 1e-3), 1),
+        "prefill_ms_per_call": round(pre_max, 5),
+        "flop_per_step": flop,
+        "bytes_per_step_min": A.prefill_bytes(b.context_lens, b.chunk_lens, b.num_q_heads, b.num_kv_heads,
+                                              b.head_dim),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "paged_prefill (tcgen05, 128x128 tiles)",
+            "achieved": round(achieved, 1), "peak": peak,
+            "peak_source": (f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops; fp16 has the same nominal rate)"
+                            if peak_kind == "measured" else "fallback"),
+            "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "traffic": None,
+        },
+        "clocks": clock,
+        "gpu_launches": 2 * K,
+    }
+    if e2e:
+        line["e2e"] = {"value": round(flop_all / (e2e_ms / K * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_ms / K, 5)}
+    if cpu:
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
     return 0
 
@@ -544,6 +780,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if is_prefill(args.workload):
+        return run_prefill(args)
     return run_ours(args)
 
 

@@ -67,3 +67,23 @@ def block_fragmentation(context_lens, block_size: int) -> float:
     lens = np.asarray(context_lens, dtype=np.int64)
     alloc = ((lens + block_size - 1) // block_size) * block_size
     return float((alloc - lens).sum() / alloc.sum())
+
+
+def prefill_flops(context_lens, chunk_lens, num_q_heads: int, head_dim: int) -> float:
+    """Algorithmic FLOPs of a causal prefill call: the chunk's token at
+    position p attends over p + 1 keys, 2 D FLOPs each for Q K^T and for P V,
+    per query head."""
+    total = 0
+    for L, C in zip(np.asarray(context_lens).tolist(), np.asarray(chunk_lens).tolist()):
+        # sum over p = L - C .. L - 1 of (p + 1)
+        total += (L * (L + 1) - (L - C) * (L - C + 1)) // 2
+    return float(4 * head_dim * num_q_heads * total)
+
+
+def prefill_bytes(context_lens, chunk_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                  elem_bytes: int = 2) -> int:
+    """Bytes a prefill call must move at least once: every context token's K
+    and V, the chunk's queries and outputs."""
+    kv = int(np.sum(context_lens)) * num_kv_heads * head_dim * elem_bytes * 2
+    qo = int(np.sum(chunk_lens)) * num_q_heads * head_dim * elem_bytes * 2
+    return kv + qo

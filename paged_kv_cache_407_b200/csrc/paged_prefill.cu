@@ -38,19 +38,20 @@ namespace {
 constexpr int kRows = 128;    // query rows per tile (MMA M)
 constexpr int kKv = 128;      // tokens per K/V tile
 constexpr int kDim = 128;     // head_dim
-constexpr int kSoftmaxWarps = 4;  // warps 0-3: one thread per query row
+constexpr int kSoftmaxWarps = 8;  // warps 0-7: (query row, token half) per thread
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
-constexpr int kLoadKWarp = 4;     // TMA loads of K tiles (and Q)
-constexpr int kLoadVWarp = 5;     // TMA loads of V tiles
-constexpr int kMmaWarp = 6;       // issues every tcgen05.mma
-constexpr int kThreads = 32 * 7;
+constexpr int kLoadKWarp = 8;     // TMA loads of K tiles (and Q)
+constexpr int kLoadVWarp = 9;     // TMA loads of V tiles
+constexpr int kMmaWarp = 10;      // issues every tcgen05.mma
+constexpr int kThreads = 32 * 11;
+constexpr int kHalf = 64;         // tokens of a K/V tile per softmax half
 constexpr uint32_t kChunk = 128u * 128u;  // [128 rows][64 elements] of 16-bit: 16 KB
 constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
 constexpr uint32_t kQOff = 0;
 constexpr uint32_t kKOff = kTile;            // two K stages
 constexpr uint32_t kVOff = 3u * kTile;       // two V stages
 constexpr uint32_t kPOff = 5u * kTile;       // P high, then P residual (bf16)
-constexpr uint32_t kTmemCols = 512;          // S buffers: columns [0, 256), O: [256, 384)
+constexpr uint32_t kTmemCols = 512;          // S buffers [0, 256), O of half 0 / 1 [256, 512)
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
 
@@ -134,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t holder = bars + 128;
   volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 128);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 132);
+  const uint32_t bar_x = bars + 144;      // softmax halves' final (m, l) exchanged
 
   if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
   if (tid == 0) {
@@ -145,11 +147,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_v + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
       mbar_init(bar_s + 8 * i, 1);
-      mbar_init(bar_sfree + 8 * i, kSoftmaxThreads);
+      mbar_init(bar_sfree + 8 * i, kSoftmaxWarps);
     }
-    mbar_init(bar_p, kSoftmaxThreads);
+    mbar_init(bar_p, kSoftmaxWarps);
     mbar_init(bar_o, 1);
     mbar_init(bar_done, 1);
+    mbar_init(bar_x, kSoftmaxWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -157,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *holder_ptr;
-  const uint32_t tO = tmem + 2 * kKv;
+  const uint32_t tO = tmem + 2 * kKv;  // O of half h at tO + h * kDim
 
   // A wait that gives up after ~1 s (then every role stops).
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
@@ -258,15 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         tc::fence_after_sync();
         const uint32_t vb = sb + kVOff + b * kTile;
+        // O_h += P_h V_h: half h of the tile is P chunk h and V rows 64h..
 #pragma unroll
         for (int k = 0; k < kKv / 16; ++k) {
-          const uint32_t poff = (k >> 2) * kChunk + (k & 3) * 32u;
+          const uint32_t h = k >> 2;
+          const uint32_t poff = h * kChunk + (k & 3) * 32u;
           const uint64_t vdesc = tc::smem_desc_sw128(vb + k * 2048u, kChunk, 1024u);
-          tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + poff, 16u, 1024u), vdesc, kIdescO,
-                         (j > 0 || k > 0) ? 1u : 0u);
+          tc::mma_f16_ss(tO + h * kDim, tc::smem_desc_sw128(sb + kPOff + poff, 16u, 1024u), vdesc,
+                         kIdescO, (j > 0 || (k & 3) > 0) ? 1u : 0u);
           if constexpr (kSplit)
-            tc::mma_f16_ss(tO, tc::smem_desc_sw128(sb + kPOff + kTile + poff, 16u, 1024u), vdesc,
-                           kIdescO, 1u);
+            tc::mma_f16_ss(tO + h * kDim, tc::smem_desc_sw128(sb + kPOff + kTile + poff, 16u, 1024u),
+                           vdesc, kIdescO, 1u);
         }
         tc::commit(bar_o);
         tc::commit(bar_vfree + 8 * b);
@@ -282,12 +287,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (run) issue_pv(ntiles - 1);
   } else if (warp < kSoftmaxWarps) {
-    // ------------------------------------------------- softmax, row = tid
-    const int t_row = tok0 + tid / G;  // chunk token of the row
-    const int h_row = tid % G;
+    // ------------------------------------- softmax, (row, token half) per thread
+    // Each half of the threads runs its own online softmax over its half of
+    // every K/V tile, with its own O accumulator in TMEM; the two partial
+    // states of a row are merged once at the end (split-K identity).
+    const int row = tid & (kRows - 1);
+    const int half = tid >> 7;
+    const int t_row = tok0 + row / G;  // chunk token of the row
+    const int h_row = row % G;
     const bool row_valid = t_row < C;
     const int p_row = L - C + t_row;  // >= L for rows past the chunk
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tOh = tO + half * kDim;
     float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
     float l_sum = 0.f;
     bool run = true;
@@ -295,24 +306,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = j & 1;
       if (!(run = wait(bar_s + 8 * b, (j >> 1) & 1))) break;
       tc::fence_after_sync();
-      float x[kKv];
+      float x[kHalf];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t r[32];
-        tc::ld_32x32b_x32(tmem + b * kKv + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+        tc::ld_32x32b_x32(tmem + b * kKv + (lane_off | static_cast<uint32_t>(half * kHalf + cc * 32)), r);
         tc::wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]);
       }
       tc::fence_before_sync();
-      mbar_arrive(bar_sfree + 8 * b);
-      const int lim = min(p_row + 1, L) - j * kKv;  // columns < lim are visible
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sfree + 8 * b);
+      const int lim = min(p_row + 1, L) - (j * kKv + half * kHalf);  // columns < lim are visible
+      if (lim < kHalf) {
+#pragma unroll
+        for (int c = 0; c < kHalf; ++c) x[c] = c < lim ? x[c] : -INFINITY;
+      }
       float mt = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kKv; ++c) {
-        x[c] = c < lim ? x[c] * a.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[c]);
-      }
+      for (int c = 0; c < kHalf; ++c) mt = fmaxf(mt, x[c]);
+      mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
       // previous P V done: P memory and O are free
       if (j > 0) {
         if (!(run = wait(bar_o, (j - 1) & 1))) break;
@@ -329,23 +343,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
-          tc::ld_32x32b_x32(tO + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+          tc::ld_32x32b_x32(tOh + (lane_off | static_cast<uint32_t>(cc * 32)), r);
           tc::wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tc::st_32x32b_x32(tO + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+          tc::st_32x32b_x32(tOh + (lane_off | static_cast<uint32_t>(cc * 32)), r);
         }
         tc::wait_st();
       }
-      // P to shared memory (K-major, 128-byte swizzle)
-      uint8_t *prow = smem + kPOff + tid * 128;
+      // P of this half to P chunk `half` (K-major, 128-byte swizzle)
+      const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
+      uint8_t *prow = smem + kPOff + half * kChunk + row * 128;
 #pragma unroll
-      for (int u = 0; u < kKv / 8; ++u) {  // 16 units of 8 tokens
+      for (int u = 0; u < kHalf / 8; ++u) {  // 8 units of 8 tokens
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = fast_exp2(x[u * 8 + 2 * e] - m_ref);
-          const float p1 = fast_exp2(x[u * 8 + 2 * e + 1] - m_ref);
+          const float p0 = fast_exp2(fmaf(x[u * 8 + 2 * e], a.scale_log2, -mref));
+          const float p1 = fast_exp2(fmaf(x[u * 8 + 2 * e + 1], a.scale_log2, -mref));
           l_sum += p0 + p1;
           hi[e] = Pack<T>::pack(p0, p1);
           if constexpr (kSplit) {
@@ -353,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             lo[e] = Pack<T>::pack(p0 - f.x, p1 - f.y);
           }
         }
-        const uint32_t off = (u >> 3) * kChunk + ((((u & 7) ^ (tid & 7))) << 4);
+        const uint32_t off = static_cast<uint32_t>((u ^ (row & 7)) << 4);
         *reinterpret_cast<uint4 *>(prow + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         if constexpr (kSplit)
           *reinterpret_cast<uint4 *>(prow + kTile + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -371,28 +386,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc::fence_before_sync();
-      mbar_arrive(bar_p);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p);
     }
     if (run) run = wait(bar_o, (ntiles - 1) & 1);
     if (run) {
       tc::fence_after_sync();
-      const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      // merge the two halves' states of the row; P memory is free now
+      float2 *xch = reinterpret_cast<float2 *>(smem + kPOff);
+      xch[half * kRows + row] = make_float2(m_ref, l_sum);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_x);
+      run = wait(bar_x, 0);
+    }
+    if (run) {
+      const float2 *xch = reinterpret_cast<const float2 *>(smem + kPOff);
+      const float2 o0 = xch[row];
+      const float2 o1 = xch[kRows + row];
+      const float M = fmaxf(o0.x, o1.x);
+      const float w0 = o0.x == -INFINITY ? 0.f : fast_exp2(o0.x - M);
+      const float w1 = o1.x == -INFINITY ? 0.f : fast_exp2(o1.x - M);
+      const float Ls = w0 * o0.y + w1 * o1.y;
+      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+      const float c0 = w0 * inv, c1 = w1 * inv;
+      // this thread writes output columns half*64 .. half*64 + 63
       T *orow = static_cast<T *>(a.out) +
-                (static_cast<size_t>(t_begin + t_row) * a.num_q_heads + g * G + h_row) * kDim;
+                (static_cast<size_t>(t_begin + t_row) * a.num_q_heads + g * G + h_row) * kDim + half * kHalf;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        tc::ld_32x32b_x32(tO + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t r0[32], r1[32];
+        const uint32_t col = static_cast<uint32_t>(half * kHalf + cc * 32);
+        tc::ld_32x32b_x32(tO + (lane_off | col), r0);
+        tc::ld_32x32b_x32(tO + kDim + (lane_off | col), r1);
         tc::wait_ld();
         if (row_valid) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 0]) * inv, __uint_as_float(r[q4 * 8 + 1]) * inv);
-            v.y = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 2]) * inv, __uint_as_float(r[q4 * 8 + 3]) * inv);
-            v.z = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 4]) * inv, __uint_as_float(r[q4 * 8 + 5]) * inv);
-            v.w = Pack<T>::pack(__uint_as_float(r[q4 * 8 + 6]) * inv, __uint_as_float(r[q4 * 8 + 7]) * inv);
-            *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) = v;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              v[e] = c0 * __uint_as_float(r0[q4 * 8 + e]) + c1 * __uint_as_float(r1[q4 * 8 + e]);
+            *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) =
+                make_uint4(Pack<T>::pack(v[0], v[1]), Pack<T>::pack(v[2], v[3]), Pack<T>::pack(v[4], v[5]),
+                           Pack<T>::pack(v[6], v[7]));
           }
         }
       }

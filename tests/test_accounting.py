@@ -41,3 +41,17 @@ def test_fragmentation_under_one_block_per_sequence():
 def test_copy_and_write_bytes():
     assert A.copy_blocks_bytes(128, 8, 16, 128) == 128 * (4 * 8 * 16 * 128 * 2 + 16)
     assert A.reshape_and_cache_bytes(256, 8, 128) == 2 * 256 * 8 * 128 * 2 * 2 + 8 * 256
+
+
+def test_prefill_flops_is_the_causal_count():
+    """Brute force: the chunk token at position p attends over p + 1 keys;
+    Q K^T and P V are 2 D FLOPs per (key, query head) each."""
+    from paged_kv_cache_407_b200 import accounting as A
+    lens, chunks, Hq, D = [10, 7, 300, 1], [10, 3, 17, 1], 6, 64
+    brute = 0
+    for L, C in zip(lens, chunks):
+        for p in range(L - C, L):
+            brute += Hq * (2 * D * (p + 1) + 2 * D * (p + 1))
+    assert A.prefill_flops(lens, chunks, Hq, D) == brute
+    assert A.prefill_flops([4096] * 4, [4096] * 4, 32, 128) == 4 * 4 * 128 * 32 * 4096 * 4097 // 2
+    assert A.prefill_bytes([100], [20], 8, 2, 64) == 100 * 2 * 64 * 2 * 2 + 20 * 8 * 64 * 2 * 2

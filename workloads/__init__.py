@@ -589,3 +589,24 @@ def prefill_batch(seed: int, *, dtype: str, num_q_heads: int, num_kv_heads: int,
         value=np.concatenate(new_v) if T else np.zeros(shape0, np.uint16),
         slot_mapping=np.asarray(slots, dtype=np.int64), seed=seed,
     )
+
+
+def prefill_llama7b(seed: int = 6) -> PrefillBatch:
+    """Llama-7B-shaped multi-head prefill: 4 prompts of 4096 tokens, 32 = 32
+    heads, head_dim 128, 16-token blocks, fp16; the whole prompt is the chunk."""
+    return prefill_batch(seed, dtype=F16, num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=16,
+                         context_lens=[4096] * 4, chunk_lens=[4096] * 4, name="prefill_llama7b")
+
+
+def prefill_gqa_chunked(seed: int = 7) -> PrefillBatch:
+    """Chunked prefill with grouped-query heads: 8 sequences whose 1024-token
+    chunks end 8192-token contexts (7168 tokens already cached), 32 q / 8 kv
+    heads, head_dim 128, 16-token blocks, bf16."""
+    return prefill_batch(seed, dtype=BF16, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                         context_lens=[8192] * 8, chunk_lens=[1024] * 8, name="prefill_gqa_chunked")
+
+
+PREFILL_WORKLOADS = {
+    "prefill_llama7b": prefill_llama7b,
+    "prefill_gqa_chunked": prefill_gqa_chunked,
+}
