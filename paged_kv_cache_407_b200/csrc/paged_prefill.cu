@@ -9,20 +9,24 @@
 // One CTA per (128-row query tile, kv head, sequence); a tile row is one
 // (token, query head of the group) pair, so 128 / G tokens per tile.  Roles
 // (warp-specialised, synchronised only through mbarriers):
-//   warps 0-3  softmax, one thread per row: tcgen05.ld of its TMEM lane of S,
-//              causal mask, running max with lazy rescaling (the reference
-//              max moves only when the row max grows by more than 2^8; then
-//              the row of O in TMEM is rescaled), P to shared memory (fp16,
-//              or bf16 high + bf16 residual, since bf16 alone would round P
-//              by 2^-9), finally O / l to the output;
-//   warp 4     TMA: the Q tile (rank-3 map over [T][Hq][D]) and the K tiles,
+//   warps 0-7  softmax, two threads per row, each owning one 64-token half of
+//              every K/V tile with its own running max, sum and O
+//              accumulator (merged once at the end): tcgen05.ld of its TMEM
+//              lane of S, causal mask, lazy rescaling (the reference max moves
+//              only when the row max grows by more than 2^8; then O_h in TMEM
+//              is rescaled, after P V(j-1) is done), P written back into the
+//              same TMEM columns (fp16, or bf16 high + bf16 residual, since
+//              bf16 alone would round P by 2^-9), finally the merged O / l;
+//   warp 8     TMA: the Q tile (rank-3 map over [T][Hq][D]) and the K tiles,
 //              128 tokens gathered block by block through the Block Table
 //              (rank-4 map over [N][Hkv][B][D]), two stages;
-//   warp 5     TMA: the V tiles, two stages;
-//   warp 6     tcgen05.mma, one thread: S(j) = Q K(j)^T (128x128x128) into
-//              one of two TMEM buffers, O += P(j) V(j) (V MN-major) into TMEM,
-//              in the order S(0), S(1), PV(0), S(2), PV(1), ... so that S(j+1)
-//              and P V(j-1) run on the tensor cores during softmax(j).
+//   warp 9     TMA: the V tiles, two stages;
+//   warp 10    tcgen05.mma, one thread: S(j) = Q K(j)^T (128x128x128) into
+//              one of two TMEM buffers; O_h += P_h(j) V_h(j) with P read from
+//              tensor memory (the S buffer) and V from shared memory
+//              (MN-major), in the order S(0), S(1), PV(0), S(2), PV(1), ...; the
+//              in-order tensor pipe finishes P V(j) before S(j+2) reuses the
+//              buffer.
 // Every wait is bounded; after a timeout every role stops, PKV_DEV_TIMEOUT is
 // raised, outstanding tensor-core work and loads are drained (bounded) and
 // TMEM is freed.
@@ -50,7 +54,7 @@ constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
 constexpr uint32_t kQOff = 0;
 constexpr uint32_t kKOff = kTile;            // two K stages
 constexpr uint32_t kVOff = 3u * kTile;       // two V stages
-constexpr uint32_t kPOff = 5u * kTile;       // P high, then P residual (bf16)
+constexpr uint32_t kXOff = 5u * kTile;       // final (m, l) exchange of the softmax halves
 constexpr uint32_t kTmemCols = 512;          // S buffers [0, 256), O of half 0 / 1 [256, 512)
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
@@ -58,7 +62,7 @@ constexpr uint32_t kFullMask = 0xffffffffu;
 template <typename T>
 struct PrefillTune {
   static constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
-  static constexpr uint32_t kBarOff = kPOff + (kSplit ? 2u : 1u) * kTile;
+  static constexpr uint32_t kBarOff = kXOff + 2u * kRows * 8u;
   static constexpr uint32_t kSmem = kBarOff + 192u + 1024u;
 };
 
@@ -128,7 +132,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_v = bars + 40;       // [2] V stage loaded
   const uint32_t bar_vfree = bars + 56;   // [2] V stage read by P V
   const uint32_t bar_s = bars + 72;       // [2] S buffer written (MMA commit)
-  const uint32_t bar_sfree = bars + 88;   // [2] S buffer read by the 128 softmax threads
   const uint32_t bar_p = bars + 104;      // P in shared memory, O rescaled (128 threads)
   const uint32_t bar_o = bars + 112;      // P V done (MMA commit)
   const uint32_t bar_done = bars + 120;   // drain on the error path
@@ -147,7 +150,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_v + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
       mbar_init(bar_s + 8 * i, 1);
-      mbar_init(bar_sfree + 8 * i, kSoftmaxWarps);
     }
     mbar_init(bar_p, kSoftmaxWarps);
     mbar_init(bar_o, 1);
@@ -238,7 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_s = [&](int j) -> bool {
       const int b = j & 1;
       if (!wait(bar_k + 8 * b, (j >> 1) & 1)) return false;
-      if (j >= 2 && !wait(bar_sfree + 8 * b, ((j - 2) >> 1) & 1)) return false;
       if (lane == 0) {
         tc::fence_after_sync();
         const uint32_t kb = sb + kKOff + b * kTile;
@@ -261,17 +262,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         tc::fence_after_sync();
         const uint32_t vb = sb + kVOff + b * kTile;
-        // O_h += P_h V_h: half h of the tile is P chunk h and V rows 64h..
+        // O_h += P_h V_h: P_h sits in the S buffer's columns of half h
+        // (high part in its first 32 columns, bf16 residual in the next 32),
+        // V_h is V rows 64h .. 64h + 63.
 #pragma unroll
         for (int k = 0; k < kKv / 16; ++k) {
           const uint32_t h = k >> 2;
-          const uint32_t poff = h * kChunk + (k & 3) * 32u;
+          const uint32_t pcol = tmem + b * kKv + h * kHalf + (k & 3) * 8u;
           const uint64_t vdesc = tc::smem_desc_sw128(vb + k * 2048u, kChunk, 1024u);
-          tc::mma_f16_ss(tO + h * kDim, tc::smem_desc_sw128(sb + kPOff + poff, 16u, 1024u), vdesc,
-                         kIdescO, (j > 0 || (k & 3) > 0) ? 1u : 0u);
-          if constexpr (kSplit)
-            tc::mma_f16_ss(tO + h * kDim, tc::smem_desc_sw128(sb + kPOff + kTile + poff, 16u, 1024u),
-                           vdesc, kIdescO, 1u);
+          tc::mma_f16_ts(tO + h * kDim, pcol, vdesc, kIdescO, (j > 0 || (k & 3) > 0) ? 1u : 0u);
+          if constexpr (kSplit) tc::mma_f16_ts(tO + h * kDim, pcol + 32u, vdesc, kIdescO, 1u);
         }
         tc::commit(bar_o);
         tc::commit(bar_vfree + 8 * b);
@@ -315,9 +315,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]);
       }
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree + 8 * b);
       const int lim = min(p_row + 1, L) - (j * kKv + half * kHalf);  // columns < lim are visible
       if (lim < kHalf) {
 #pragma unroll
@@ -327,11 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < kHalf; ++c) mt = fmaxf(mt, x[c]);
       mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
-      // previous P V done: P memory and O are free
-      if (j > 0) {
-        if (!(run = wait(bar_o, (j - 1) & 1))) break;
-        tc::fence_after_sync();
-      }
       const bool move = mt > m_ref + kLazyRescale;
       float alpha = 1.f;
       if (move) {
@@ -340,6 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_sum *= alpha;
       }
       if (j > 0 && __any_sync(kFullMask, move)) {
+        // O_h must hold P V(j-1) before it is rescaled
+        if (!(run = wait(bar_o, (j - 1) & 1))) break;
+        tc::fence_after_sync();
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
@@ -351,16 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::wait_st();
       }
-      // P of this half to P chunk `half` (K-major, 128-byte swizzle)
+      // P of this half into the S buffer's columns of the half (A operand of
+      // P V in tensor memory): high part, then the bf16 residual
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
-      uint8_t *prow = smem + kPOff + half * kChunk + row * 128;
+      {
+        uint32_t hi[32], lo[32];
 #pragma unroll
-      for (int u = 0; u < kHalf / 8; ++u) {  // 8 units of 8 tokens
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = fast_exp2(fmaf(x[u * 8 + 2 * e], a.scale_log2, -mref));
-          const float p1 = fast_exp2(fmaf(x[u * 8 + 2 * e + 1], a.scale_log2, -mref));
+        for (int e = 0; e < kHalf / 2; ++e) {
+          const float p0 = fast_exp2(fmaf(x[2 * e], a.scale_log2, -mref));
+          const float p1 = fast_exp2(fmaf(x[2 * e + 1], a.scale_log2, -mref));
           l_sum += p0 + p1;
           hi[e] = Pack<T>::pack(p0, p1);
           if constexpr (kSplit) {
@@ -368,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             lo[e] = Pack<T>::pack(p0 - f.x, p1 - f.y);
           }
         }
-        const uint32_t off = static_cast<uint32_t>((u ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4 *>(prow + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        if constexpr (kSplit)
-          *reinterpret_cast<uint4 *>(prow + kTile + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        const uint32_t pcol = tmem + b * kKv + half * kHalf;
+        tc::st_32x32b_x32(pcol + lane_off, hi);
+        if constexpr (kSplit) tc::st_32x32b_x32(pcol + 32u + lane_off, lo);
+        tc::wait_st();
       }
       // V(j) landed; tokens past the context get zero rows, so that P = 0
       // never meets a NaN in stale shared memory
@@ -384,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           v4[kChunk / 16 + u] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();
+      if (valid_tok < kKv) fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p);
@@ -392,15 +386,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (run) run = wait(bar_o, (ntiles - 1) & 1);
     if (run) {
       tc::fence_after_sync();
-      // merge the two halves' states of the row; P memory is free now
-      float2 *xch = reinterpret_cast<float2 *>(smem + kPOff);
+      // merge the two halves' states of the row
+      float2 *xch = reinterpret_cast<float2 *>(smem + kXOff);
       xch[half * kRows + row] = make_float2(m_ref, l_sum);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_x);
       run = wait(bar_x, 0);
     }
     if (run) {
-      const float2 *xch = reinterpret_cast<const float2 *>(smem + kPOff);
+      const float2 *xch = reinterpret_cast<const float2 *>(smem + kXOff);
       const float2 o0 = xch[row];
       const float2 o1 = xch[kRows + row];
       const float M = fmaxf(o0.x, o1.x);
