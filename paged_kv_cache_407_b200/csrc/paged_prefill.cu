@@ -101,7 +101,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int qt = blockIdx.x;
+  // Query tiles launch last-first: later tiles see more keys (causal), so
+  // the longest CTAs start first and the short ones fill the tail.
+  const int qt = gridDim.x - 1 - blockIdx.x;
   const int g = blockIdx.y;
   const int s = blockIdx.z;
   const int G = a.group;
