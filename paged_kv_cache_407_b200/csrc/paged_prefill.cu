@@ -309,22 +309,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(run = wait(bar_s + 8 * b, (j >> 1) & 1))) break;
       tc::fence_after_sync();
       float x[kHalf];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t r[32];
-        tc::ld_32x32b_x32(tmem + b * kKv + (lane_off | static_cast<uint32_t>(half * kHalf + cc * 32)), r);
+      {
+        uint32_t r0[32], r1[32];  // both loads in flight, one wait
+        const uint32_t col = tmem + b * kKv + (lane_off | static_cast<uint32_t>(half * kHalf));
+        tc::ld_32x32b_x32(col, r0);
+        tc::ld_32x32b_x32(col + 32u, r1);
         tc::wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(r0[i]);
+          x[32 + i] = __uint_as_float(r1[i]);
+        }
       }
       const int lim = min(p_row + 1, L) - (j * kKv + half * kHalf);  // columns < lim are visible
       if (lim < kHalf) {
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) x[c] = c < lim ? x[c] : -INFINITY;
       }
-      float mt = -INFINITY;
+      float mp[8];  // eight independent partial maxima
 #pragma unroll
-      for (int c = 0; c < kHalf; ++c) mt = fmaxf(mt, x[c]);
+      for (int i = 0; i < 8; ++i) mp[i] = x[i];
+#pragma unroll
+      for (int c = 8; c < kHalf; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
+      float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
       const bool move = mt > m_ref + kLazyRescale;
       float alpha = 1.f;
@@ -338,13 +346,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(run = wait(bar_o, (j - 1) & 1))) break;
         tc::fence_after_sync();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t r[32];
-          tc::ld_32x32b_x32(tOh + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+        for (int cc = 0; cc < 4; cc += 2) {
+          uint32_t r0[32], r1[32];
+          const uint32_t col = tOh + (lane_off | static_cast<uint32_t>(cc * 32));
+          tc::ld_32x32b_x32(col, r0);
+          tc::ld_32x32b_x32(col + 32u, r1);
           tc::wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tc::st_32x32b_x32(tOh + (lane_off | static_cast<uint32_t>(cc * 32)), r);
+          for (int i = 0; i < 32; ++i) {
+            r0[i] = __float_as_uint(__uint_as_float(r0[i]) * alpha);
+            r1[i] = __float_as_uint(__uint_as_float(r1[i]) * alpha);
+          }
+          tc::st_32x32b_x32(col, r0);
+          tc::st_32x32b_x32(col + 32u, r1);
         }
         tc::wait_st();
       }
@@ -353,17 +367,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
       {
         uint32_t hi[32], lo[32];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
         for (int e = 0; e < kHalf / 2; ++e) {
           const float p0 = fast_exp2(fmaf(x[2 * e], a.scale_log2, -mref));
           const float p1 = fast_exp2(fmaf(x[2 * e + 1], a.scale_log2, -mref));
-          l_sum += p0 + p1;
+          ls[e & 3] += p0 + p1;
           hi[e] = Pack<T>::pack(p0, p1);
           if constexpr (kSplit) {
             const float2 f = Pack<T>::unpack(hi[e]);
             lo[e] = Pack<T>::pack(p0 - f.x, p1 - f.y);
           }
         }
+        l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         const uint32_t pcol = tmem + b * kKv + half * kHalf;
         tc::st_32x32b_x32(pcol + lane_off, hi);
         if constexpr (kSplit) tc::st_32x32b_x32(pcol + 32u + lane_off, lo);

@@ -84,3 +84,41 @@ def test_chunk_of_one_token_matches_decode():
     out, st = _run(b)
     assert st == 0
     compare(bits(out), _oracle(b), W.BF16, "one-token chunks")
+
+
+def test_bad_lengths_and_block_ids_are_flagged_not_faulted():
+    """A sequence whose chunk is longer than its context is skipped with
+    PKV_DEV_BAD_LEN (its rows untouched); a Block Table entry outside the
+    pool raises PKV_DEV_BAD_BLOCK.  The other sequences are still exact."""
+    b = W.prefill_batch(79, dtype=W.F16, num_q_heads=8, num_kv_heads=4, head_dim=128, block_size=16,
+                        context_lens=[200, 150, 300], chunk_lens=[40, 50, 60])
+    db = upload_prefill(b)
+    st = status_tensor()
+    pkv.reshape_and_cache(db.key, db.value, db.k_cache, db.v_cache, db.slot_mapping, d_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    lens = db.context_lens.clone()
+    lens[1] = 20  # chunk of 50 tokens in a context of 20
+    out = torch.full_like(db.q, 5.0)
+    pkv.paged_prefill(out, db.q, db.k_cache, db.v_cache, db.block_tables, db.query_start, lens, b.max_query_len,
+                      b.scale, d_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & pkv.DEV_BAD_LEN
+    ref = _oracle(b)
+    got = bits(out)
+    for s in (0, 2):
+        t0, t1 = int(b.query_start[s]), int(b.query_start[s + 1])
+        compare(got[t0:t1], ref[t0:t1], W.F16, f"seq {s}")
+    t0, t1 = int(b.query_start[1]), int(b.query_start[2])
+    assert np.all(out[t0:t1].float().cpu().numpy() == 5.0)
+    st.zero_()
+    tables = db.block_tables.clone()
+    tables[2, 3] = b.k_cache.shape[0] + 7
+    pkv.paged_prefill(out, db.q, db.k_cache, db.v_cache, tables, db.query_start, db.context_lens, b.max_query_len,
+                      b.scale, d_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & pkv.DEV_BAD_BLOCK
+    got = bits(out)
+    for s in (0, 1):
+        t0, t1 = int(b.query_start[s]), int(b.query_start[s + 1])
+        compare(got[t0:t1], ref[t0:t1], W.F16, f"seq {s}")
