@@ -143,10 +143,12 @@ PKV_API size_t pkv_paged_attention_workspace_size(int32_t num_seqs, int32_t num_
 /*
  * pkv_paged_attention_partition_size - the partition size (tokens) that
  * pkv_paged_attention_decode uses for these arguments: partition_size itself
- * when it is non-zero, otherwise the automatic choice (1024 tokens, halved
- * down to 256 while num_seqs * num_kv_heads * ceil(max_context_len / size)
- * stays below 1776, i.e. about 12 work units per SM).  Returns -1 for invalid
- * arguments.  A result >= max_context_len means no sequence is split.
+ * when it is non-zero, otherwise the automatic choice: no split (the result
+ * covers max_context_len) when max_context_len <= 2048 and num_seqs *
+ * num_kv_heads >= 1776 (about 12 work units per SM); else 1024 tokens,
+ * halved down to 256 while num_seqs * num_kv_heads * ceil(max_context_len /
+ * size) stays below 1776.  Returns -1 for invalid arguments.  A result >=
+ * max_context_len means no sequence is split.
  */
 PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num_kv_heads,
                                            int32_t block_size, int32_t max_context_len,

@@ -500,12 +500,18 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-// Automatic partition size: 1024 tokens, halved (down to 256) while the grid
-// would hold fewer than about 12 units per SM of a 148-SM B200, judged from
-// the largest possible batch (every sequence at max_context_len).
+// Automatic partition size.  No split when the (sequence, kv head) units
+// alone give about 12 per SM of a 148-SM B200 and no sequence exceeds 2048
+// tokens (a whole sequence is then at most 128 blocks of 16 per CTA, short
+// next to the call; splitting would only add the merge).  Otherwise 1024
+// tokens, halved (down to 256) while the grid would hold fewer than 12 units
+// per SM, judged from the largest possible batch (every sequence at
+// max_context_len); long sequences are split so that none of them is a tail.
 int auto_part_blocks(int block_size, int num_seqs, int num_kv_heads, int max_context_len) {
-  int tokens = 1024;
   const long long want = 148ll * 12;
+  if (max_context_len <= 2048 && static_cast<long long>(num_seqs) * num_kv_heads >= want)
+    return std::max(1, (max_context_len + block_size - 1) / block_size);
+  int tokens = 1024;
   while (tokens > 256) {
     const long long parts = (max_context_len + tokens - 1) / tokens;
     if (static_cast<long long>(num_seqs) * num_kv_heads * std::max(1ll, parts) >= want) break;

@@ -86,7 +86,10 @@ def test_host_validation_without_device(lib):
 
 def test_workspace_and_partition_queries(lib):
     # automatic partitions of 1024 tokens, smaller when the grid would be thin
-    assert bd.partition_size(64, 32, 16, 2048) == 1024
+    assert bd.partition_size(64, 32, 16, 2048) == 2048  # enough (seq, kv head) units: no split
+    assert bd.partition_size(64, 32, 16, 2035) == 2048
+    assert bd.partition_size(256, 8, 16, 4096) == 1024  # long tail: split
+    assert bd.partition_size(32, 32, 16, 2048) == 1024  # too few units
     assert bd.partition_size(4, 8, 32, 131072) == 1024
     assert bd.partition_size(1, 8, 16, 32768) == 256
     assert bd.partition_size(4, 8, 16, 32768) == 512
