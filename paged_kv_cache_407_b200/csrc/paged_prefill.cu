@@ -80,11 +80,6 @@ struct PrefillArgs {
   float scale_log2;
 };
 
-// Bounded wait by every thread, made uniform over the CTA.
-__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity) {
-  return __syncthreads_and(mbar_wait(bar, parity) ? 1 : 0) != 0;
-}
-
 template <typename T, int BS>
 __global__ void __launch_bounds__(kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
