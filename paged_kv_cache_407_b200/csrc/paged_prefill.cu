@@ -129,12 +129,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_v = bars + 40;       // [2] V stage loaded
   const uint32_t bar_vfree = bars + 56;   // [2] V stage read by P V
   const uint32_t bar_s = bars + 72;       // [2] S buffer written (MMA commit)
-  const uint32_t bar_p = bars + 104;      // P in shared memory, O rescaled (128 threads)
-  const uint32_t bar_o = bars + 112;      // P V done (MMA commit)
-  const uint32_t bar_done = bars + 120;   // drain on the error path
-  const uint32_t holder = bars + 128;
-  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 128);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 132);
+  // P-ready comes one per S buffer: a softmax warp may arrive for tile j+1
+  // before a slower one arrives for tile j, and those arrivals must not
+  // count towards the same phase.
+  const uint32_t bar_p = bars + 104;      // [2] P in TMEM, O rescaled (one arrival per softmax warp)
+  const uint32_t bar_o = bars + 120;      // P V done (MMA commit)
+  const uint32_t bar_done = bars + 128;   // drain on the error path
+  const uint32_t holder = bars + 136;
+  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 136);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 140);
   const uint32_t bar_x = bars + 144;      // softmax halves' final (m, l) exchanged
 
   if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
@@ -147,8 +150,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_v + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
       mbar_init(bar_s + 8 * i, 1);
+      mbar_init(bar_p + 8 * i, kSoftmaxWarps);
     }
-    mbar_init(bar_p, kSoftmaxWarps);
     mbar_init(bar_o, 1);
     mbar_init(bar_done, 1);
     mbar_init(bar_x, kSoftmaxWarps);
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](int j) -> bool {
       const int b = j & 1;
       if (!wait(bar_v + 8 * b, (j >> 1) & 1)) return false;
-      if (!wait(bar_p, j & 1)) return false;
+      if (!wait(bar_p + 8 * b, (j >> 1) & 1)) return false;
       if (lane == 0) {
         tc::fence_after_sync();
         const uint32_t vb = sb + kVOff + b * kTile;
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (valid_tok < kKv) fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p);
+      if (lane == 0) mbar_arrive(bar_p + 8 * b);
     }
     if (run) run = wait(bar_o, (ntiles - 1) & 1);
     if (run) {
