@@ -130,10 +130,11 @@ PKV_API pkv_status pkv_reshape_and_cache(const void *key, const void *value, int
  * pkv_paged_attention_workspace_size - bytes of scratch that
  * pkv_paged_attention_decode needs for these sizes: 0 when no sequence can
  * span more than one partition; otherwise num_seqs * num_kv_heads int32
- * arrival counters (padded to 16 bytes) followed by num_seqs * num_q_heads *
- * max_partitions * (head_dim + 2) floats of partials.  partition_size follows
- * the rules of pkv_paged_attention_decode (0 = automatic).  Returns 0 for
- * invalid sizes.
+ * arrival counters and one int32 unit count (padded to 16 bytes), the plan's
+ * list of num_seqs * max_partitions (sequence, partition) int32 pairs
+ * (padded to 16 bytes), then num_seqs * num_q_heads * max_partitions *
+ * (head_dim + 2) floats of partials.  partition_size follows the rules of
+ * pkv_paged_attention_decode (0 = automatic).  Returns 0 for invalid sizes.
  */
 PKV_API size_t pkv_paged_attention_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                           int32_t num_kv_heads, int32_t head_dim,
@@ -170,8 +171,11 @@ PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num
  * Long contexts are cut into partitions of partition_size tokens; each
  * partition yields (max score, sum of exponentials, unnormalised output) and
  * they are merged by log-sum-exp (by the last partition of each sequence to
- * finish, or by a second kernel for splits of more than 32 partitions).  Arithmetic: fp16/bf16 products,
- * fp32 accumulation and softmax; the output is rounded once to fp16/bf16.
+ * finish, or by a second kernel for splits of more than 32 partitions).  A
+ * call whose longest sequence spans 3 to 32 partitions first runs a one-CTA
+ * planning kernel that lists the non-empty (sequence, partition) units,
+ * largest first, so the attention grid starts the long units first.  Arithmetic: fp16/bf16 products, fp32 accumulation
+ * and softmax; the output is rounded once to fp16/bf16.
  *
  * out              device, [num_seqs][num_q_heads][head_dim], cache dtype.
  * query            device, [num_seqs][num_q_heads][head_dim], cache dtype.

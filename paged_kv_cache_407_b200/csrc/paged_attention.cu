@@ -64,6 +64,8 @@ struct DecodeArgs {
   int max_parts;
   float scale_log2;  // softmax scale * log2(e) (times k_scale for 8-bit pools)
   float out_scale;   // 1, or v_scale for 8-bit pools
+  const int2 *units;           // split calls: (sequence, partition) per unit, longest first
+  const int32_t *unit_count;   // number of units in `units`
 };
 
 // ---------------------------------------------------------------------------
@@ -242,12 +244,16 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap *tmk,
 // Grid kernel: one CTA per (kv head, sequence, partition)
 // ---------------------------------------------------------------------------
 
-// Launch shape: a CTA's rings take about 64 KB so three CTAs fit on an SM.
+// Launch shape: a CTA's rings take about 64 KB so three CTAs fit on an SM
+// (48 KB and four CTAs for 8-bit pools with 32-token blocks).
 template <int D, int BS, int ESZ = 2>
 struct GridTune {
   static constexpr int kStage = 2 * BS * D * ESZ;
-  static constexpr int kWarps = kStage >= 16384 ? 2 : 4;
-  static constexpr int kFit = 65536 / (kWarps * kStage);
+  // 8-bit pools with 32-token blocks: two warps with three stages each (four
+  // CTAs per SM) measured best; four warps spill under the register cap.
+  static constexpr bool kKv8Bs32 = ESZ == 1 && BS == 32;
+  static constexpr int kWarps = kKv8Bs32 ? 2 : (kStage >= 16384 ? 2 : 4);
+  static constexpr int kFit = kKv8Bs32 ? 3 : 65536 / (kWarps * kStage);
   static constexpr int kStages = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
   // Three CTAs per SM fit in shared memory; ask the register allocation for
   // three as well (at most 168 registers with four warps).
@@ -270,9 +276,23 @@ __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMi
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int g = blockIdx.x;
-  const int s = blockIdx.y;
-  const int part = blockIdx.z;
+  // Without a plan: grid (kv head, sequence, partition slot).  With a plan:
+  // one CTA per (unit, kv head) with the kv head fastest; the units come
+  // longest first, so long partitions start early and the unused tail exits
+  // at once.
+  int g, s, part;
+  if (a.units == nullptr) {
+    g = blockIdx.x;
+    s = blockIdx.y;
+    part = blockIdx.z;
+  } else {
+    const int unit = static_cast<int>(blockIdx.x / static_cast<unsigned>(a.num_kv_heads));
+    g = static_cast<int>(blockIdx.x % static_cast<unsigned>(a.num_kv_heads));
+    if (unit >= __ldg(a.unit_count)) return;  // uniform over the CTA
+    const int2 u = __ldg(a.units + unit);
+    s = u.x;
+    part = u.y;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = a.group;
@@ -498,6 +518,68 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
+// Plan of a split call: every non-empty (sequence, partition) unit, ordered
+// by its number of blocks, largest first (a counting sort; the order inside
+// one size is arbitrary and does not change any result, since partitions are
+// merged in partition order).  A sequence without tokens keeps one unit, which
+// writes its zero output.  One CTA; it also zeroes the arrival counters.
+// ---------------------------------------------------------------------------
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 1024;  // unit sizes of 1023 blocks and more share the top bucket
+
+__device__ __forceinline__ int plan_len(const int32_t *lens, int s, int len_limit) {
+  const int len = lens[s];
+  return len < 0 ? 0 : (len > len_limit ? len_limit : len);
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+    decode_plan_kernel(const int32_t *__restrict__ context_lens, int num_seqs, int block_size,
+                       int part_blocks, int max_parts, int len_limit, int2 *__restrict__ units,
+                       int32_t *__restrict__ unit_count, int32_t *__restrict__ counters,
+                       int num_counters) {
+  __shared__ int hist[kPlanBuckets];
+  __shared__ int warp_sums[kPlanThreads / 32];
+  const int tid = threadIdx.x;
+  hist[tid] = 0;
+  for (int i = tid; i < num_counters; i += kPlanThreads) counters[i] = 0;
+  __syncthreads();
+  // candidate units (sequence, partition) in partition-major order, spread
+  // over the threads
+  const long long total = static_cast<long long>(num_seqs) * max_parts;
+  auto for_units = [&](auto &&fn) {
+    for (long long u = tid; u < total; u += kPlanThreads) {
+      const int p = static_cast<int>(u / num_seqs);
+      const int s = static_cast<int>(u - static_cast<long long>(p) * num_seqs);
+      const int nb = (plan_len(context_lens, s, len_limit) + block_size - 1) / block_size;
+      if (p >= parts_of(nb, part_blocks)) continue;
+      const int size = min(part_blocks, nb - p * part_blocks);
+      fn(s, p, min(max(size, 0), kPlanBuckets - 1));
+    }
+  };
+  for_units([&](int, int, int key) { atomicAdd(&hist[key], 1); });
+  __syncthreads();
+  // offsets in descending key order: offs[k] = sum of hist[k'] over k' > k
+  const int key = kPlanBuckets - 1 - tid;  // thread tid scans bucket key
+  const int v = hist[key];
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if ((tid & 31) >= off) incl += t;
+  }
+  if ((tid & 31) == 31) warp_sums[tid >> 5] = incl;
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < (tid >> 5); ++w) base += warp_sums[w];
+  const int excl = base + incl - v;
+  __syncthreads();
+  hist[key] = excl;  // now the next free position of each bucket
+  if (tid == kPlanThreads - 1) *unit_count = base + incl;
+  __syncthreads();
+  for_units([&](int s, int p, int k) { units[atomicAdd(&hist[k], 1)] = make_int2(s, p); });
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 // Automatic partition size.  No split when the (sequence, kv head) units
@@ -525,7 +607,8 @@ bool valid_block_size(int bs) { return bs == 8 || bs == 16 || bs == 32 || bs == 
 struct Plan {
   int part_blocks;
   int max_parts;
-  size_t ctrl_bytes;  // arrival counters, zeroed per call
+  size_t ctrl_bytes;   // arrival counters and the unit count, zeroed per call
+  size_t units_bytes;  // the plan's unit list
   size_t ws_bytes;
 };
 
@@ -550,8 +633,9 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int3
   plan->part_blocks = part_blocks;
   plan->max_parts = static_cast<int>(std::min<long long>(parts, 1ll << 30));
   const bool split = parts > 1 && num_seqs > 0;
-  plan->ctrl_bytes = split ? (static_cast<size_t>(num_seqs) * num_kv_heads * 4 + 15) / 16 * 16 : 0;
-  plan->ws_bytes = plan->ctrl_bytes +
+  plan->ctrl_bytes = split ? (static_cast<size_t>(num_seqs) * num_kv_heads * 4 + 4 + 15) / 16 * 16 : 0;
+  plan->units_bytes = split ? (static_cast<size_t>(num_seqs) * parts * 8 + 15) / 16 * 16 : 0;
+  plan->ws_bytes = plan->ctrl_bytes + plan->units_bytes +
                    (split ? static_cast<size_t>(num_seqs) * num_q_heads * parts *
                                 (static_cast<size_t>(head_dim) + 2) * sizeof(float)
                           : 0);
@@ -566,8 +650,10 @@ pkv_status launch_grid(const CUtensorMap &tmk, const CUtensorMap &tmv, const Dec
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TN::kSmem) !=
       cudaSuccess)
     return PKV_ERR_CUDA;
-  dim3 grid(static_cast<unsigned>(args.num_kv_heads), static_cast<unsigned>(args.num_seqs),
-            static_cast<unsigned>(args.max_parts));
+  dim3 grid = args.units == nullptr
+                  ? dim3(static_cast<unsigned>(args.num_kv_heads), static_cast<unsigned>(args.num_seqs),
+                         static_cast<unsigned>(args.max_parts))
+                  : dim3(static_cast<unsigned>(args.num_kv_heads) * args.num_seqs * args.max_parts);
   kern<<<grid, TN::kWarps * 32, TN::kSmem, stream>>>(tmk, tmv, args);
   return launch_status();
 }
@@ -683,7 +769,9 @@ pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, 
   if (!make_plan(num_seqs, num_q_heads, cache.num_kv_heads, cache.head_dim, cache.block_size,
                  max_context_len, partition_size, &plan))
     return PKV_ERR_BAD_PARTITION;
-  if (plan.max_parts > 65535) return PKV_ERR_TOO_LARGE;
+  if (plan.max_parts > 65535) return PKV_ERR_TOO_LARGE;  // grid z without a plan
+  if (static_cast<long long>(num_seqs) * plan.max_parts * cache.num_kv_heads > 2147483647ll)
+    return PKV_ERR_TOO_LARGE;  // one CTA per (unit, kv head) in a 1-D grid with a plan
   if (plan.ws_bytes > 0) {
     if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return PKV_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return PKV_ERR_MISALIGNED;
@@ -708,8 +796,16 @@ pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   args.counters = reinterpret_cast<int32_t *>(ws);
   const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * plan.max_parts;
-  float *part = plan.ws_bytes ? reinterpret_cast<float *>(ws + plan.ctrl_bytes) : nullptr;
+  float *part = plan.ws_bytes ? reinterpret_cast<float *>(ws + plan.ctrl_bytes + plan.units_bytes) : nullptr;
   const bool split = plan.max_parts > 1;
+  // A plan pays when lengths can be spread over several partitions that the
+  // attention kernel merges itself (3 .. 32); with two partitions every tail
+  // is short, and beyond 32 all sequences are long.
+  const bool use_plan = split && plan.max_parts >= 3 && plan.max_parts <= kFuseMaxParts;
+  // unit count right after the arrival counters, the unit list after that
+  args.unit_count = use_plan ? reinterpret_cast<int32_t *>(ws) + static_cast<size_t>(num_seqs) * cache.num_kv_heads
+                             : nullptr;
+  args.units = use_plan ? reinterpret_cast<const int2 *>(ws + plan.ctrl_bytes) : nullptr;
   args.ws_o = split ? part : nullptr;
   args.ws_m = split ? part + rows * cache.head_dim : nullptr;
   args.ws_l = split ? part + rows * (cache.head_dim + 1) : nullptr;
@@ -728,8 +824,15 @@ pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, 
   args.out_scale = kv8 ? v_scale : 1.f;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (plan.ctrl_bytes > 0 && cudaMemsetAsync(ws, 0, plan.ctrl_bytes, s) != cudaSuccess)
+  if (split && !use_plan && cudaMemsetAsync(ws, 0, plan.ctrl_bytes, s) != cudaSuccess)
     return PKV_ERR_CUDA;
+  if (use_plan) {  // the plan (which also zeroes the arrival counters)
+    decode_plan_kernel<<<1, kPlanThreads, 0, s>>>(
+        context_lens, num_seqs, cache.block_size, plan.part_blocks, plan.max_parts, args.len_limit,
+        reinterpret_cast<int2 *>(ws + plan.ctrl_bytes), const_cast<int32_t *>(args.unit_count),
+        args.counters, num_seqs * cache.num_kv_heads);
+    if ((st = launch_status()) != PKV_OK) return st;
+  }
   const bool big = args.group > 8;
   const bool bf16 = act == PKV_BF16;
   if (kv8)

@@ -99,6 +99,7 @@ def test_workspace_and_partition_queries(lib):
     assert bd.workspace_size(4, 4, 4, 64, 16, 33) == 0
     # 131072 tokens in 512-token partitions: one int32 arrival counter per
     # (seq, kv head), then 256 partials of (D + 2) floats per (seq, head)
-    assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 512) == 4 * 8 * 4 + 4 * 32 * 256 * 130 * 4
-    assert bd.workspace_size(3, 4, 1, 64, 16, 2000, 256) == 16 + 3 * 4 * 8 * 66 * 4
+    # [arrival counters + unit count, 16-byte padded][unit list (int2), padded][partials]
+    assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 512) == 144 + 4 * 256 * 8 + 4 * 32 * 256 * 130 * 4
+    assert bd.workspace_size(3, 4, 1, 64, 16, 2000, 256) == 16 + 3 * 8 * 8 + 3 * 4 * 8 * 66 * 4
     assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 24) == 0  # invalid partition
