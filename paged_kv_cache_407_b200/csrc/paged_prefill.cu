@@ -324,13 +324,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < kHalf; ++c) x[c] = c < lim ? x[c] : -INFINITY;
       }
-      float mp[8];  // eight independent partial maxima
+      float mp[8];  // eight independent partial maxima, two columns per step
 #pragma unroll
       for (int i = 0; i < 8; ++i) mp[i] = x[i];
 #pragma unroll
-      for (int c = 8; c < kHalf; ++c) mp[c & 7] = fmaxf(mp[c & 7], x[c]);
-      float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                       fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      for (int c = 8; c < kHalf; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
+      float mt = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
       mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
       const bool move = mt > m_ref + kLazyRescale;
       float alpha = 1.f;
@@ -365,19 +364,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
       {
         uint32_t hi[32], lo[32];
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+        // column pairs in packed fp32 arithmetic (one instruction per pair)
+        const float2 sc = make_float2(a.scale_log2, a.scale_log2);
+        const float2 nm = make_float2(-mref, -mref);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // independent partial sums
 #pragma unroll
         for (int e = 0; e < kHalf / 2; ++e) {
-          const float p0 = fast_exp2(fmaf(x[2 * e], a.scale_log2, -mref));
-          const float p1 = fast_exp2(fmaf(x[2 * e + 1], a.scale_log2, -mref));
-          ls[e & 3] += p0 + p1;
-          hi[e] = Pack<T>::pack(p0, p1);
+          const float2 t = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc, nm);
+          const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          ls[e & 1] = __fadd2_rn(ls[e & 1], p);
+          hi[e] = Pack<T>::pack(p.x, p.y);
           if constexpr (kSplit) {
-            const float2 f = Pack<T>::unpack(hi[e]);
-            lo[e] = Pack<T>::pack(p0 - f.x, p1 - f.y);
+            const float2 r = __ffma2_rn(Pack<T>::unpack(hi[e]), make_float2(-1.f, -1.f), p);
+            lo[e] = Pack<T>::pack(r.x, r.y);
           }
         }
-        l_sum += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        const float2 lsum = __fadd2_rn(ls[0], ls[1]);
+        l_sum += lsum.x + lsum.y;
         const uint32_t pcol = tmem + b * kKv + half * kHalf;
         tc::st_32x32b_x32(pcol + lane_off, hi);
         if constexpr (kSplit) tc::st_32x32b_x32(pcol + 32u + lane_off, lo);
@@ -434,8 +437,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q4 = 0; q4 < 4; ++q4) {
             float v[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              v[e] = c0 * __uint_as_float(r0[q4 * 8 + e]) + c1 * __uint_as_float(r1[q4 * 8 + e]);
+            for (int e = 0; e < 8; e += 2) {
+              const int i = q4 * 8 + e;
+              const float2 w = __ffma2_rn(make_float2(__uint_as_float(r0[i]), __uint_as_float(r0[i + 1])),
+                                          make_float2(c0, c0),
+                                          __fmul2_rn(make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1])),
+                                                     make_float2(c1, c1)));
+              v[e] = w.x;
+              v[e + 1] = w.y;
+            }
             *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) =
                 make_uint4(Pack<T>::pack(v[0], v[1]), Pack<T>::pack(v[2], v[3]), Pack<T>::pack(v[4], v[5]),
                            Pack<T>::pack(v[6], v[7]));
