@@ -59,6 +59,13 @@ constexpr uint32_t kTmemCols = 512;          // S buffers [0, 256), O of half 0 
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 template <typename T>
 struct PrefillTune {
   static constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;

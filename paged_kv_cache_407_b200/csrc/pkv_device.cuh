@@ -234,11 +234,4 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// max(a, b, c) in one instruction (three-input max.f32, sm_100).
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
 }  // namespace pkv
