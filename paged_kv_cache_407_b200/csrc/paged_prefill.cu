@@ -18,18 +18,24 @@
 //              same TMEM columns (fp16, or bf16 high + bf16 residual, since
 //              bf16 alone would round P by 2^-9), finally the merged O / l;
 //   warp 8     TMA: the Q tile (rank-3 map over [T][Hq][D]) and the K tiles,
-//              128 tokens gathered block by block through the Block Table
-//              (rank-4 map over [N][Hkv][B][D]), two stages;
+//              128 tokens gathered through the Block Table, one TMA box per
+//              block (a rank-5 view of [N][Hkv][B][D] that lands the block
+//              as groups of 8 rows, so that the tile's 8-row groups sit at
+//              one fixed stride for the tensor core), two stages;
 //   warp 9     TMA: the V tiles, two stages;
 //   warp 10    tcgen05.mma, one thread: S(j) = Q K(j)^T (128x128x128) into
-//              one of two TMEM buffers; O_h += P_h(j) V_h(j) with P read from
+//              one of two TMEM buffers, once P V(j-2) has read that buffer;
+//   warp 11    tcgen05.mma, one thread: O_h += P_h(j) V_h(j) with P read from
 //              tensor memory (the S buffer) and V from shared memory
-//              (MN-major), in the order S(0), S(1), PV(0), S(2), PV(1), ...; the
-//              in-order tensor pipe finishes P V(j) before S(j+2) reuses the
-//              buffer.
+//              (MN-major).  Two issuers, because a thread that has just
+//              issued a batch of MMAs waits for the tensor pipe to take them
+//              before its next barrier test completes: with one issuer every
+//              operand wait sat on the pipe's critical path.
 // Every wait is bounded; after a timeout every role stops, PKV_DEV_TIMEOUT is
 // raised, outstanding tensor-core work and loads are drained (bounded) and
 // TMEM is freed.
+#include <cudaTypedefs.h>
+
 #include <type_traits>
 
 #include "pkv_device.cuh"
@@ -46,8 +52,9 @@ constexpr int kSoftmaxWarps = 8;  // warps 0-7: (query row, token half) per thre
 constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
 constexpr int kLoadKWarp = 8;     // TMA loads of K tiles (and Q)
 constexpr int kLoadVWarp = 9;     // TMA loads of V tiles
-constexpr int kMmaWarp = 10;      // issues every tcgen05.mma
-constexpr int kThreads = 32 * 11;
+constexpr int kMmaWarp = 10;      // issues the S = Q K^T MMAs
+constexpr int kPvWarp = 11;       // issues the O += P V MMAs
+constexpr int kThreads = 32 * 12;
 constexpr int kHalf = 64;         // tokens of a K/V tile per softmax half
 constexpr uint32_t kChunk = 128u * 128u;  // [128 rows][64 elements] of 16-bit: 16 KB
 constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
@@ -65,6 +72,12 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+
+// K/V tiles in shared memory: 16 groups of 8 token rows, group i at 2048 i;
+// within a group the two 64-element halves of head_dim at +0 / +1024, each
+// 8 rows of 128 bytes (128-byte swizzle).  Token groups are 2048 bytes apart
+// whatever the block size, so one descriptor stride covers a whole tile.
+constexpr uint32_t kGroupBytes = 2048;
 
 template <typename T>
 struct PrefillTune {
@@ -84,6 +97,7 @@ struct PrefillArgs {
   int num_q_heads;
   int group;
   int num_blocks;
+  int num_kv_heads;
   float scale_log2;
 };
 
@@ -146,6 +160,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 136);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 140);
   const uint32_t bar_x = bars + 144;      // softmax halves' final (m, l) exchanged
+  const uint32_t bar_pfree = bars + 152;  // [2] P in the S buffer read by P V (MMA commit)
+  // The last P V done (MMA commit, one phase).  The final read of O cannot
+  // use bar_o: when the softmax warps finish their last tile, P V(n-2) may
+  // still be running as well as P V(n-1), and a parity wait cannot tell two
+  // outstanding phases from none.
+  const uint32_t bar_end = bars + 168;
 
   if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
   if (tid == 0) {
@@ -160,7 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_p + 8 * i, kSoftmaxWarps);
     }
     mbar_init(bar_o, 1);
-    mbar_init(bar_done, 1);
+    mbar_init(bar_done, 2);
+    mbar_init(bar_pfree, 1);
+    mbar_init(bar_pfree + 8, 1);
+    mbar_init(bar_end, 1);
     mbar_init(bar_x, kSoftmaxWarps);
     *abort_flag = 0;
     fence_barrier_init();
@@ -230,17 +253,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int bi = 0; bi < kBlocksPerTile; ++bi) {
             const int lb = j * kBlocksPerTile + bi;
-            if (lb < nb && static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks)) {
-#pragma unroll
-              for (int c = 0; c < 2; ++c)
-                tma_load_4d(dst + c * kChunk + bi * BS * 128u, map, bar, c * 64, 0, g, idv[bi], policy);
-            }
+            if (lb < nb && static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
+              tma_load_5d(dst + bi * (BS / 8) * kGroupBytes, map, bar, 0, 0, 0, 0, idv[bi] * a.num_kv_heads + g,
+                          policy);
           }
         }
       }
       ids = next;
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
     // --------------------------------------------------------- MMA issuer
     constexpr uint32_t kIdescS = tc::idesc_f16(kBf16, false, 128, 128);
     constexpr uint32_t kIdescO = tc::idesc_f16(kBf16, true, 128, 128);
@@ -253,8 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kDim / 16; ++k) {
           const uint32_t koff = (k >> 2) * kChunk + (k & 3) * 32u;
+          const uint32_t kkoff = (k >> 2) * 1024u + (k & 3) * 32u;
           tc::mma_f16_ss(tmem + b * kKv, tc::smem_desc_sw128(sb + kQOff + koff, 16u, 1024u),
-                         tc::smem_desc_sw128(kb + koff, 16u, 1024u), kIdescS, k > 0 ? 1u : 0u);
+                         tc::smem_desc_sw128(kb + kkoff, 16u, kGroupBytes), kIdescS, k > 0 ? 1u : 0u);
         }
         tc::commit(bar_s + 8 * b);
         tc::commit(bar_kfree + 8 * b);
@@ -276,23 +298,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < kKv / 16; ++k) {
           const uint32_t h = k >> 2;
           const uint32_t pcol = tmem + b * kKv + h * kHalf + (k & 3) * 8u;
-          const uint64_t vdesc = tc::smem_desc_sw128(vb + k * 2048u, kChunk, 1024u);
+          const uint64_t vdesc = tc::smem_desc_sw128(vb + k * 2u * kGroupBytes, 1024u, kGroupBytes);
           tc::mma_f16_ts(tO + h * kDim, pcol, vdesc, kIdescO, (j > 0 || (k & 3) > 0) ? 1u : 0u);
           if constexpr (kSplit) tc::mma_f16_ts(tO + h * kDim, pcol + 32u, vdesc, kIdescO, 1u);
         }
         tc::commit(bar_o);
         tc::commit(bar_vfree + 8 * b);
+        tc::commit(bar_pfree + 8 * b);
+        if (j == ntiles - 1) tc::commit(bar_end);
       }
       __syncwarp();
       return true;
     };
-    bool run = wait(bar_q, 0);
-    // order on the tensor pipe: S(0), S(1), PV(0), S(2), PV(1), ...
-    for (int j = 0; run && j < ntiles; ++j) {
-      run = issue_s(j);
-      if (run && j >= 1) run = issue_pv(j - 1);
+    // Two issuing warps feed the one tensor pipe, so that neither kind of
+    // MMA waits behind the other's operands: S(j) goes as soon as K(j) is in
+    // and P V(j-2) has read the S buffer it overwrites; P V(j) as soon as
+    // V(j) and P(j) are ready.
+    if (warp == kMmaWarp) {
+      bool run = wait(bar_q, 0);
+      for (int j = 0; run && j < ntiles; ++j) {
+        if (j >= 2 && !(run = wait(bar_pfree + 8 * (j & 1), ((j - 2) >> 1) & 1))) break;
+        run = issue_s(j);
+      }
+    } else {
+      bool run = true;
+      for (int j = 0; run && j < ntiles; ++j) run = issue_pv(j);
     }
-    if (run) issue_pv(ntiles - 1);
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------- softmax, (row, token half) per thread
     // Each half of the threads runs its own online softmax over its half of
@@ -346,7 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_sum *= alpha;
       }
       if (j > 0 && __any_sync(kFullMask, move)) {
-        // O_h must hold P V(j-1) before it is rescaled
+        // O_h must hold P V(j-1) before it is rescaled.  P V(j-2) is done
+        // (S(j) waited for it) and P V(j) needs this warp's P(j), so
+        // exactly one phase of bar_o can be outstanding here.
         if (!(run = wait(bar_o, (j - 1) & 1))) break;
         tc::fence_after_sync();
 #pragma unroll
@@ -398,10 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int valid_tok = min(kKv, L - j * kKv);
       if (valid_tok < kKv) {
         if (!(run = wait(bar_v + 8 * b, (j >> 1) & 1))) break;
-        uint4 *v4 = reinterpret_cast<uint4 *>(smem + kVOff + b * kTile);
-        for (int u = valid_tok * 8 + tid; u < kKv * 8; u += kSoftmaxThreads) {
-          v4[u] = make_uint4(0u, 0u, 0u, 0u);
-          v4[kChunk / 16 + u] = make_uint4(0u, 0u, 0u, 0u);
+        uint8_t *vt = smem + kVOff + b * kTile;
+        for (int u = valid_tok * 16 + tid; u < kKv * 16; u += kSoftmaxThreads) {
+          const int r = u >> 4, w = u & 15;  // token row, 16-byte unit of its 256 bytes
+          *reinterpret_cast<uint4 *>(vt + (r >> 3) * kGroupBytes + (w >> 3) * 1024 + (r & 7) * 128 + (w & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
         }
       }
       if (valid_tok < kKv) fence_proxy_async_smem();
@@ -409,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p + 8 * b);
     }
-    if (run) run = wait(bar_o, (ntiles - 1) & 1);
+    if (run) run = wait(bar_end, 0);
     if (run) {
       tc::fence_after_sync();
       // merge the two halves' states of the row
@@ -470,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // loads still in flight finish (bounded) before TMEM and shared memory
     // are released.
     if (tid == 0) raise_flag(a.d_status, PKV_DEV_TIMEOUT);
-    if (warp == kMmaWarp && lane == 0) tc::commit(bar_done);
+    if ((warp == kMmaWarp || warp == kPvWarp) && lane == 0) tc::commit(bar_done);
     (void)mbar_wait(bar_done, 0);
     for (int i = 0; i < 2; ++i) {
       (void)mbar_wait(bar_k + 8 * i, 0);
@@ -484,6 +518,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Rank-5 view of a pool [N][Hkv][B][D] (16-bit, D = 128) for one box per
+// block: (64 elements, 8 rows, 2 halves of head_dim, B / 8 row groups,
+// N * Hkv (block, head) pairs); the box is a whole block, landing as
+// [row group][half][8 rows][128 B].
+pkv_status encode_grouped_map(CUtensorMap *map, const void *pool, const pkv_cache_desc &c) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    return (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+               ? reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f)
+               : nullptr;
+  }();
+  if (fn == nullptr) return PKV_ERR_CUDA;
+  const cuuint64_t row = static_cast<cuuint64_t>(c.head_dim) * 2;
+  cuuint64_t dims[5] = {64, 8, 2, static_cast<cuuint64_t>(c.block_size / 8),
+                        static_cast<cuuint64_t>(c.num_blocks) * c.num_kv_heads};
+  cuuint64_t strides[4] = {row, 128, 8 * row, static_cast<cuuint64_t>(c.block_size) * row};
+  cuuint32_t box[5] = {64, 8, 2, static_cast<cuuint32_t>(c.block_size / 8), 1};
+  cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 5, const_cast<void *>(pool), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PKV_OK : PKV_ERR_CUDA;
 }
 
 template <typename T>
@@ -543,8 +603,8 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
 
   CUtensorMap tq, tk, tv;
   if ((st = encode_query_map(&tq, query, num_tokens, num_q_heads, kDim, G)) != PKV_OK) return st;
-  if ((st = encode_cache_map(&tk, k_cache, cache)) != PKV_OK) return st;
-  if ((st = encode_cache_map(&tv, v_cache, cache)) != PKV_OK) return st;
+  if ((st = encode_grouped_map(&tk, k_cache, cache)) != PKV_OK) return st;
+  if ((st = encode_grouped_map(&tv, v_cache, cache)) != PKV_OK) return st;
 
   PrefillArgs args{};
   args.out = out;
@@ -557,6 +617,7 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
   args.num_q_heads = num_q_heads;
   args.group = G;
   args.num_blocks = cache.num_blocks;
+  args.num_kv_heads = cache.num_kv_heads;
   args.scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(static_cast<unsigned>(qtiles), static_cast<unsigned>(cache.num_kv_heads),
             static_cast<unsigned>(num_seqs));
