@@ -49,6 +49,10 @@ KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/pkv_host.cu",
                   "paged_kv_cache_407_b200/csrc/paged_attention.cu",
                   "paged_kv_cache_407_b200/csrc/decode_core.cuh",
                   "paged_kv_cache_407_b200/csrc/pkv_device.cuh"]
+PREFILL_SOURCES = ["paged_kv_cache_407_b200/csrc/pkv_host.cu",
+                   "paged_kv_cache_407_b200/csrc/paged_prefill.cu",
+                   "paged_kv_cache_407_b200/csrc/tcgen05.cuh",
+                   "paged_kv_cache_407_b200/csrc/pkv_device.cuh"]
 
 
 def parse_args(argv=None):
@@ -66,9 +70,9 @@ def parse_args(argv=None):
     return p.parse_args(argv)
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -84,19 +88,20 @@ def measured_peak(key: str = "hbm_gbs"):
         return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
-def profiled_traffic(workload: str, kv_dtype: str = "f16"):
+def profiled_traffic(workload: str, kv_dtype: str = "f16", kernel: str = "paged_decode_kernel"):
     """DRAM bytes per launch of the attention kernel from the committed ncu
     summary, if it was taken on the current kernel source; else None."""
     suffix = "_e4m3" if kv_dtype == "e4m3" else ""
-    path = os.path.join(PROFILE_DIR, f"paged_decode_kernel{suffix}_{workload}.txt")
+    sources = PREFILL_SOURCES if kernel == "paged_prefill_kernel" else KERNEL_SOURCES
+    path = os.path.join(PROFILE_DIR, f"{kernel}{suffix}_{workload}.txt")
     try:
         kv = {}
         with open(path, encoding="utf-8") as f:
             for line in f:
                 if ":" in line and not line.startswith("#"):
                     k, v = line.split(":", 1)
-                    kv[k.strip()] = v.strip()
-        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+                    kv[k.strip()] = (v.split() or [""])[0]
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash(sources):
             return None
         return float(kv["dram_bytes_per_launch_full_workload"])
     except (OSError, KeyError, ValueError):
@@ -526,7 +531,7 @@ def run_prefill(args):
             "peak_source": (f"{peak_kind} (MEASURED_PEAKS.json bf16_tflops; fp16 has the same nominal rate)"
                             if peak_kind == "measured" else "fallback"),
             "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "traffic": None,
+            "traffic": profiled_traffic(b.name, kernel="paged_prefill_kernel"),
         },
         "clocks": clock,
         "gpu_launches": 2 * K,
