@@ -311,10 +311,12 @@ PKV_API pkv_status pkv_paged_attention_decode_fp8(
  *              are not written.
  * context_lens: int32 [num_seqs] device, C <= L <= max_blocks_per_seq * B.
  * block_tables: as for decode.  max_query_len >= every C (host value; it
- *              sizes the grid).
+ *              sets the number of 128-row query tiles per (sequence, kv
+ *              head)).  PKV_ERR_TOO_LARGE when query tiles x num_kv_heads x
+ *              num_seqs exceeds 2^31 - 1.
  * head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
  * Runs on tcgen05 tensor cores: 128-row query tiles x 128-token K/V tiles,
- * fp32 accumulation in tensor memory.
+ * fp32 accumulation in tensor memory; a persistent grid of one CTA per SM.
  * Device-detected errors: a sequence whose lengths break the rules above is
  * skipped with PKV_DEV_BAD_LEN; a block id outside the pool raises
  * PKV_DEV_BAD_BLOCK (that block's tokens are garbage); a wait past ~1 s

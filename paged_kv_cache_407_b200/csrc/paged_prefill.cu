@@ -6,9 +6,12 @@
 // sequence, the chunk's token at position p = L - C + j (its K/V already
 // written to the cache) attends over positions 0..p through the Block Table.
 //
-// One CTA per (128-row query tile, kv head, sequence); a tile row is one
-// (token, query head of the group) pair, so 128 / G tokens per tile.  Roles
-// (warp-specialised, synchronised only through mbarriers):
+// A work item is a (128-row query tile, kv head, sequence); a tile row is one
+// (token, query head of the group) pair, so 128 / G tokens per tile.  The
+// grid is persistent (one CTA per SM), each CTA walking a fixed share of the
+// items, so that the next item's Q tile and first K/V tiles load while the
+// current one finishes.  Roles (warp-specialised, synchronised only through
+// mbarriers):
 //   warps 0-7  softmax, two threads per row, each owning one 64-token half of
 //              every K/V tile with its own running max, sum and O
 //              accumulator (merged once at the end): tcgen05.ld of its TMEM
@@ -17,7 +20,8 @@
 //              is rescaled, after P V(j-1) is done), P written back into the
 //              same TMEM columns (fp16, or bf16 high + bf16 residual, since
 //              bf16 alone would round P by 2^-9), finally the merged O / l;
-//   warp 8     TMA: the Q tile (rank-3 map over [T][Hq][D]) and the K tiles,
+//   warp 8     TMA: the Q tiles (rank-3 map over [T][Hq][D], two buffers)
+//              and the K tiles,
 //              128 tokens gathered through the Block Table, one TMA box per
 //              block (a rank-5 view of [N][Hkv][B][D] that lands the block
 //              as groups of 8 rows, so that the tile's 8-row groups sit at
@@ -58,10 +62,10 @@ constexpr int kThreads = 32 * 12;
 constexpr int kHalf = 64;         // tokens of a K/V tile per softmax half
 constexpr uint32_t kChunk = 128u * 128u;  // [128 rows][64 elements] of 16-bit: 16 KB
 constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
-constexpr uint32_t kQOff = 0;
-constexpr uint32_t kKOff = kTile;            // two K stages
-constexpr uint32_t kVOff = 3u * kTile;       // two V stages
-constexpr uint32_t kXOff = 5u * kTile;       // final (m, l) exchange of the softmax halves
+constexpr uint32_t kQOff = 0;               // two Q buffers (this item's, the next one's)
+constexpr uint32_t kKOff = 2u * kTile;       // two K stages
+constexpr uint32_t kVOff = 4u * kTile;       // two V stages
+constexpr uint32_t kXOff = 6u * kTile;       // final (m, l) exchange of the softmax halves
 constexpr uint32_t kTmemCols = 512;          // S buffers [0, 256), O of half 0 / 1 [256, 512)
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
@@ -93,13 +97,65 @@ struct PrefillArgs {
   const int32_t *context_lens;
   int32_t *d_status;
   int num_tokens;
+  int num_seqs;
   int max_blocks_per_seq;
   int num_q_heads;
   int group;
   int num_blocks;
   int num_kv_heads;
+  int qtiles;      // query tiles of the longest chunk
+  int items;       // qtiles * num_kv_heads * num_seqs work items
   float scale_log2;
 };
+
+// One work item: a 128-row query tile of one (sequence, kv head).  Items are
+// numbered in groups of kPairsPerGroup (sequence, kv head) pairs; inside a
+// group, longest first (query tile qtiles - 1 of each pair, then qtiles - 2,
+// ...: later query tiles see more keys).  The CTAs working at one time then
+// share the K/V of a few pairs, which stay in L2.
+constexpr int kPairsPerGroup = 8;
+struct Item {
+  int s, g, t_begin, C, L, tok0, ntiles, nb;
+};
+
+template <int BS>
+__device__ __forceinline__ bool item_at(const PrefillArgs &a, int i, Item &it, bool report) {
+  const int pairs = a.num_kv_heads * a.num_seqs;
+  const int group_items = kPairsPerGroup * a.qtiles;
+  const int full = pairs / kPairsPerGroup;  // complete groups
+  const int grp = i / group_items;
+  const int width = grp < full ? kPairsPerGroup : pairs - full * kPairsPerGroup;
+  const int rem = i - grp * group_items;
+  const int qt = a.qtiles - 1 - rem / width;
+  const int pair = grp * kPairsPerGroup + rem % width;
+  it.g = pair % a.num_kv_heads;
+  it.s = pair / a.num_kv_heads;
+  it.t_begin = a.query_start[it.s];
+  const int t_end = a.query_start[it.s + 1];
+  it.C = t_end - it.t_begin;
+  it.L = a.context_lens[it.s];
+  if (it.C < 0 || it.t_begin < 0 || t_end > a.num_tokens || it.L < it.C ||
+      static_cast<long long>(it.L) > static_cast<long long>(a.max_blocks_per_seq) * BS) {
+    if (report && it.g == 0 && qt == 0) raise_flag(a.d_status, PKV_DEV_BAD_LEN);
+    return false;
+  }
+  it.tok0 = qt * (kRows / a.group);
+  if (it.tok0 >= it.C) return false;
+  const int last_tok = min(it.tok0 + kRows / a.group, it.C) - 1;
+  it.ntiles = (it.L - it.C + last_tok + kKv) / kKv;  // K/V tiles up to the largest position
+  it.nb = (it.L + BS - 1) / BS;
+  return true;
+}
+
+// The k-th item of this CTA (-1 past the end): rounds of gridDim.x items,
+// alternate rounds walked in opposite directions so that every CTA gets a
+// similar share of long and short items.
+__device__ __forceinline__ int item_index(const PrefillArgs &a, int k) {
+  const int P = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
+  const long long i = static_cast<long long>(k) * P + ((k & 1) ? P - 1 - c : c);
+  return i < a.items ? static_cast<int>(i) : -1;
+}
 
 template <typename T, int BS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -117,74 +173,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  // Query tiles launch last-first: later tiles see more keys (causal), so
-  // the longest CTAs start first and the short ones fill the tail.
-  const int qt = gridDim.x - 1 - blockIdx.x;
-  const int g = blockIdx.y;
-  const int s = blockIdx.z;
   const int G = a.group;
-  const int tok_per_tile = kRows / G;
-
-  // ---- geometry of this tile (uniform over the CTA) ----------------------
-  const int t_begin = a.query_start[s];
-  const int t_end = a.query_start[s + 1];
-  const int C = t_end - t_begin;
-  const int L = a.context_lens[s];
-  if (C < 0 || t_begin < 0 || t_end > a.num_tokens || L < C ||
-      static_cast<long long>(L) > static_cast<long long>(a.max_blocks_per_seq) * BS) {
-    if (tid == 0 && g == 0 && qt == 0) raise_flag(a.d_status, PKV_DEV_BAD_LEN);
-    return;
-  }
-  const int tok0 = qt * tok_per_tile;
-  if (tok0 >= C) return;
-  const int last_tok = min(tok0 + tok_per_tile, C) - 1;
-  const int p_max = L - C + last_tok;      // largest position among the tile's rows
-  const int ntiles = (p_max + kKv) / kKv;  // K/V tiles to visit (>= 1)
-  const int nb = (L + BS - 1) / BS;
 
   // ---- barriers (see the role loops for who arrives on which) ------------
+  // Every role walks the same items in the same order and keeps running
+  // counts (items, K/V tiles), so stage indices and phase parities carry on
+  // across items.
   const uint32_t bars = sb + TN::kBarOff;
-  const uint32_t bar_q = bars;
-  const uint32_t bar_k = bars + 8;        // [2] K stage loaded (TMA bytes)
-  const uint32_t bar_kfree = bars + 24;   // [2] K stage read by S (MMA commit)
-  const uint32_t bar_v = bars + 40;       // [2] V stage loaded
-  const uint32_t bar_vfree = bars + 56;   // [2] V stage read by P V
-  const uint32_t bar_s = bars + 72;       // [2] S buffer written (MMA commit)
+  const uint32_t bar_q = bars;            // [2] Q buffer loaded (TMA bytes)
+  const uint32_t bar_qfree = bars + 16;   // [2] Q buffer read by the item's last S (MMA commit)
+  const uint32_t bar_k = bars + 32;       // [2] K stage loaded (TMA bytes)
+  const uint32_t bar_kfree = bars + 48;   // [2] K stage read by S (MMA commit)
+  const uint32_t bar_v = bars + 64;       // [2] V stage loaded
+  const uint32_t bar_vfree = bars + 80;   // [2] V stage read by P V
+  const uint32_t bar_s = bars + 96;       // [2] S buffer written (MMA commit)
   // P-ready comes one per S buffer: a softmax warp may arrive for tile j+1
   // before a slower one arrives for tile j, and those arrivals must not
   // count towards the same phase.
-  const uint32_t bar_p = bars + 104;      // [2] P in TMEM, O rescaled (one arrival per softmax warp)
-  const uint32_t bar_o = bars + 120;      // P V done (MMA commit)
-  const uint32_t bar_done = bars + 128;   // drain on the error path
-  const uint32_t holder = bars + 136;
-  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 136);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 140);
-  const uint32_t bar_x = bars + 144;      // softmax halves' final (m, l) exchanged
-  const uint32_t bar_pfree = bars + 152;  // [2] P in the S buffer read by P V (MMA commit)
-  // The last P V done (MMA commit, one phase).  The final read of O cannot
-  // use bar_o: when the softmax warps finish their last tile, P V(n-2) may
-  // still be running as well as P V(n-1), and a parity wait cannot tell two
+  const uint32_t bar_p = bars + 112;      // [2] P in TMEM, O rescaled (one arrival per softmax warp)
+  const uint32_t bar_pfree = bars + 128;  // [2] P in the S buffer read by P V (MMA commit)
+  const uint32_t bar_o = bars + 144;      // P V done (MMA commit)
+  // The item's last P V done (MMA commit).  The final read of O cannot use
+  // bar_o: when the softmax warps finish their last tile, P V(n-2) may still
+  // be running as well as P V(n-1), and a parity wait cannot tell two
   // outstanding phases from none.
-  const uint32_t bar_end = bars + 168;
+  const uint32_t bar_end = bars + 152;
+  const uint32_t bar_x = bars + 168;      // softmax halves' final (m, l) exchanged
+  const uint32_t bar_done = bars + 176;   // drain on the error path
+  const uint32_t holder = bars + 184;
+  volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 184);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 188);
 
   if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
   if (tid == 0) {
-    mbar_init(bar_q, 1);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_q + 8 * i, 1);
+      mbar_init(bar_qfree + 8 * i, 1);
       mbar_init(bar_k + 8 * i, 1);
       mbar_init(bar_kfree + 8 * i, 1);
       mbar_init(bar_v + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
       mbar_init(bar_s + 8 * i, 1);
       mbar_init(bar_p + 8 * i, kSoftmaxWarps);
+      mbar_init(bar_pfree + 8 * i, 1);
     }
     mbar_init(bar_o, 1);
-    mbar_init(bar_done, 2);
-    mbar_init(bar_pfree, 1);
-    mbar_init(bar_pfree + 8, 1);
     mbar_init(bar_end, 1);
     mbar_init(bar_x, kSoftmaxWarps);
+    mbar_init(bar_done, 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -206,255 +243,288 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- producers
     const bool is_k = warp == kLoadKWarp;
     const CUtensorMap *map = is_k ? &tm_k : &tm_v;
-    if (lane == 0) prefetch_tensormap(map);
-    if (is_k && lane == 0) {
-      prefetch_tensormap(&tm_q);
-      mbar_arrive_expect_tx(bar_q, kTile);
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-        tma_load_3d(sb + kQOff + c * kChunk, &tm_q, bar_q, c * 64, g * G, t_begin + tok0,
-                    l2_evict_first_policy());
+    if (lane == 0) {
+      prefetch_tensormap(map);
+      if (is_k) prefetch_tensormap(&tm_q);
     }
     const uint64_t policy = l2_evict_first_policy();
-    const int32_t *trow = a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq;
     const uint32_t full = is_k ? bar_k : bar_v;
     const uint32_t empty = is_k ? bar_kfree : bar_vfree;
     const uint32_t stage0 = sb + (is_k ? kKOff : kVOff);
-    auto ids_of = [&](int j) -> int {
-      const int lb = j * kBlocksPerTile + lane;
-      return (j < ntiles && lane < kBlocksPerTile && lb < nb) ? __ldg(trow + lb) : -1;
-    };
-    int ids = ids_of(0);
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
-      const int next = ids_of(j + 1);  // in flight while this tile is issued
-      if (j >= 2 && !wait(empty + 8 * st, ((j - 2) >> 1) & 1)) break;
-      uint32_t bytes = 0;
-      int idv[kBlocksPerTile];
+    bool run = true;
+    int n = 0;   // items so far
+    int jt = 0;  // K/V tiles so far
+    for (int k = 0; run; ++k) {
+      const int i = item_index(a, k);
+      if (i < 0) break;
+      Item it;
+      if (!item_at<BS>(a, i, it, false)) continue;
+      if (is_k) {
+        // the item's Q tile into Q buffer n % 2, once the item two back has
+        // done its last S
+        const int qb = n & 1;
+        if (n >= 2 && !(run = wait(bar_qfree + 8 * qb, ((n - 2) >> 1) & 1))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_q + 8 * qb, kTile);
 #pragma unroll
-      for (int bi = 0; bi < kBlocksPerTile; ++bi) {
-        idv[bi] = __shfl_sync(kFullMask, ids, bi);
-        const int lb = j * kBlocksPerTile + bi;
-        if (lb < nb) {
-          if (static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
-            bytes += 2u * 64u * BS * 2u;
-          else if (lane == 0)
-            raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sb + kQOff + qb * kTile + c * kChunk, &tm_q, bar_q + 8 * qb, c * 64, it.g * G,
+                        it.t_begin + it.tok0, policy);
         }
       }
-      if (lane == 0) {
-        const uint32_t bar = full + 8 * st;
-        const uint32_t dst = stage0 + st * kTile;
-        fence_proxy_async_smem();
-        if (bytes == 0) {
-          mbar_arrive(bar);
-        } else {
-          mbar_arrive_expect_tx(bar, bytes);
+      const int32_t *trow = a.block_tables + static_cast<size_t>(it.s) * a.max_blocks_per_seq;
+      auto ids_of = [&](int j) -> int {
+        const int lb = j * kBlocksPerTile + lane;
+        return (j < it.ntiles && lane < kBlocksPerTile && lb < it.nb) ? __ldg(trow + lb) : -1;
+      };
+      int ids = ids_of(0);
+      for (int j = 0; j < it.ntiles; ++j, ++jt) {
+        const int st = jt & 1;
+        const int next = ids_of(j + 1);  // in flight while this tile is issued
+        if (jt >= 2 && !(run = wait(empty + 8 * st, ((jt - 2) >> 1) & 1))) break;
+        uint32_t bytes = 0;
+        int idv[kBlocksPerTile];
 #pragma unroll
-          for (int bi = 0; bi < kBlocksPerTile; ++bi) {
-            const int lb = j * kBlocksPerTile + bi;
-            if (lb < nb && static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
-              tma_load_5d(dst + bi * (BS / 8) * kGroupBytes, map, bar, 0, 0, 0, 0, idv[bi] * a.num_kv_heads + g,
-                          policy);
+        for (int bi = 0; bi < kBlocksPerTile; ++bi) {
+          idv[bi] = __shfl_sync(kFullMask, ids, bi);
+          const int lb = j * kBlocksPerTile + bi;
+          if (lb < it.nb) {
+            if (static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
+              bytes += 2u * 64u * BS * 2u;
+            else if (lane == 0)
+              raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
           }
         }
+        if (lane == 0) {
+          const uint32_t bar = full + 8 * st;
+          const uint32_t dst = stage0 + st * kTile;
+          fence_proxy_async_smem();
+          if (bytes == 0) {
+            mbar_arrive(bar);
+          } else {
+            mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+            for (int bi = 0; bi < kBlocksPerTile; ++bi) {
+              const int lb = j * kBlocksPerTile + bi;
+              if (lb < it.nb && static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
+                tma_load_5d(dst + bi * (BS / 8) * kGroupBytes, map, bar, 0, 0, 0, 0,
+                            idv[bi] * a.num_kv_heads + it.g, policy);
+            }
+          }
+        }
+        ids = next;
       }
-      ids = next;
+      ++n;
     }
   } else if (warp == kMmaWarp || warp == kPvWarp) {
-    // --------------------------------------------------------- MMA issuer
-    constexpr uint32_t kIdescS = tc::idesc_f16(kBf16, false, 128, 128);
-    constexpr uint32_t kIdescO = tc::idesc_f16(kBf16, true, 128, 128);
-    auto issue_s = [&](int j) -> bool {
-      const int b = j & 1;
-      if (!wait(bar_k + 8 * b, (j >> 1) & 1)) return false;
-      if (lane == 0) {
-        tc::fence_after_sync();
-        const uint32_t kb = sb + kKOff + b * kTile;
-#pragma unroll
-        for (int k = 0; k < kDim / 16; ++k) {
-          const uint32_t koff = (k >> 2) * kChunk + (k & 3) * 32u;
-          const uint32_t kkoff = (k >> 2) * 1024u + (k & 3) * 32u;
-          tc::mma_f16_ss(tmem + b * kKv, tc::smem_desc_sw128(sb + kQOff + koff, 16u, 1024u),
-                         tc::smem_desc_sw128(kb + kkoff, 16u, kGroupBytes), kIdescS, k > 0 ? 1u : 0u);
-        }
-        tc::commit(bar_s + 8 * b);
-        tc::commit(bar_kfree + 8 * b);
-      }
-      __syncwarp();
-      return true;
-    };
-    auto issue_pv = [&](int j) -> bool {
-      const int b = j & 1;
-      if (!wait(bar_v + 8 * b, (j >> 1) & 1)) return false;
-      if (!wait(bar_p + 8 * b, (j >> 1) & 1)) return false;
-      if (lane == 0) {
-        tc::fence_after_sync();
-        const uint32_t vb = sb + kVOff + b * kTile;
-        // O_h += P_h V_h: P_h sits in the S buffer's columns of half h
-        // (high part in its first 32 columns, bf16 residual in the next 32),
-        // V_h is V rows 64h .. 64h + 63.
-#pragma unroll
-        for (int k = 0; k < kKv / 16; ++k) {
-          const uint32_t h = k >> 2;
-          const uint32_t pcol = tmem + b * kKv + h * kHalf + (k & 3) * 8u;
-          const uint64_t vdesc = tc::smem_desc_sw128(vb + k * 2u * kGroupBytes, 1024u, kGroupBytes);
-          tc::mma_f16_ts(tO + h * kDim, pcol, vdesc, kIdescO, (j > 0 || (k & 3) > 0) ? 1u : 0u);
-          if constexpr (kSplit) tc::mma_f16_ts(tO + h * kDim, pcol + 32u, vdesc, kIdescO, 1u);
-        }
-        tc::commit(bar_o);
-        tc::commit(bar_vfree + 8 * b);
-        tc::commit(bar_pfree + 8 * b);
-        if (j == ntiles - 1) tc::commit(bar_end);
-      }
-      __syncwarp();
-      return true;
-    };
+    // --------------------------------------------------------- MMA issuers
     // Two issuing warps feed the one tensor pipe, so that neither kind of
     // MMA waits behind the other's operands: S(j) goes as soon as K(j) is in
     // and P V(j-2) has read the S buffer it overwrites; P V(j) as soon as
     // V(j) and P(j) are ready.
-    if (warp == kMmaWarp) {
-      bool run = wait(bar_q, 0);
-      for (int j = 0; run && j < ntiles; ++j) {
-        if (j >= 2 && !(run = wait(bar_pfree + 8 * (j & 1), ((j - 2) >> 1) & 1))) break;
-        run = issue_s(j);
+    constexpr uint32_t kIdescS = tc::idesc_f16(kBf16, false, 128, 128);
+    constexpr uint32_t kIdescO = tc::idesc_f16(kBf16, true, 128, 128);
+    const bool is_s = warp == kMmaWarp;
+    bool run = true;
+    int n = 0;
+    int jt = 0;
+    for (int k = 0; run; ++k) {
+      const int i = item_index(a, k);
+      if (i < 0) break;
+      Item it;
+      if (!item_at<BS>(a, i, it, false)) continue;
+      const int qb = n & 1;
+      if (is_s) {
+        if (!(run = wait(bar_q + 8 * qb, (n >> 1) & 1))) break;
+        const uint32_t qbase = sb + kQOff + qb * kTile;
+        for (int j = 0; j < it.ntiles; ++j, ++jt) {
+          const int b = jt & 1;
+          if (jt >= 2 && !(run = wait(bar_pfree + 8 * b, ((jt - 2) >> 1) & 1))) break;
+          if (!(run = wait(bar_k + 8 * b, (jt >> 1) & 1))) break;
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint32_t kb = sb + kKOff + b * kTile;
+#pragma unroll
+            for (int kk = 0; kk < kDim / 16; ++kk) {
+              const uint32_t qoff = (kk >> 2) * kChunk + (kk & 3) * 32u;
+              const uint32_t koff = (kk >> 2) * 1024u + (kk & 3) * 32u;
+              tc::mma_f16_ss(tmem + b * kKv, tc::smem_desc_sw128(qbase + qoff, 16u, 1024u),
+                             tc::smem_desc_sw128(kb + koff, 16u, kGroupBytes), kIdescS, kk > 0 ? 1u : 0u);
+            }
+            tc::commit(bar_s + 8 * b);
+            tc::commit(bar_kfree + 8 * b);
+            if (j == it.ntiles - 1) tc::commit(bar_qfree + 8 * qb);
+          }
+          __syncwarp();
+        }
+      } else {
+        for (int j = 0; j < it.ntiles; ++j, ++jt) {
+          const int b = jt & 1;
+          if (!(run = wait(bar_v + 8 * b, (jt >> 1) & 1))) break;
+          if (!(run = wait(bar_p + 8 * b, (jt >> 1) & 1))) break;
+          // The first P V of an item overwrites O.  It needs P from every
+          // softmax warp, which each writes only after reading out the
+          // previous item's O, so bar_p orders that too.
+          if (lane == 0) {
+            tc::fence_after_sync();
+            const uint32_t vb = sb + kVOff + b * kTile;
+            // O_h += P_h V_h: P_h sits in the S buffer's columns of half h
+            // (high part in its first 32 columns, bf16 residual in the next
+            // 32), V_h is V rows 64h .. 64h + 63.
+#pragma unroll
+            for (int kk = 0; kk < kKv / 16; ++kk) {
+              const uint32_t h = kk >> 2;
+              const uint32_t pcol = tmem + b * kKv + h * kHalf + (kk & 3) * 8u;
+              const uint64_t vdesc = tc::smem_desc_sw128(vb + kk * 2u * kGroupBytes, 1024u, kGroupBytes);
+              tc::mma_f16_ts(tO + h * kDim, pcol, vdesc, kIdescO, (j > 0 || (kk & 3) > 0) ? 1u : 0u);
+              if constexpr (kSplit) tc::mma_f16_ts(tO + h * kDim, pcol + 32u, vdesc, kIdescO, 1u);
+            }
+            tc::commit(bar_o);
+            tc::commit(bar_vfree + 8 * b);
+            tc::commit(bar_pfree + 8 * b);
+            if (j == it.ntiles - 1) tc::commit(bar_end);
+          }
+          __syncwarp();
+        }
       }
-    } else {
-      bool run = true;
-      for (int j = 0; run && j < ntiles; ++j) run = issue_pv(j);
+      ++n;
     }
   } else if (warp < kSoftmaxWarps) {
     // ------------------------------------- softmax, (row, token half) per thread
     // Each half of the threads runs its own online softmax over its half of
     // every K/V tile, with its own O accumulator in TMEM; the two partial
-    // states of a row are merged once at the end (split-K identity).
+    // states of a row are merged once at the end of the item (split-K
+    // identity).
     const int row = tid & (kRows - 1);
     const int half = tid >> 7;
-    const int t_row = tok0 + row / G;  // chunk token of the row
-    const int h_row = row % G;
-    const bool row_valid = t_row < C;
-    const int p_row = L - C + t_row;  // >= L for rows past the chunk
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tOh = tO + half * kDim;
-    float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
-    float l_sum = 0.f;
     bool run = true;
-    for (int j = 0; run && j < ntiles; ++j) {
-      const int b = j & 1;
-      if (!(run = wait(bar_s + 8 * b, (j >> 1) & 1))) break;
-      tc::fence_after_sync();
-      float x[kHalf];
-      {
-        uint32_t r0[32], r1[32];  // both loads in flight, one wait
-        const uint32_t col = tmem + b * kKv + (lane_off | static_cast<uint32_t>(half * kHalf));
-        tc::ld_32x32b_x32(col, r0);
-        tc::ld_32x32b_x32(col + 32u, r1);
-        tc::wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = __uint_as_float(r0[i]);
-          x[32 + i] = __uint_as_float(r1[i]);
-        }
-      }
-      const int lim = min(p_row + 1, L) - (j * kKv + half * kHalf);  // columns < lim are visible
-      if (lim < kHalf) {
-#pragma unroll
-        for (int c = 0; c < kHalf; ++c) x[c] = c < lim ? x[c] : -INFINITY;
-      }
-      float mp[8];  // eight independent partial maxima, two columns per step
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mp[i] = x[i];
-#pragma unroll
-      for (int c = 8; c < kHalf; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
-      float mt = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
-      mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
-      const bool move = mt > m_ref + kLazyRescale;
-      float alpha = 1.f;
-      if (move) {
-        alpha = fast_exp2(m_ref - mt);  // 0 while m_ref is -inf
-        m_ref = mt;
-        l_sum *= alpha;
-      }
-      if (j > 0 && __any_sync(kFullMask, move)) {
-        // O_h must hold P V(j-1) before it is rescaled.  P V(j-2) is done
-        // (S(j) waited for it) and P V(j) needs this warp's P(j), so
-        // exactly one phase of bar_o can be outstanding here.
-        if (!(run = wait(bar_o, (j - 1) & 1))) break;
+    int n = 0;
+    int jt = 0;
+    for (int k = 0; run; ++k) {
+      const int i = item_index(a, k);
+      if (i < 0) break;
+      Item it;
+      if (!item_at<BS>(a, i, it, tid == 0)) continue;
+      const int t_row = it.tok0 + row / G;  // chunk token of the row
+      const int h_row = row % G;
+      const bool row_valid = t_row < it.C;
+      const int p_row = it.L - it.C + t_row;  // >= L for rows past the chunk
+      float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
+      float l_sum = 0.f;
+      for (int j = 0; j < it.ntiles; ++j, ++jt) {
+        const int b = jt & 1;
+        if (!(run = wait(bar_s + 8 * b, (jt >> 1) & 1))) break;
         tc::fence_after_sync();
-#pragma unroll
-        for (int cc = 0; cc < 4; cc += 2) {
-          uint32_t r0[32], r1[32];
-          const uint32_t col = tOh + (lane_off | static_cast<uint32_t>(cc * 32));
+        float x[kHalf];
+        {
+          uint32_t r0[32], r1[32];  // both loads in flight, one wait
+          const uint32_t col = tmem + b * kKv + (lane_off | static_cast<uint32_t>(half * kHalf));
           tc::ld_32x32b_x32(col, r0);
           tc::ld_32x32b_x32(col + 32u, r1);
           tc::wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            r0[i] = __float_as_uint(__uint_as_float(r0[i]) * alpha);
-            r1[i] = __float_as_uint(__uint_as_float(r1[i]) * alpha);
+          for (int q = 0; q < 32; ++q) {
+            x[q] = __uint_as_float(r0[q]);
+            x[32 + q] = __uint_as_float(r1[q]);
           }
-          tc::st_32x32b_x32(col, r0);
-          tc::st_32x32b_x32(col + 32u, r1);
         }
-        tc::wait_st();
-      }
-      // P of this half into the S buffer's columns of the half (A operand of
-      // P V in tensor memory): high part, then the bf16 residual
-      const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
-      {
-        uint32_t hi[32], lo[32];
-        // column pairs in packed fp32 arithmetic (one instruction per pair)
-        const float2 sc = make_float2(a.scale_log2, a.scale_log2);
-        const float2 nm = make_float2(-mref, -mref);
-        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // independent partial sums
+        const int lim = min(p_row + 1, it.L) - (j * kKv + half * kHalf);  // columns < lim are visible
+        if (lim < kHalf) {
 #pragma unroll
-        for (int e = 0; e < kHalf / 2; ++e) {
-          const float2 t = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc, nm);
-          const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-          ls[e & 1] = __fadd2_rn(ls[e & 1], p);
-          hi[e] = Pack<T>::pack(p.x, p.y);
-          if constexpr (kSplit) {
-            const float2 r = __ffma2_rn(Pack<T>::unpack(hi[e]), make_float2(-1.f, -1.f), p);
-            lo[e] = Pack<T>::pack(r.x, r.y);
+          for (int c = 0; c < kHalf; ++c) x[c] = c < lim ? x[c] : -INFINITY;
+        }
+        float mp[8];  // eight independent partial maxima, two columns per step
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mp[q] = x[q];
+#pragma unroll
+        for (int c = 8; c < kHalf; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
+        float mt = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+        mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
+        const bool move = mt > m_ref + kLazyRescale;
+        float alpha = 1.f;
+        if (move) {
+          alpha = fast_exp2(m_ref - mt);  // 0 while m_ref is -inf
+          m_ref = mt;
+          l_sum *= alpha;
+        }
+        if (j > 0 && __any_sync(kFullMask, move)) {
+          // O_h must hold P V(j-1) before it is rescaled.  P V(j-2) is done
+          // (S(j) waited for it) and P V(j) needs this warp's P(j), so
+          // exactly one phase of bar_o can be outstanding here.
+          if (!(run = wait(bar_o, (jt - 1) & 1))) break;
+          tc::fence_after_sync();
+#pragma unroll
+          for (int cc = 0; cc < 4; cc += 2) {
+            uint32_t r0[32], r1[32];
+            const uint32_t col = tOh + (lane_off | static_cast<uint32_t>(cc * 32));
+            tc::ld_32x32b_x32(col, r0);
+            tc::ld_32x32b_x32(col + 32u, r1);
+            tc::wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              r0[q] = __float_as_uint(__uint_as_float(r0[q]) * alpha);
+              r1[q] = __float_as_uint(__uint_as_float(r1[q]) * alpha);
+            }
+            tc::st_32x32b_x32(col, r0);
+            tc::st_32x32b_x32(col + 32u, r1);
           }
+          tc::wait_st();
         }
-        const float2 lsum = __fadd2_rn(ls[0], ls[1]);
-        l_sum += lsum.x + lsum.y;
-        const uint32_t pcol = tmem + b * kKv + half * kHalf;
-        tc::st_32x32b_x32(pcol + lane_off, hi);
-        if constexpr (kSplit) tc::st_32x32b_x32(pcol + 32u + lane_off, lo);
-        tc::wait_st();
-      }
-      // V(j) landed; tokens past the context get zero rows, so that P = 0
-      // never meets a NaN in stale shared memory
-      const int valid_tok = min(kKv, L - j * kKv);
-      if (valid_tok < kKv) {
-        if (!(run = wait(bar_v + 8 * b, (j >> 1) & 1))) break;
-        uint8_t *vt = smem + kVOff + b * kTile;
-        for (int u = valid_tok * 16 + tid; u < kKv * 16; u += kSoftmaxThreads) {
-          const int r = u >> 4, w = u & 15;  // token row, 16-byte unit of its 256 bytes
-          *reinterpret_cast<uint4 *>(vt + (r >> 3) * kGroupBytes + (w >> 3) * 1024 + (r & 7) * 128 + (w & 7) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
+        // P of this half into the S buffer's columns of the half (A operand
+        // of P V in tensor memory): high part, then the bf16 residual
+        const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
+        {
+          uint32_t hi[32], lo[32];
+          // column pairs in packed fp32 arithmetic (one instruction per pair)
+          const float2 sc = make_float2(a.scale_log2, a.scale_log2);
+          const float2 nm = make_float2(-mref, -mref);
+          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // independent partial sums
+#pragma unroll
+          for (int e = 0; e < kHalf / 2; ++e) {
+            const float2 t = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc, nm);
+            const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+            ls[e & 1] = __fadd2_rn(ls[e & 1], p);
+            hi[e] = Pack<T>::pack(p.x, p.y);
+            if constexpr (kSplit) {
+              const float2 r = __ffma2_rn(Pack<T>::unpack(hi[e]), make_float2(-1.f, -1.f), p);
+              lo[e] = Pack<T>::pack(r.x, r.y);
+            }
+          }
+          const float2 lsum = __fadd2_rn(ls[0], ls[1]);
+          l_sum += lsum.x + lsum.y;
+          const uint32_t pcol = tmem + b * kKv + half * kHalf;
+          tc::st_32x32b_x32(pcol + lane_off, hi);
+          if constexpr (kSplit) tc::st_32x32b_x32(pcol + 32u + lane_off, lo);
+          tc::wait_st();
         }
+        // V(j) landed; tokens past the context get zero rows, so that P = 0
+        // never meets a NaN in stale shared memory
+        const int valid_tok = min(kKv, it.L - j * kKv);
+        if (valid_tok < kKv) {
+          if (!(run = wait(bar_v + 8 * b, (jt >> 1) & 1))) break;
+          uint8_t *vt = smem + kVOff + b * kTile;
+          for (int u = valid_tok * 16 + tid; u < kKv * 16; u += kSoftmaxThreads) {
+            const int r = u >> 4, w = u & 15;  // token row, 16-byte unit of its 256 bytes
+            *reinterpret_cast<uint4 *>(vt + (r >> 3) * kGroupBytes + (w >> 3) * 1024 + (r & 7) * 128 +
+                                       (w & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p + 8 * b);
       }
-      if (valid_tok < kKv) fence_proxy_async_smem();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p + 8 * b);
-    }
-    if (run) run = wait(bar_end, 0);
-    if (run) {
+      if (!run) break;
+      // ---- epilogue of the item: merge the two halves' states of the row
+      if (!(run = wait(bar_end, n & 1))) break;
       tc::fence_after_sync();
-      // merge the two halves' states of the row
       float2 *xch = reinterpret_cast<float2 *>(smem + kXOff);
       xch[half * kRows + row] = make_float2(m_ref, l_sum);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_x);
-      run = wait(bar_x, 0);
-    }
-    if (run) {
-      const float2 *xch = reinterpret_cast<const float2 *>(smem + kXOff);
+      if (!(run = wait(bar_x, n & 1))) break;
       const float2 o0 = xch[row];
       const float2 o1 = xch[kRows + row];
       const float M = fmaxf(o0.x, o1.x);
@@ -465,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float c0 = w0 * inv, c1 = w1 * inv;
       // this thread writes output columns half*64 .. half*64 + 63
       T *orow = static_cast<T *>(a.out) +
-                (static_cast<size_t>(t_begin + t_row) * a.num_q_heads + g * G + h_row) * kDim + half * kHalf;
+                (static_cast<size_t>(it.t_begin + t_row) * a.num_q_heads + it.g * G + h_row) * kDim + half * kHalf;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t r0[32], r1[32];
@@ -479,10 +549,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[8];
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
-              const int i = q4 * 8 + e;
-              const float2 w = __ffma2_rn(make_float2(__uint_as_float(r0[i]), __uint_as_float(r0[i + 1])),
+              const int q = q4 * 8 + e;
+              const float2 w = __ffma2_rn(make_float2(__uint_as_float(r0[q]), __uint_as_float(r0[q + 1])),
                                           make_float2(c0, c0),
-                                          __fmul2_rn(make_float2(__uint_as_float(r1[i]), __uint_as_float(r1[i + 1])),
+                                          __fmul2_rn(make_float2(__uint_as_float(r1[q]), __uint_as_float(r1[q + 1])),
                                                      make_float2(c1, c1)));
               v[e] = w.x;
               v[e + 1] = w.y;
@@ -493,6 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      ++n;
     }
   }
 
@@ -507,6 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if ((warp == kMmaWarp || warp == kPvWarp) && lane == 0) tc::commit(bar_done);
     (void)mbar_wait(bar_done, 0);
     for (int i = 0; i < 2; ++i) {
+      (void)mbar_wait(bar_q + 8 * i, 0);
+      (void)mbar_wait(bar_q + 8 * i, 1);
       (void)mbar_wait(bar_k + 8 * i, 0);
       (void)mbar_wait(bar_k + 8 * i, 1);
       (void)mbar_wait(bar_v + 8 * i, 0);
@@ -591,14 +664,15 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
   if (G > 16 || (kRows % G) != 0) return PKV_ERR_BAD_SHAPE;
   if (!(scale > 0.f) || !(scale < INFINITY)) return PKV_ERR_BAD_SHAPE;
   if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PKV_OK;
-  if (num_seqs > 65535 || cache.num_kv_heads > 65535) return PKV_ERR_TOO_LARGE;
+  if (cache.num_kv_heads > 65535) return PKV_ERR_TOO_LARGE;
   if (!out || !query || !k_cache || !v_cache || !block_tables || !query_start || !context_lens)
     return PKV_ERR_NULL_POINTER;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(query, 16) || !aligned(out, 16) ||
       !aligned(block_tables, 4) || !aligned(query_start, 4) || !aligned(context_lens, 4))
     return PKV_ERR_MISALIGNED;
   const long long qtiles = (static_cast<long long>(max_query_len) * G + kRows - 1) / kRows;
-  if (qtiles > 2147483647ll) return PKV_ERR_TOO_LARGE;
+  const long long items = qtiles * cache.num_kv_heads * num_seqs;
+  if (items > 2147483647ll) return PKV_ERR_TOO_LARGE;
   if ((st = check_device()) != PKV_OK) return st;
 
   CUtensorMap tq, tk, tv;
@@ -618,9 +692,17 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
   args.group = G;
   args.num_blocks = cache.num_blocks;
   args.num_kv_heads = cache.num_kv_heads;
+  args.num_seqs = num_seqs;
+  args.qtiles = static_cast<int>(qtiles);
+  args.items = static_cast<int>(items);
   args.scale_log2 = scale * 1.4426950408889634f;
-  dim3 grid(static_cast<unsigned>(qtiles), static_cast<unsigned>(cache.num_kv_heads),
-            static_cast<unsigned>(num_seqs));
+  // Persistent grid: one CTA per SM (the kernel's shared memory and tensor
+  // memory allow one), each walking its share of the items.
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return PKV_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(items < sms ? items : sms));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return cache.dtype == PKV_BF16 ? launch_prefill_bs<__nv_bfloat16>(cache.block_size, grid, tq, tk, tv, args, s)
                                  : launch_prefill_bs<__half>(cache.block_size, grid, tq, tk, tv, args, s);

@@ -1,0 +1,220 @@
+"""A randomised model of the barrier protocol of the persistent prefill
+kernel (``csrc/paged_prefill.cu``), run on the CPU.
+
+Roles are generators that wait and arrive exactly as the kernel's warps do:
+the K and V load warps (Q tiles into two buffers, K/V tiles into two stages),
+the S-issuing and the P V-issuing MMA warps, and eight softmax warps (with a
+random lazy rescale of O and the per-item epilogue).  mbarriers complete a
+phase when their expected arrivals are in; a wait is the parity test the
+hardware does.  tcgen05 work runs on one in-order pipe, a commit arrives once
+everything its thread issued before it is done; TMA loads land in any order.
+
+Checked on every schedule: no deadlock; every parity wait releases exactly on
+the phase it means (a wait that could be satisfied by an older or a newer
+phase is a bug even when the schedule happens to be benign); no buffer (Q, K
+and V stages, S buffers in tensor memory, O) is rewritten while an
+asynchronous reader is pending, or read before its writer completed.  Each
+synchronisation the kernel relies on, removed, makes some schedule fail.
+"""
+
+import random
+
+import pytest
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.arrivals, self.done = name, count, 0, 0
+
+    def arrive(self):
+        self.arrivals += 1
+        assert self.arrivals <= self.count, f"{self.name}: too many arrivals"
+        if self.arrivals == self.count:
+            self.arrivals, self.done = 0, self.done + 1
+
+
+def run_model(ntiles_per_item, seed, drop=None):
+    """ntiles_per_item: K/V tiles of each item of one CTA (0 = an empty item,
+    skipped by every role).  drop: name of one synchronisation to remove."""
+    rnd = random.Random(seed)
+    bars = {}
+
+    def bar(name, count=1):
+        bars[name] = Bar(name, count)
+
+    for i in range(2):
+        for nm in ("q", "qfree", "k", "kfree", "v", "vfree", "s", "pfree"):
+            bar(f"{nm}{i}")
+        bar(f"p{i}", 8)
+    bar("o")
+    bar("end")
+    bar("x", 8)
+    pipe, loads = [], []
+    pending = {}          # resource -> list of async ops reading it
+    s_ops = {}            # global tile -> S op
+    st = {"pv_item": -1, "o_readers": 0}
+
+    def wait(name, phase):
+        b = bars[name]
+        while (b.done & 1) == (phase & 1):
+            assert b.done <= phase, f"{name}: phase {phase} overtaken ({b.done} done)"
+            yield
+        assert b.done == phase + 1, f"{name}: released with {b.done} phases done, meant phase {phase}"
+
+    def busy(res):
+        return [op for op in pending.get(res, []) if not op["done"]]
+
+    def read(op, *res):
+        for r in res:
+            pending.setdefault(r, []).append(op)
+
+    items = [n for n in ntiles_per_item]
+
+    def producer(kind):
+        n = jt = 0
+        for nt in items:
+            if nt == 0:
+                continue
+            if kind == "K":
+                qb = n & 1
+                if n >= 2 and drop != "qfree":
+                    yield from wait(f"qfree{qb}", (n - 2) >> 1)
+                assert not busy(f"Q{qb}"), "Q buffer rewritten while S reads it"
+                loads.append((f"q{qb}", {"done": False}))
+            for _ in range(nt):
+                b = jt & 1
+                if jt >= 2:
+                    yield from wait(f"{kind.lower()}free{b}", (jt - 2) >> 1)
+                assert not busy(f"{kind}{b}"), f"{kind} stage rewritten while read"
+                loads.append((f"{kind.lower()}{b}", {"done": False}))
+                jt += 1
+                yield
+            n += 1
+
+    def s_issuer():
+        n = jt = 0
+        for nt in items:
+            if nt == 0:
+                continue
+            qb = n & 1
+            yield from wait(f"q{qb}", n >> 1)
+            for j in range(nt):
+                b = jt & 1
+                if jt >= 2 and drop != "pfree":
+                    yield from wait(f"pfree{b}", (jt - 2) >> 1)
+                yield from wait(f"k{b}", jt >> 1)
+                assert not busy(f"S{b}"), "S buffer rewritten while P V reads P"
+                op = {"done": False}
+                read(op, f"Q{qb}", f"K{b}")
+                s_ops[jt] = op
+                pipe.extend([("op", op), ("commit", f"s{b}"), ("commit", f"kfree{b}")])
+                if j == nt - 1:
+                    pipe.append(("commit", f"qfree{qb}"))
+                jt += 1
+                yield
+            n += 1
+
+    def pv_issuer():
+        n = jt = 0
+        for nt in items:
+            if nt == 0:
+                continue
+            for j in range(nt):
+                b = jt & 1
+                yield from wait(f"v{b}", jt >> 1)
+                yield from wait(f"p{b}", jt >> 1)
+                assert st["o_readers"] == 0, "P V writes O while a softmax warp reads it"
+                op = {"done": False}
+                read(op, f"V{b}", f"S{b}")
+                pending.setdefault("O", []).append(op)
+                st["pv_item"] = max(st["pv_item"], n)
+                pipe.extend([("op", op), ("commit", "o"), ("commit", f"vfree{b}"), ("commit", f"pfree{b}")])
+                if j == nt - 1 and drop != "end":
+                    pipe.append(("commit", "end"))
+                jt += 1
+                yield
+            n += 1
+
+    def softmax():
+        n = jt = 0
+        for nt in items:
+            if nt == 0:
+                continue
+            for j in range(nt):
+                b = jt & 1
+                yield from wait(f"s{b}", jt >> 1)
+                assert s_ops[jt]["done"], "S read before its MMA completed"
+                if j > 0 and rnd.random() < 0.3:
+                    yield from wait("o", jt - 1)
+                    assert not busy("O"), "O rescaled while a P V is pending"
+                    st["o_readers"] += 1
+                    yield
+                    st["o_readers"] -= 1
+                yield
+                bars[f"p{b}"].arrive()
+                jt += 1
+            if drop == "end":
+                yield from wait("o", jt - 1)
+            else:
+                yield from wait("end", n)
+            assert not busy("O"), "epilogue reads O with a P V pending"
+            bars["x"].arrive()
+            yield from wait("x", n)
+            st["o_readers"] += 1
+            yield
+            assert st["pv_item"] <= n, "next item's P V issued while O is read out"
+            st["o_readers"] -= 1
+            yield
+            n += 1
+
+    roles = [producer("K"), producer("V"), s_issuer(), pv_issuer()] + [softmax() for _ in range(8)]
+    alive = list(range(len(roles)))
+    for _ in range(400000):
+        if not (alive or pipe or loads):
+            return
+        r = rnd.random()
+        if pipe and r < 0.15:
+            kind, x = pipe.pop(0)
+            if kind == "op":
+                x["done"] = True
+            else:
+                bars[x].arrive()
+            continue
+        if loads and r < 0.3:
+            name, op = loads.pop(rnd.randrange(len(loads)))
+            op["done"] = True
+            bars[name].arrive()
+            continue
+        if alive:
+            k = rnd.choice(alive)
+            try:
+                next(roles[k])
+            except StopIteration:
+                alive.remove(k)
+    raise AssertionError("deadlock")
+
+
+def _items(seed):
+    rnd = random.Random(seed)
+    return [rnd.choice([0, 1, 1, 2, 3, 5, 8]) for _ in range(rnd.randint(1, 9))]
+
+
+def test_protocol_holds_on_random_schedules():
+    for seed in range(300):
+        run_model(_items(seed), seed)
+
+
+@pytest.mark.parametrize("drop", ["qfree", "pfree", "end"])
+def test_each_synchronisation_is_needed(drop):
+    """Removing the Q-buffer release, the S-buffer release (P V done) or the
+    one-phase final barrier (falling back to a parity wait on the per-tile
+    P V barrier) breaks some schedule."""
+    failures = 0
+    for seed in range(300):
+        try:
+            run_model(_items(seed), seed, drop=drop)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
