@@ -112,8 +112,9 @@ struct PrefillArgs {
 // numbered in groups of kPairsPerGroup (sequence, kv head) pairs; inside a
 // group, longest first (query tile qtiles - 1 of each pair, then qtiles - 2,
 // ...: later query tiles see more keys).  The CTAs working at one time then
-// share the K/V of a few pairs, which stay in L2.
-constexpr int kPairsPerGroup = 8;
+// share the K/V of a few pairs, which stay in L2 (one pair per group measured
+// best: 1 to 4 % over groups of 2 to 8 pairs).
+constexpr int kPairsPerGroup = 1;
 struct Item {
   int s, g, t_begin, C, L, tok0, ntiles, nb;
 };
