@@ -191,8 +191,9 @@ PKV_API int32_t pkv_paged_attention_partition_size(int32_t num_seqs, int32_t num
  * workspace        device, >= pkv_paged_attention_workspace_size(...) bytes,
  *                  16-byte aligned; may be NULL when that size is 0.  Holds
  *                  one arrival counter per (sequence, kv head) and the split
- *                  partials; the call zeroes the counters itself (an async
- *                  memset on `stream`), so no content is expected on entry.
+ *                  partials; the call zeroes the counters itself (in its
+ *                  planning kernel, else with an async memset on `stream`),
+ *                  so no content is expected on entry.
  * Errors: host checks -> status.  A table entry outside [0, num_blocks) ->
  *   PKV_DEV_BAD_BLOCK and that block is treated as empty; a context length
  *   outside [0, min(max_context_len, max_blocks_per_seq*B)] -> PKV_DEV_BAD_LEN
