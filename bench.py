@@ -203,6 +203,30 @@ def step_bytes(batch, kv_bytes=2):
     return att, write, copy
 
 
+def decode_accounting(batch, kv_bytes: int, ms_step: float) -> dict:
+    """Side figures of a decode step beside the headline GB/s: internal
+    fragmentation of the pool's used blocks, K/V bytes counted whole-block and
+    per distinct physical block (a shared prefix once), and the rates those
+    give, plus the cache write + attention rate."""
+    from paged_kv_cache_407_b200 import accounting as A
+
+    att, write, copy = step_bytes(batch, kv_bytes=kv_bytes)
+    padded = A.decode_bytes_padded_kv(batch.context_lens, batch.num_kv_heads, batch.head_dim, batch.block_size,
+                                      elem_bytes=kv_bytes)
+    unique = A.unique_kv_bytes(batch.block_tables, batch.context_lens, batch.num_kv_heads, batch.head_dim,
+                               batch.block_size, elem_bytes=kv_bytes)
+    other = att["total"] - att["kv"]
+    sec = ms_step * 1e-3
+    return {
+        "pool_fragmentation": round(A.block_fragmentation(batch.context_lens, batch.block_size), 5),
+        "kv_bytes_logical": att["kv"],
+        "kv_bytes_padded_to_blocks": padded,
+        "kv_bytes_unique_blocks": unique,
+        "unique_gbs": round((unique + other) / sec / 1e9, 2),
+        "write_plus_attention_gbs": round((att["total"] + write) / sec / 1e9, 2),
+    }
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -755,6 +779,7 @@ def run_ours(args):
         "bytes_per_step": {"attention": att_bytes["total"], "attention_kv": att_bytes["kv"],
                            "cache_write": write_bytes, "block_copy": copy_bytes},
         "attention_ms_per_call": round(att_ms_max, 5),
+        "kv_accounting": decode_accounting(batch, 1 if e4m3 else 2, ms_step),
         "split_k": {"partition_tokens": P, "split": bool(split)},
         "roofline": {
             "bound": "hbm",

@@ -36,6 +36,22 @@ def decode_bytes_padded_kv(context_lens, num_kv_heads: int, head_dim: int, block
     return int(nb.sum()) * block_size * num_kv_heads * head_dim * elem_bytes * 2
 
 
+def unique_kv_bytes(block_tables, context_lens, num_kv_heads: int, head_dim: int, block_size: int,
+                    elem_bytes: int = 2) -> int:
+    """K+V bytes of the distinct physical blocks a call reads, each at the
+    largest number of its tokens any sequence uses (a block shared by several
+    sequences' tables counts once)."""
+    tables = np.asarray(block_tables)
+    lens = np.asarray(context_lens, dtype=np.int64)
+    used = {}
+    for s, L in enumerate(lens):
+        nb = (int(L) + block_size - 1) // block_size
+        for j in range(nb):
+            blk = int(tables[s, j])
+            used[blk] = max(used.get(blk, 0), min(block_size, int(L) - j * block_size))
+    return sum(used.values()) * num_kv_heads * head_dim * elem_bytes * 2
+
+
 def reshape_and_cache_bytes(num_tokens: int, num_kv_heads: int, head_dim: int,
                             elem_bytes: int = 2, cache_elem_bytes: int | None = None) -> int:
     """Read the new K and V rows, write them into the pool, read the slots."""

@@ -55,3 +55,39 @@ def test_prefill_flops_is_the_causal_count():
     assert A.prefill_flops(lens, chunks, Hq, D) == brute
     assert A.prefill_flops([4096] * 4, [4096] * 4, 32, 128) == 4 * 4 * 128 * 32 * 4096 * 4097 // 2
     assert A.prefill_bytes([100], [20], 8, 2, 64) == 100 * 2 * 64 * 2 * 2 + 20 * 8 * 64 * 2 * 2
+
+
+def test_unique_kv_bytes_counts_a_shared_block_once():
+    """Two sequences whose tables share their first two blocks: the shared
+    blocks count once, each at the most tokens any sequence uses in it; with
+    disjoint tables the unique count equals the logical one."""
+    Hkv, D, B = 2, 8, 4
+    per_token = Hkv * D * 2 * 2
+    tables = np.array([[5, 6, 7, -1], [5, 6, 9, 3]])
+    lens = [10, 13]  # seq 0: 4 + 4 + 2 tokens; seq 1: 4 + 4 + 4 + 1
+    assert A.unique_kv_bytes(tables, lens, Hkv, D, B) == (4 + 4 + 2 + 4 + 1) * per_token
+    disjoint = np.array([[1, 2, 3, -1], [4, 5, 6, 7]])
+    logical = A.decode_bytes(lens, 4, Hkv, D, B)["kv"]
+    assert A.unique_kv_bytes(disjoint, lens, Hkv, D, B) == logical
+    # a block shared where one sequence fills it and the other uses its head
+    assert A.unique_kv_bytes(np.array([[0, -1], [0, 1]]), [2, 6], Hkv, D, B) == (4 + 2) * per_token
+
+
+def test_bench_decode_accounting_on_the_workloads():
+    """The bench's side figures on the prefix workload: the shared 1024-token
+    prefix counts once in the unique bytes; with private tables (7B batch)
+    unique equals logical."""
+    import bench
+    import workloads as W
+
+    b = W.WORKLOADS["prefix_share"]()
+    acc = bench.decode_accounting(b, 2, 1.0)
+    per_token = b.num_kv_heads * b.head_dim * 2 * 2
+    suffix = int(np.sum(np.asarray(b.context_lens) - 1024))
+    # prefix blocks 0..62 shared by every table; block 63 copied per sequence
+    assert acc["kv_bytes_unique_blocks"] == (63 * 16 + len(b.context_lens) * 16 + suffix) * per_token
+    assert acc["kv_bytes_logical"] == int(np.sum(b.context_lens)) * per_token
+    b7 = W.WORKLOADS["tiny"]()
+    acc7 = bench.decode_accounting(b7, 2, 1.0)
+    assert acc7["kv_bytes_unique_blocks"] == acc7["kv_bytes_logical"]
+    assert acc7["kv_bytes_padded_to_blocks"] >= acc7["kv_bytes_logical"]
