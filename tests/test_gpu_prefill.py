@@ -163,3 +163,35 @@ def test_long_chunks_sampled_rows_and_repeat_calls_bit_identical():
             hs = [h for h in range(Hq) if O.kv_head_of(h, Hq, Hkv) == g]
             ref[i, hs] = O.attend(q[hs], K[g, : p + 1], V[g, : p + 1], b.scale)
     compare(bits(outs[0])[rows], ref, W.BF16, "long chunks, sampled rows")
+
+
+@pytest.mark.parametrize("name", sorted(W.PREFILL_WORKLOADS))
+def test_bench_prefill_workloads_sampled_rows(name):
+    """The bench's prefill batches at full size, in the launch the bench times:
+    sampled rows (every 509th token, all heads) against the oracle, and no
+    device status."""
+    b = W.PREFILL_WORKLOADS[name]()
+    db = upload_prefill(b)
+    st = status_tensor()
+    pkv.reshape_and_cache(db.key, db.value, db.k_cache, db.v_cache, db.slot_mapping, d_status=st)
+    out = torch.empty_like(db.q)
+    pkv.paged_prefill(out, db.q, db.k_cache, db.v_cache, db.block_tables, db.query_start, db.context_lens,
+                      b.max_query_len, b.scale, d_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    kc, vc = O.reshape_and_cache(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, b.block_size)
+    rows = np.arange(0, b.num_tokens, 509)
+    qs = np.asarray(b.query_start)
+    Hq, Hkv = b.q.shape[1], kc.shape[1]
+    ref = np.zeros((len(rows),) + b.q.shape[1:])
+    for i, t in enumerate(rows):
+        s = int(np.searchsorted(qs, t, side="right") - 1)
+        L, C = int(b.context_lens[s]), int(qs[s + 1] - qs[s])
+        p = L - C + (t - qs[s])
+        K = O.decode_bits(O.materialize(kc, b.block_tables[s], p + 1, b.block_size), b.dtype)
+        V = O.decode_bits(O.materialize(vc, b.block_tables[s], p + 1, b.block_size), b.dtype)
+        q = O.decode_bits(b.q[t], b.dtype)
+        for g in range(Hkv):
+            hs = [h for h in range(Hq) if O.kv_head_of(h, Hq, Hkv) == g]
+            ref[i, hs] = O.attend(q[hs], K[g], V[g], b.scale)
+    compare(bits(out)[rows], ref, b.dtype, f"{name}, sampled rows")
