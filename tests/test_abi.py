@@ -103,3 +103,30 @@ def test_workspace_and_partition_queries(lib):
     assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 512) == 144 + 4 * 256 * 8 + 4 * 32 * 256 * 130 * 4
     assert bd.workspace_size(3, 4, 1, 64, 16, 2000, 256) == 16 + 3 * 8 * 8 + 3 * 4 * 8 * 66 * 4
     assert bd.workspace_size(4, 32, 8, 128, 32, 131072, 24) == 0  # invalid partition
+
+
+def test_prefill_host_validation_without_device(lib):
+    """pkv_paged_prefill checks its arguments on the host before it looks for
+    a device: each broken rule returns its status, empty calls return OK."""
+    null = None
+    A = ctypes.c_void_p(0x10000)       # 16-byte aligned stand-ins, never dereferenced
+    odd = ctypes.c_void_p(0x10008)     # 8-byte aligned only
+    pre = lib.pkv_paged_prefill
+
+    def call(desc=None, out=A, q=A, k=A, v=A, tables=A, qs=A, lens=A, S=2, T=64, maxq=32, Hq=8,
+             scale=0.125):
+        return pre(out, q, k, v, desc or _desc(N=64, B=16, H=4, D=128), tables, 8, qs, lens, S, T, maxq, Hq,
+                   ctypes.c_float(scale), null, null)
+
+    assert call(desc=_desc(D=64)) == 3                 # head_dim must be 128
+    assert call(desc=_desc(D=128, dt=2)) == 2          # 8-bit pools: not for prefill
+    assert call(Hq=6) == 3                             # Hq not a multiple of Hkv
+    assert call(Hq=4 * 32) == 3                        # group of 32 > 16
+    assert call(Hq=12, desc=_desc(N=64, B=16, H=4, D=128)) == 3  # group of 3 does not divide 128 rows
+    assert call(scale=0.0) == 3
+    assert call(scale=float("inf")) == 3
+    assert call(S=0) == 0 and call(T=0) == 0 and call(maxq=0) == 0  # nothing to do
+    assert call(q=null) == 1 and call(lens=null) == 1 and call(qs=null) == 1
+    assert call(k=odd) == 4 and call(out=odd) == 4     # pools and rows must be 16-byte aligned
+    # query tiles x kv heads x sequences beyond 2^31 - 1
+    assert call(S=40, maxq=2**31 - 1, Hq=4) == 7
