@@ -130,3 +130,24 @@ def test_prefill_host_validation_without_device(lib):
     assert call(k=odd) == 4 and call(out=odd) == 4     # pools and rows must be 16-byte aligned
     # query tiles x kv heads x sequences beyond 2^31 - 1
     assert call(S=40, maxq=2**31 - 1, Hq=4) == 7
+
+
+def test_split_state_calls_validate_on_the_host(lib):
+    """The attention-state entry points of the cross-GPU split check their
+    arguments before any device work."""
+    null = None
+    A = ctypes.c_void_p(0x10000)
+    merge = lib.pkv_merge_attention_states
+    assert merge(A, 2, A, 129, 2, 1, 128, null) == 2        # 8-bit output: not accepted
+    assert merge(A, 0, A, 97, 2, 1, 96, null) == 3          # head_dim 96
+    assert merge(A, 0, A, 128, 2, 1, 128, null) == 3        # stride below rows * (D + 1)
+    assert merge(A, 0, A, 0, 2, 0, 128, null) == 0          # no rows: nothing to do
+    assert merge(null, 0, A, 129, 2, 1, 128, null) == 1
+    assert merge(A, 0, null, 129, 2, 1, 128, null) == 1
+    assert merge(A, 1, ctypes.c_void_p(0x10002), 129, 2, 1, 128, null) == 4
+    lse = lib.pkv_paged_attention_decode_lse
+    desc = _desc(N=16, B=16, H=4, D=64)
+    # NULL log-sum-exp output with sequences to do
+    assert lse(A, null, A, A, A, desc, A, 4, A, 2, 4, 64, ctypes.c_float(0.125), 0, null, 0, null, null) == 1
+    # otherwise the decode rules: partition not a multiple of the block size
+    assert lse(A, A, A, A, A, desc, A, 4, A, 2, 4, 64, ctypes.c_float(0.125), 24, null, 0, null, null) == 6
