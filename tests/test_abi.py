@@ -151,3 +151,39 @@ def test_split_state_calls_validate_on_the_host(lib):
     assert lse(A, null, A, A, A, desc, A, 4, A, 2, 4, 64, ctypes.c_float(0.125), 0, null, 0, null, null) == 1
     # otherwise the decode rules: partition not a multiple of the block size
     assert lse(A, A, A, A, A, desc, A, 4, A, 2, 4, 64, ctypes.c_float(0.125), 24, null, 0, null, null) == 6
+
+
+def test_fp8_calls_validate_on_the_host(lib):
+    """The 8-bit write and decode check pool dtype, shapes, scales, pointers,
+    alignment and workspace on the host."""
+    null = None
+    A = ctypes.c_void_p(0x10000)
+    f8 = _desc(N=16, B=16, H=4, D=128, dt=2)
+    wr = lib.pkv_reshape_and_cache_fp8
+    f = ctypes.c_float
+
+    def write(desc=f8, in_dt=0, T=3, ks=0.5, vs=0.5, key=A):
+        return wr(key, A, 0, 0, in_dt, A, A, desc, A, T, f(ks), f(vs), null, null)
+
+    assert write(desc=_desc(N=16, B=16, H=4, D=128, dt=0)) == 2   # 16-bit pool
+    assert write(in_dt=2) == 2                                      # 8-bit input
+    assert write(desc=_desc(N=16, B=8, H=4, D=128, dt=2)) == 3      # 8-token blocks
+    assert write(ks=0.0) == 3 and write(vs=float("nan")) == 3
+    assert write(T=0) == 0
+    assert write(key=null) == 1
+    dec = lib.pkv_paged_attention_decode_fp8
+
+    def decode(desc=f8, q_dt=1, ks=0.5, P=0, ws=null, ws_bytes=0, maxlen=64, out=A):
+        return dec(out, A, q_dt, A, A, desc, A, 64, A, 2, 8, maxlen, f(0.125), f(ks), f(0.5), P, ws, ws_bytes,
+                   null, null)
+
+    assert decode(desc=_desc(N=16, B=16, H=4, D=64, dt=2)) == 3    # head_dim 64 on 8-bit pools
+    assert decode(q_dt=2) == 2
+    assert decode(ks=-1.0) == 3
+    assert decode(P=24) == 6
+    assert decode(out=ctypes.c_void_p(0x10002)) == 4
+    # a call that splits needs its workspace
+    need = bd.workspace_size(2, 8, 4, 128, 16, 1024, 256)
+    assert need > 0
+    assert decode(P=256, maxlen=1024) == 5
+    assert decode(P=256, maxlen=1024, ws=A, ws_bytes=need - 1) == 5
