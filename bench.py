@@ -203,6 +203,12 @@ def step_bytes(batch, kv_bytes=2):
     return att, write, copy
 
 
+def split_partials_bytes(batch, partition_tokens: int) -> int:
+    from paged_kv_cache_407_b200 import accounting as A
+
+    return A.split_partials_bytes(batch.context_lens, batch.num_q_heads, batch.head_dim, partition_tokens)
+
+
 def decode_accounting(batch, kv_bytes: int, ms_step: float) -> dict:
     """Side figures of a decode step beside the headline GB/s: internal
     fragmentation of the pool's used blocks, K/V bytes counted whole-block and
@@ -780,7 +786,8 @@ def run_ours(args):
                            "cache_write": write_bytes, "block_copy": copy_bytes},
         "attention_ms_per_call": round(att_ms_max, 5),
         "kv_accounting": decode_accounting(batch, 1 if e4m3 else 2, ms_step),
-        "split_k": {"partition_tokens": P, "split": bool(split)},
+        "split_k": {"partition_tokens": P, "split": bool(split), "workspace_bytes": ws_bytes,
+                    "partials_bytes_moved": split_partials_bytes(batch, P)},
         "roofline": {
             "bound": "hbm",
             "kernel": "paged_attention_decode (attention kernel + log-sum-exp merge, timed together)",

@@ -52,6 +52,16 @@ def unique_kv_bytes(block_tables, context_lens, num_kv_heads: int, head_dim: int
     return sum(used.values()) * num_kv_heads * head_dim * elem_bytes * 2
 
 
+def split_partials_bytes(context_lens, num_q_heads: int, head_dim: int, partition_tokens: int) -> int:
+    """Workspace traffic of split-K (implementation overhead, not algorithmic):
+    every sequence that spans more than one partition writes one fp32 (m, l,
+    o[D]) state per (query head, partition) and its merge reads each back."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    parts = (lens + partition_tokens - 1) // partition_tokens
+    states = int(parts[parts > 1].sum()) * num_q_heads
+    return states * (head_dim + 2) * 4 * 2
+
+
 def reshape_and_cache_bytes(num_tokens: int, num_kv_heads: int, head_dim: int,
                             elem_bytes: int = 2, cache_elem_bytes: int | None = None) -> int:
     """Read the new K and V rows, write them into the pool, read the slots."""

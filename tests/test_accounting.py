@@ -91,3 +91,16 @@ def test_bench_decode_accounting_on_the_workloads():
     acc7 = bench.decode_accounting(b7, 2, 1.0)
     assert acc7["kv_bytes_unique_blocks"] == acc7["kv_bytes_logical"]
     assert acc7["kv_bytes_padded_to_blocks"] >= acc7["kv_bytes_logical"]
+
+
+def test_split_partials_bytes():
+    """Only sequences spanning several partitions write and read states:
+    lengths 100, 600, 1025 at P = 512 -> 0 + 2 + 3 states per query head."""
+    assert A.split_partials_bytes([100, 600, 1025], 4, 128, 512) == (2 + 3) * 4 * 130 * 4 * 2
+    assert A.split_partials_bytes([512, 1], 8, 64, 512) == 0
+    import types
+
+    import bench
+
+    long_ctx = types.SimpleNamespace(context_lens=[131072] * 4, num_q_heads=32, head_dim=128)
+    assert bench.split_partials_bytes(long_ctx, 512) == 4 * 256 * 32 * 130 * 4 * 2  # 34 MB per call
