@@ -146,6 +146,12 @@ def run_model(ntiles_per_item, seed, drop=None):
                 b = jt & 1
                 yield from wait(f"s{b}", jt >> 1)
                 assert s_ops[jt]["done"], "S read before its MMA completed"
+                if j == nt - 1 and rnd.random() < 0.5:
+                    # the item's last tile reaches past the context: this warp
+                    # zeroes the tail rows of the V stage before arriving on P
+                    yield from wait(f"v{b}", jt >> 1)
+                    assert not busy(f"V{b}"), "V stage zeroed while a P V reads it"
+                    assert not any(name == f"v{b}" for name, _ in loads), "V stage zeroed under a landing load"
                 if j > 0 and rnd.random() < 0.3:
                     yield from wait("o", jt - 1)
                     assert not busy("O"), "O rescaled while a P V is pending"
