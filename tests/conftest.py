@@ -22,6 +22,22 @@ def pytest_collection_modifyitems(config, items):
     return
 
 
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print the error statistics of every GPU-vs-oracle comparison of the run
+    (maximum absolute and relative error, the storage floor of the output
+    dtype, and whether the literal 2e-3 / 1e-2 limits hold)."""
+    parity = sys.modules.get("parity")
+    records = getattr(parity, "RECORDS", None)
+    if not records:
+        return
+    tr = terminalreporter
+    tr.section("parity statistics (gpu vs fp64 oracle)")
+    tr.write_line(f"{'comparison':62s} {'dtype':5s} {'max_abs':>9s} {'max_rel':>9s} {'floor':>9s} literal")
+    for where, dtype, st in records:
+        tr.write_line(f"{where[:62]:62s} {dtype:5s} {st['max_abs']:9.2e} {st['max_rel']:9.2e} "
+                      f"{st['storage_floor_abs']:9.2e} {'yes' if st['literal_ok'] else 'no'}")
+
+
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(HERE, "golden")

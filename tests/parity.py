@@ -1,12 +1,22 @@
 """Helpers shared by the GPU parity tests: run a batch through the C-ABI
 binding and compare with the oracle.
 
-Tolerance for attention outputs (fp16/bf16 storage, fp32 accumulation), per
-element: |gpu - oracle| <= ATOL + RTOL * |oracle|, with ATOL = 2e-3 and
-RTOL = 1e-2.  Rounding the exact result to bf16 alone moves it by up to
-2^-8 |x| (3.9e-3 at |x| = 1), so a plain absolute bound of 2e-3 cannot hold
-for every element of a bf16 output; the combined bound can.  Cache writes and
-block copies must match bit for bit.
+Tolerance for attention outputs (fp16/bf16 storage, fp32 accumulation): a
+maximum absolute error of 2e-3 and a maximum relative error of 1e-2.
+
+* Every output, fp16 or bf16, must satisfy the combined per-element bound
+  |gpu - oracle| <= ATOL + RTOL * |oracle| (ATOL = 2e-3, RTOL = 1e-2).
+* fp16 outputs must also satisfy the two limits literally and separately:
+  max |gpu - oracle| <= 2e-3 over every element, and max |gpu - oracle| /
+  |oracle| <= 1e-2 over the elements with |oracle| >= 0.2 (below that the
+  relative error of a value near zero says nothing).
+* bf16 outputs are held to the combined bound only: rounding the exact result
+  to bf16 alone moves a value in [1, 2) by up to 2^-8 (3.9e-3), so a plain
+  absolute bound of 2e-3 cannot hold for every element of a bf16 output.
+  The statistics record that storage floor beside the measured error.
+
+Cache writes and block copies must match bit for bit.  Every comparison's
+statistics are kept in RECORDS and printed at the end of the pytest run.
 """
 
 from __future__ import annotations
@@ -22,30 +32,58 @@ ATOL = 2e-3
 RTOL = 1e-2
 
 
-def compare(gpu_bits: np.ndarray, ref: np.ndarray, dtype: str, where: str = "") -> dict:
+LITERAL_REL_FLOOR = 0.2  # relative errors are taken over |oracle| >= this
+
+# (where, dtype, statistics) of every comparison made in this process
+RECORDS: list[tuple[str, str, dict]] = []
+
+
+def error_stats(got: np.ndarray, ref: np.ndarray, dtype: str) -> dict:
+    """Maximum absolute and relative errors of float64 values ``got`` against
+    ``ref``, the error that rounding ``ref`` to ``dtype`` alone would leave,
+    and whether the combined and the literal bounds hold."""
+    err = np.abs(got - ref)
+    big = np.abs(ref) >= LITERAL_REL_FLOOR
+    floor = np.abs(O.decode_bits(O.encode_bits(ref, dtype), dtype) - ref)
+    max_abs = float(err.max())
+    max_rel = float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0
+    return {
+        "max_abs": max_abs,
+        "max_rel": max_rel,
+        "storage_floor_abs": float(floor.max()),
+        "combined_ok": bool(np.all(err <= ATOL + RTOL * np.abs(ref))),
+        "literal_ok": bool(max_abs <= ATOL and max_rel <= RTOL),
+        "n": int(err.size),
+    }
+
+
+def compare(gpu_bits: np.ndarray, ref: np.ndarray, dtype: str, where: str = "",
+            literal: bool | None = None) -> dict:
     """Element-wise check of fp16/bf16 GPU output bits against float64 oracle
-    values (rows of ``ref`` that are NaN are not compared)."""
+    values (rows of ``ref`` that are NaN are not compared).  Asserts the
+    combined bound always and the literal limits when ``literal`` (default:
+    for fp16 outputs); returns the statistics."""
     got = O.decode_bits(gpu_bits, dtype)
     rows = ~np.isnan(ref).any(axis=-1)
     got, ref = got[rows], ref[rows]
     assert got.size > 0, "nothing compared"
+    if literal is None:
+        literal = dtype == "f16"
+    stats = error_stats(got, ref, dtype)
+    RECORDS.append((where, dtype, stats))
     err = np.abs(got - ref)
-    bound = ATOL + RTOL * np.abs(ref)
-    bad = ~(err <= bound)
+    bad = ~(err <= ATOL + RTOL * np.abs(ref))
     if bad.any():
         idx = np.argwhere(bad)[0]
         raise AssertionError(
             f"{where}: {int(bad.sum())} of {bad.size} elements outside {ATOL} + {RTOL}|ref|; "
             f"first at {tuple(idx)}: gpu={got[tuple(idx)]!r} ref={ref[tuple(idx)]!r}; "
             f"max abs err {err.max():.3e}")
-    big = np.abs(ref) >= 0.2
-    floor = np.abs(O.decode_bits(O.encode_bits(ref, dtype), dtype) - ref)
-    return {
-        "max_abs": float(err.max()),
-        "max_rel": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
-        "storage_floor_abs": float(floor.max()),
-        "n": int(err.size),
-    }
+    if literal:
+        assert stats["literal_ok"], (
+            f"{where}: max abs err {stats['max_abs']:.3e} (limit {ATOL}) / max rel err "
+            f"{stats['max_rel']:.3e} over |ref| >= {LITERAL_REL_FLOOR} (limit {RTOL})")
+    return stats
 
 
 def status_tensor(device="cuda"):

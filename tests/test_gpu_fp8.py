@@ -141,13 +141,62 @@ def test_fp8_copy_blocks_bit_exact():
     assert np.array_equal(_u8(db.k_cache), kc) and np.array_equal(_u8(db.v_cache), vc)
 
 
-def test_fp8_llama7b_shaped_sampled():
-    base = W.llama7b_mha()
-    f8 = W.fp8_variant(base, 21)
+@pytest.mark.parametrize("dtype,B", [(W.F16, 16), (W.BF16, 32), (W.F16, 64)])
+def test_fp8_decode_every_finite_code(dtype, B):
+    """Pools whose codes cover all 254 finite E4M3 codes (subnormal, small and
+    large exponent fields alike), not only the mid-range codes the other
+    cases draw; scales keep the dequantised values O(1)."""
+    base = W.small_case(470 + B, num_seqs=12, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=B,
+                        dtype=dtype, max_len=700, partition_size=0)
+    f8 = W.fp8_variant(base, 13, k_scale=1.0 / 64.0, v_scale=1.0 / 448.0, full_range=True)
+    seen = set()
+    for s in range(base.num_seqs):
+        L = int(base.context_lens[s])
+        nb = -(-L // B)
+        seen |= set(np.unique(f8.k_cache[base.block_tables[s, :nb]]).tolist())
+        seen |= set(np.unique(f8.v_cache[base.block_tables[s, :nb]]).tolist())
+    assert seen >= set(range(256)) - {0x7F, 0xFF}, "the pools do not hold every finite code"
     st = status_tensor()
     db = _fp8_step(f8, d_status=st)
-    seqs = sorted(np.random.default_rng(2).choice(base.num_seqs, 6, replace=False).tolist())
-    kc, vc, ref = _oracle_step(f8, seqs=seqs)
+    kc, vc, ref = _oracle_step(f8)
     assert np.array_equal(_u8(db.k_cache), kc) and np.array_equal(_u8(db.v_cache), vc)
-    compare(db.out.view(torch.int16).cpu().numpy().view(np.uint16), ref, W.F16, "fp8 7B")
+    compare(db.out.view(torch.int16).cpu().numpy().view(np.uint16), ref, dtype,
+            f"fp8 decode, every finite code, {dtype} B{B}")
     assert int(st.item()) == 0
+
+
+# ------------------------------------------------ bench batches at full size
+# The 8-bit variants of the decode batches that the benchmark times with
+# --kv-dtype e4m3, built with the same seed (777) and run in the same launch
+# configuration (the batch's own partition size: automatic, or 512 tokens for
+# the long-context batch); the oracle computes a seeded sample of sequences.
+
+def _fp8_bench_case(base, sample, where):
+    f8 = W.fp8_variant(base, 777)
+    st = status_tensor()
+    db = _fp8_step(f8, partition_size=base.partition_size, d_status=st)
+    assert int(st.item()) == 0
+    kc, vc, ref = _oracle_step(f8, seqs=sample)
+    assert np.array_equal(_u8(db.k_cache), kc) and np.array_equal(_u8(db.v_cache), vc)
+    return compare(db.out.view(torch.int16).cpu().numpy().view(np.uint16), ref, base.dtype, where)
+
+
+def test_fp8_llama7b_shaped_sampled():
+    base = W.llama7b_mha()
+    seqs = sorted(np.random.default_rng(2).choice(base.num_seqs, 6, replace=False).tolist())
+    stats = _fp8_bench_case(base, seqs, "fp8 llama7b_mha (bench batch)")
+    assert stats["literal_ok"]
+
+
+def test_fp8_gqa_write_sampled():
+    base = W.gqa_write()
+    seqs = sorted(np.random.default_rng(3).choice(base.num_seqs, 24, replace=False).tolist())
+    stats = _fp8_bench_case(base, seqs, "fp8 gqa_write (bench batch)")
+    assert stats["combined_ok"]
+
+
+def test_fp8_long_context_sampled():
+    base = W.long_context()
+    assert base.partition_size == 512
+    stats = _fp8_bench_case(base, [0, 2], "fp8 long_context (bench batch)")
+    assert stats["combined_ok"]

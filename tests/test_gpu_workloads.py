@@ -39,28 +39,37 @@ def _check_workload(batch, sample, check_pool=True):
     return compare(bits(db.out), ref, batch.dtype, batch.name)
 
 
+# fp16 workloads meet the 2e-3 / 1e-2 limits literally; bf16 ones the
+# combined per-element bound (a bf16 output cannot meet 2e-3 absolute in
+# [1, 2) after its own rounding).
+
 def test_tiny_every_output():
     b = W.tiny()
     stats = _check_workload(b, None)
     assert stats["n"] == 4 * 4 * 64
+    assert stats["literal_ok"], stats
 
 
 def test_llama7b_mha_sampled():
     b = W.llama7b_mha()
-    _check_workload(b, _sample(b.num_seqs, 8, 2))
+    stats = _check_workload(b, _sample(b.num_seqs, 8, 2))
+    assert stats["literal_ok"], stats
 
 
 def test_gqa_write_sampled():
     b = W.gqa_write()
-    _check_workload(b, _sample(b.num_seqs, 24, 3))
+    stats = _check_workload(b, _sample(b.num_seqs, 24, 3))
+    assert stats["combined_ok"], stats
 
 
 def test_prefix_share_sampled():
     b = W.prefix_share()
-    _check_workload(b, _sample(b.num_seqs, 12, 4))
+    stats = _check_workload(b, _sample(b.num_seqs, 12, 4))
+    assert stats["literal_ok"], stats
 
 
 def test_long_context_sampled():
     b = W.long_context()
     assert b.partition_size == 512
-    _check_workload(b, [1, 3], check_pool=False)
+    stats = _check_workload(b, [1, 3], check_pool=False)
+    assert stats["combined_ok"], stats

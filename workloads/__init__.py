@@ -465,11 +465,23 @@ class Fp8Batch:
         return getattr(self.base, name)
 
 
-def fp8_variant(batch: PagedBatch, seed: int, k_scale: float = 0.125, v_scale: float = 0.0625) -> Fp8Batch:
+def all_finite_e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """Random E4M3 codes uniform over all 254 finite codes (every exponent
+    field 0..15, subnormals and both zeros included; only the two NaN codes
+    0x7F and 0xFF are left out)."""
+    c = rng.integers(0, 254, size=shape, dtype=np.int32)
+    return (c + (c >= 0x7F)).astype(np.uint8)
+
+
+def fp8_variant(batch: PagedBatch, seed: int, k_scale: float = 0.125, v_scale: float = 0.0625,
+                full_range: bool = False) -> Fp8Batch:
     """Replace the pools of ``batch`` by 8-bit pools: every position a sequence
     attends to (except this step's new tokens, which the step writes) holds a
-    random code; every other slot holds the NaN code."""
+    random code; every other slot holds the NaN code.  Codes have exponent
+    fields 4..10 (``random_e4m3_codes``), or with ``full_range`` are uniform
+    over all 254 finite codes."""
     rng = np.random.default_rng(seed)
+    draw = all_finite_e4m3_codes if full_range else random_e4m3_codes
     N, Hkv, B, D = batch.k_cache.shape
     kc = np.full((N, Hkv, B, D), FP8_POISON, dtype=np.uint8)
     vc = np.full((N, Hkv, D, B), FP8_POISON, dtype=np.uint8)
@@ -477,8 +489,8 @@ def fp8_variant(batch: PagedBatch, seed: int, k_scale: float = 0.125, v_scale: f
         L = int(batch.context_lens[s])
         if L == 0:
             continue
-        kt = random_e4m3_codes(rng, (L, Hkv, D))
-        vt = random_e4m3_codes(rng, (L, Hkv, D))
+        kt = draw(rng, (L, Hkv, D))
+        vt = draw(rng, (L, Hkv, D))
         nb = _blocks_for(L, B)
         pad = nb * B - L
         kp = np.concatenate([kt, np.full((pad, Hkv, D), FP8_POISON, np.uint8)]).reshape(nb, B, Hkv, D)
