@@ -8,8 +8,6 @@
 // implicit device-wide synchronisation is unacceptable.  For them the scratch
 // lives in a fixed buffer compiled into this library, PKV_NOALLOC_SCRATCH_BYTES
 // per device; the caller still passes every input and output.
-#include <mutex>
-
 #include "pkv_host.h"
 
 // The scratch itself.  Every GPU that loads this library holds it until the
@@ -22,24 +20,17 @@ namespace pkv {
 namespace {
 
 constexpr size_t kScratchBytes = PKV_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 128;
-std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices];  // device address of the buffer, per device ordinal
 
-// Device address of the buffer on the current device, looked up once per device
-// (with that device current) and cached.
+// Device address of the buffer on the current device.  It is looked up on
+// every call rather than cached: the lookup is cheap next to a launch, and a
+// cached address would go stale if the device's context were destroyed and
+// created again (cudaDeviceReset), which loads the buffer anew.  The first
+// lookup on a device also loads the library's device code there.
 pkv_status scratch_address(void **addr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_DEVICE;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return PKV_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *addr = g_scratch_addr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return PKV_ERR_CUDA;
+  *addr = p;
   return PKV_OK;
 }
 
