@@ -70,7 +70,7 @@ typedef enum {
 #define PKV_DEV_BAD_BLOCK 0x1  /* a Block Table entry or copy pair outside [0, num_blocks) */
 #define PKV_DEV_BAD_SLOT 0x2   /* a slot >= num_blocks * block_size */
 #define PKV_DEV_BAD_LEN 0x4    /* context_len < 0, > max_context_len or > max_blocks_per_seq * block_size */
-#define PKV_DEV_TIMEOUT 0x8    /* a copy into shared memory did not complete within ~1 s */
+#define PKV_DEV_TIMEOUT 0x8    /* a copy into shared memory did not complete within its limit (~1 s) */
 
 typedef enum { PKV_F16 = 0, PKV_BF16 = 1, PKV_FP8_E4M3 = 2 } pkv_dtype;
 
@@ -242,9 +242,11 @@ PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_desc 
  *   - Limit: when pkv_paged_attention_workspace_size(...) for these sizes
  *     exceeds PKV_NOALLOC_SCRATCH_BYTES the call returns PKV_ERR_TOO_LARGE
  *     before anything is queued; use pkv_paged_attention_decode instead.
- *   - The first call on each device looks up the buffer's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *   - Every call looks up the buffer's device address on the current device
+ *     (cudaGetSymbolAddress), so the address stays right after the device's
+ *     context is reset.  The first call on each device also loads the
+ *     library's device code there; make that first call before any stream
+ *     capture.
  *   - All calls on a device share the one buffer and it keeps the last call's
  *     contents.  The call clears the part that must start at zero (the split
  *     arrival counters) and writes every partial before reading it, but two
@@ -331,7 +333,6 @@ PKV_API pkv_status pkv_paged_prefill(void *out, const void *query, const void *k
                                      int32_t num_q_heads, float scale, int32_t *d_status,
                                      pkv_stream_t stream);
 
-/* Static English text for a status code. */
 /*
  * pkv_paged_attention_decode_lse - decode attention over a part of each
  * sequence, returned as an attention state for a later merge.
@@ -375,6 +376,33 @@ PKV_API pkv_status pkv_merge_attention_states(void *out, pkv_dtype out_dtype, co
                                               int32_t num_rows, int32_t head_dim,
                                               pkv_stream_t stream);
 
+/*
+ * pkv_test_decode_withheld_load - fault injection for tests of the failure
+ * path; not for production use and with no counterpart on the pages.
+ *
+ * Every wait of the decode kernel for a copy into shared memory is bounded:
+ * past its limit the kernel raises PKV_DEV_TIMEOUT in *d_status, waits
+ * (again bounded) for its other copies in flight, finishes its work unit
+ * with what it has and exits, so the device stays usable.  This call runs
+ * pkv_paged_attention_decode with one load withheld - logical block
+ * withheld_block of sequence 0, kv head 0, never issued, so its barrier never
+ * completes - and with every wait limited to wait_limit_us microseconds
+ * (1 .. 1000000) instead of about one second.  Expected result: the call's
+ * kernels end, *d_status has PKV_DEV_TIMEOUT, the rows of sequence 0's kv
+ * head 0 are unspecified and every other row is the normal result.
+ * Arguments as pkv_paged_attention_decode; only fp16 pools with head_dim 128
+ * and block_size 16 and at most 8 query heads per kv head are accepted
+ * (PKV_ERR_BAD_SHAPE otherwise), and withheld_block must lie in the first
+ * partition (PKV_ERR_BAD_PARTITION otherwise).
+ */
+PKV_API pkv_status pkv_test_decode_withheld_load(
+    void *out, const void *query, const void *k_cache, const void *v_cache, pkv_cache_desc cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
+    int32_t partition_size, void *workspace, size_t workspace_bytes, int32_t withheld_block,
+    uint32_t wait_limit_us, int32_t *d_status, pkv_stream_t stream);
+
+/* Static English text for a status code. */
 PKV_API const char *pkv_status_string(pkv_status status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

@@ -23,6 +23,7 @@ STATUS_NAMES = {
     7: "PKV_ERR_TOO_LARGE", 8: "PKV_ERR_CUDA", 9: "PKV_ERR_DEVICE",
     10: "PKV_ERR_NO_BLOCKS", 11: "PKV_ERR_BAD_SEQUENCE",
 }
+ERR_TOO_LARGE = 7
 ERR_NO_BLOCKS = 10
 ERR_BAD_SEQUENCE = 11
 # device-side flags
@@ -81,6 +82,10 @@ SIGNATURES = {
     "pkv_paged_prefill": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc, _c_void_p, _i32,
                                          _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _f32, _c_void_p,
                                          _c_void_p]),
+    "pkv_test_decode_withheld_load": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc,
+                                                     _c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _f32, _i32,
+                                                     _c_void_p, _size_t, _i32, ctypes.c_uint32, _c_void_p,
+                                                     _c_void_p]),
     "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     # include/pkv_block_manager.h (host only)
     "pkv_bm_create": (ctypes.c_int, [_i32, _i32, _i32, ctypes.POINTER(_c_void_p)]),
@@ -307,6 +312,30 @@ def paged_prefill(out, query, k_cache, v_cache, block_tables, query_start, conte
     return out
 
 
+def test_decode_withheld_load(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                              withheld_block, wait_limit_us, partition_size=0, workspace=None, d_status=None,
+                              stream=None):
+    """Fault injection for tests: ``paged_attention_decode`` with the load of
+    logical block ``withheld_block`` of sequence 0, kv head 0 withheld and every
+    wait limited to ``wait_limit_us``; the kernel must end with the timeout bit
+    in ``d_status``."""
+    desc = cache_desc(k_cache)
+    _same_pool(k_cache, v_cache)
+    S, Hq, D = query.shape
+    if out.shape != query.shape or out.dtype != k_cache.dtype or query.dtype != k_cache.dtype:
+        raise ValueError("query/out must be [S, Hq, head_dim] in the cache dtype")
+    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = library().pkv_test_decode_withheld_load(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), S, Hq, int(max_context_len), float(scale), int(partition_size), _ptr(workspace),
+        ws_bytes, int(withheld_block), int(wait_limit_us), _ptr(d_status), _stream(stream, query.device))
+    _check(st, "pkv_test_decode_withheld_load")
+    return out
+
+
 # Capacity of the library's built-in split-K scratch (PKV_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
@@ -339,10 +368,11 @@ def paged_attention_decode_noalloc(out, query, k_cache, v_cache, block_tables, c
         _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
         int(partition_size), _ptr(d_status), _stream(stream, query.device))
-    if st == 7:
+    if st == ERR_TOO_LARGE:
         need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
-        raise PkvError(st, f"pkv_paged_attention_decode_noalloc: these sizes need {need} bytes of split-K "
-                           f"scratch, more than the built-in {NOALLOC_SCRATCH_BYTES}")
+        if need > NOALLOC_SCRATCH_BYTES:
+            raise PkvError(st, f"pkv_paged_attention_decode_noalloc: these sizes need {need} bytes of split-K "
+                               f"scratch, more than the built-in {NOALLOC_SCRATCH_BYTES}")
     _check(st, "pkv_paged_attention_decode_noalloc")
     return out
 

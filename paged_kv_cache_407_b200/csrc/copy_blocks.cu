@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(kCopyThreads)
     copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                        const int64_t *__restrict__ block_pairs, int64_t block_vecs,
                        int64_t num_blocks, int32_t *d_status) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t src = block_pairs[2 * static_cast<int64_t>(blockIdx.x)];
   const int64_t dst = block_pairs[2 * static_cast<int64_t>(blockIdx.x) + 1];
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -61,8 +63,9 @@ extern "C" pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_de
   const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyUnroll;
   const unsigned slices = static_cast<unsigned>(std::min<int64_t>((block_vecs + per_cta - 1) / per_cta, 64));
   dim3 grid(static_cast<unsigned>(num_pairs), 2u, slices);
-  copy_blocks_kernel<<<grid, kCopyThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_pairs, block_vecs,
-      cache.num_blocks, d_status);
-  return launch_status();
+  const cudaError_t err =
+      launch_pdl(copy_blocks_kernel, grid, dim3(kCopyThreads), 0, reinterpret_cast<cudaStream_t>(stream),
+                 static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_pairs, block_vecs,
+                 static_cast<int64_t>(cache.num_blocks), d_status);
+  return err == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }

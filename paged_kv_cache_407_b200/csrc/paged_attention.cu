@@ -66,6 +66,11 @@ struct DecodeArgs {
   float out_scale;   // 1, or v_scale for 8-bit pools
   const int2 *units;           // split calls: (sequence, partition) per unit, longest first
   const int32_t *unit_count;   // number of units in `units`
+  // Fault-injection instance only (FAULT = true): the load of logical block
+  // fault_block of sequence 0, kv head 0 is never issued, so its barrier
+  // never completes and the wait gives up after fault_wait_ns.
+  int fault_block;
+  uint64_t fault_wait_ns;
 };
 
 // ---------------------------------------------------------------------------
@@ -266,13 +271,19 @@ struct GridTune {
   static constexpr int kSmem = kNvOff + kWarps * kStages * 4 + 1024;
 };
 
-template <typename T, int D, int BS, int WARPS, int NST, bool BIG, bool KV8>
+// FAULT: the fault-injection instance behind pkv_test_decode_withheld_load,
+// which withholds one block's load (see DecodeArgs) to show that the bounded
+// waits end the kernel with PKV_DEV_TIMEOUT; every other instance has
+// FAULT = false and none of its code.
+template <typename T, int D, int BS, int WARPS, int NST, bool BIG, bool KV8, bool FAULT = false>
 __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMinBlocks))
     paged_decode_grid_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
   using TN = GridTune<D, BS, KV8 ? 1 : 2>;
   constexpr int kStageBytes = 2 * BS * D * (KV8 ? 1 : 2);
   using State = DecodeState<T, D, BS, BIG, KV8>;
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -344,7 +355,9 @@ __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMi
       const int st = k % NST;
       const uint32_t bar = bars + 8 * st;
       const int blk = b0 + warp + k * WARPS;
-      if (static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks)) {
+      if (FAULT && s == 0 && g == 0 && blk == a.fault_block) {
+        stage_nv[st] = 0;  // withheld: no load is issued and nothing arrives
+      } else if (static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks)) {
         stage_nv[st] = (blk == nb - 1) ? tail_nv : BS;
         fence_proxy_async_smem();
         if constexpr (KV8)
@@ -364,9 +377,10 @@ __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMi
   for (const int pro = cnt < NST ? cnt : NST; kp < pro; ++kp) issue(kp);
   int k = 0;
   bool ok = true;
+  const uint64_t wait_ns = FAULT ? a.fault_wait_ns : kWaitLimitNs;
   for (; k < cnt; ++k) {
     const int st = k % NST;
-    ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (k / NST) & 1));
+    ok = __all_sync(kFullMask, mbar_wait(bars + 8 * st, (k / NST) & 1, wait_ns));
     if (!ok) break;
     const uint32_t kb = ring + st * kStageBytes;
     st_.block(kb, kb + kStageBytes / 2, stage_nv[st], a.scale_log2, lane);
@@ -379,7 +393,7 @@ __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2>::kMi
   if (!ok) {
     if (lane == 0) raise_flag(a.d_status, PKV_DEV_TIMEOUT);
     // Let the copies still in flight land before the shared memory is reused.
-    for (int j = k; j < kp; ++j) (void)mbar_wait(bars + 8 * (j % NST), (j / NST) & 1);
+    for (int j = k; j < kp; ++j) (void)mbar_wait(bars + 8 * (j % NST), (j / NST) & 1, wait_ns);
   }
 
   st_.reduce_l();
@@ -437,6 +451,8 @@ __device__ __forceinline__ float block_reduce(float v, bool is_max, float *scrat
 
 template <typename T, int D>
 __global__ void __launch_bounds__(D) lse_combine_kernel(const CombineArgs c) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float scratch[D / 32];
   const int h = blockIdx.x;
   const int s = blockIdx.y;
@@ -489,6 +505,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(256)
     merge_states_kernel(void *out, const float *__restrict__ states, int64_t state_stride,
                         int num_states, int num_rows) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int VPL = D / 32;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -523,6 +541,10 @@ __global__ void __launch_bounds__(256)
 // one size is arbitrary and does not change any result, since partitions are
 // merged in partition order).  A sequence without tokens keeps one unit, which
 // writes its zero output.  One CTA; it also zeroes the arrival counters.
+// Every partition of a sequence but the last is full (part_blocks blocks), so
+// a thread takes whole sequences: one read of the length, one count for the
+// full partitions and one for the last; the counts of a warp are combined
+// before they reach the shared histogram.
 // ---------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanBuckets = 1024;  // unit sizes of 1023 blocks and more share the top bucket
@@ -537,26 +559,33 @@ __global__ void __launch_bounds__(kPlanThreads)
                        int part_blocks, int max_parts, int len_limit, int2 *__restrict__ units,
                        int32_t *__restrict__ unit_count, int32_t *__restrict__ counters,
                        int num_counters) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int hist[kPlanBuckets];
   __shared__ int warp_sums[kPlanThreads / 32];
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   hist[tid] = 0;
   for (int i = tid; i < num_counters; i += kPlanThreads) counters[i] = 0;
-  __syncthreads();
-  // candidate units (sequence, partition) in partition-major order, spread
-  // over the threads
-  const long long total = static_cast<long long>(num_seqs) * max_parts;
-  auto for_units = [&](auto &&fn) {
-    for (long long u = tid; u < total; u += kPlanThreads) {
-      const int p = static_cast<int>(u / num_seqs);
-      const int s = static_cast<int>(u - static_cast<long long>(p) * num_seqs);
-      const int nb = (plan_len(context_lens, s, len_limit) + block_size - 1) / block_size;
-      if (p >= parts_of(nb, part_blocks)) continue;
-      const int size = min(part_blocks, nb - p * part_blocks);
-      fn(s, p, min(max(size, 0), kPlanBuckets - 1));
-    }
+  const int full_key = min(part_blocks, kPlanBuckets - 1);
+  // a sequence's partitions: np - 1 full ones and a last one of `last` blocks
+  auto shape = [&](int s, int &np, int &last) {
+    const int nb = (plan_len(context_lens, s, len_limit) + block_size - 1) / block_size;
+    np = parts_of(nb, part_blocks);
+    last = min(max(nb - (np - 1) * part_blocks, 0), kPlanBuckets - 1);
   };
-  for_units([&](int, int, int key) { atomicAdd(&hist[key], 1); });
+  // sequences in rounds of kPlanThreads; the same rounds in both passes
+  const int rounds = (num_seqs + kPlanThreads - 1) / kPlanThreads;
+  __syncthreads();
+  for (int r = 0; r < rounds; ++r) {
+    const int s = r * kPlanThreads + tid;
+    int np = 0, last = 0;
+    if (s < num_seqs) shape(s, np, last);
+    const int nfull = s < num_seqs ? np - 1 : 0;
+    const int warp_full = __reduce_add_sync(0xffffffffu, nfull);
+    if (lane == 0 && warp_full > 0) atomicAdd(&hist[full_key], warp_full);
+    if (s < num_seqs) atomicAdd(&hist[last], 1);
+  }
   __syncthreads();
   // offsets in descending key order: offs[k] = sum of hist[k'] over k' > k
   const int key = kPlanBuckets - 1 - tid;  // thread tid scans bucket key
@@ -565,18 +594,45 @@ __global__ void __launch_bounds__(kPlanThreads)
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int t = __shfl_up_sync(0xffffffffu, incl, off);
-    if ((tid & 31) >= off) incl += t;
+    if (lane >= off) incl += t;
   }
-  if ((tid & 31) == 31) warp_sums[tid >> 5] = incl;
+  if (lane == 31) warp_sums[tid >> 5] = incl;
   __syncthreads();
-  int base = 0;
-  for (int w = 0; w < (tid >> 5); ++w) base += warp_sums[w];
-  const int excl = base + incl - v;
+  if (tid < 32) {  // exclusive scan of the 32 warp totals, in place
+    const int w = warp_sums[tid];
+    int x = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, x, off);
+      if (tid >= off) x += t;
+    }
+    warp_sums[tid] = x - w;
+    if (tid == 31) *unit_count = x;
+  }
   __syncthreads();
-  hist[key] = excl;  // now the next free position of each bucket
-  if (tid == kPlanThreads - 1) *unit_count = base + incl;
+  hist[key] = warp_sums[tid >> 5] + incl - v;  // now the next free position of each bucket
   __syncthreads();
-  for_units([&](int s, int p, int k) { units[atomicAdd(&hist[k], 1)] = make_int2(s, p); });
+  for (int r = 0; r < rounds; ++r) {
+    const int s = r * kPlanThreads + tid;
+    int np = 0, last = 0;
+    if (s < num_seqs) shape(s, np, last);
+    const int nfull = s < num_seqs ? np - 1 : 0;
+    // this thread's full partitions take consecutive places: the warp's
+    // running sum gives each thread its start within the warp's share
+    int before = nfull;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, before, off);
+      if (lane >= off) before += t;
+    }
+    const int warp_full = __shfl_sync(0xffffffffu, before, 31);
+    before -= nfull;
+    int base = 0;
+    if (lane == 0 && warp_full > 0) base = atomicAdd(&hist[full_key], warp_full);
+    base = __shfl_sync(0xffffffffu, base, 0) + before;
+    for (int p = 0; p < nfull; ++p) units[base + p] = make_int2(s, p);
+    if (s < num_seqs) units[atomicAdd(&hist[last], 1)] = make_int2(s, np - 1);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -642,20 +698,17 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int3
   return true;
 }
 
-template <typename T, int D, int BS, bool BIG, bool KV8>
+template <typename T, int D, int BS, bool BIG, bool KV8, bool FAULT = false>
 pkv_status launch_grid(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
                        cudaStream_t stream) {
   using TN = GridTune<D, BS, KV8 ? 1 : 2>;
-  auto kern = paged_decode_grid_kernel<T, D, BS, TN::kWarps, TN::kStages, BIG, KV8>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TN::kSmem) !=
-      cudaSuccess)
-    return PKV_ERR_CUDA;
+  auto kern = paged_decode_grid_kernel<T, D, BS, TN::kWarps, TN::kStages, BIG, KV8, FAULT>;
+  static std::atomic<uint64_t> smem_set{0};  // per device, this instance
   dim3 grid = args.units == nullptr
                   ? dim3(static_cast<unsigned>(args.num_kv_heads), static_cast<unsigned>(args.num_seqs),
                          static_cast<unsigned>(args.max_parts))
                   : dim3(static_cast<unsigned>(args.num_kv_heads) * args.num_seqs * args.max_parts);
-  kern<<<grid, TN::kWarps * 32, TN::kSmem, stream>>>(tmk, tmv, args);
-  return launch_status();
+  return launch_with_smem(kern, grid, dim3(TN::kWarps * 32), TN::kSmem, stream, &smem_set, tmk, tmv, args);
 }
 
 template <typename T, int D, int BS, bool BIG>
@@ -701,8 +754,8 @@ pkv_status launch_for_dim(int block_size, bool big, const CUtensorMap &tmk, cons
 template <typename T, int D>
 pkv_status launch_combine(const CombineArgs &c, int num_seqs, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(c.num_q_heads), static_cast<unsigned>(num_seqs));
-  lse_combine_kernel<T, D><<<grid, D, 0, stream>>>(c);
-  return launch_status();
+  return launch_pdl(lse_combine_kernel<T, D>, grid, dim3(D), 0, stream, c) == cudaSuccess ? PKV_OK
+                                                                                         : PKV_ERR_CUDA;
 }
 
 }  // namespace
@@ -735,13 +788,42 @@ namespace {
 // Shared body of the decode entry points.  kv8: 8-bit pools with scales
 // k_scale / v_scale; act: dtype of query (and of out unless lse is set, when
 // out is fp32 and lse receives each row's log-sum-exp).
+// The tensor maps of one pair of pools.
+struct MapCache {
+  bool valid = false;
+  bool kv8 = false;
+  const void *k = nullptr;
+  const void *v = nullptr;
+  pkv_cache_desc desc{};
+  CUtensorMap tmk, tmv;
+  bool matches(const void *k_, const void *v_, const pkv_cache_desc &d, bool kv8_) const {
+    return valid && k == k_ && v == v_ && kv8 == kv8_ && desc.num_blocks == d.num_blocks &&
+           desc.block_size == d.block_size && desc.num_kv_heads == d.num_kv_heads &&
+           desc.head_dim == d.head_dim && desc.dtype == d.dtype;
+  }
+  void set(const void *k_, const void *v_, const pkv_cache_desc &d, bool kv8_) {
+    k = k_;
+    v = v_;
+    desc = d;
+    kv8 = kv8_;
+    valid = true;
+  }
+};
+
+// Fault injection (pkv_test_decode_withheld_load only): which load to
+// withhold and how long a wait lasts.
+struct FaultSpec {
+  int block;
+  uint64_t wait_ns;
+};
+
 pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, const void *k_cache,
                        const void *v_cache, const pkv_cache_desc &cache, bool kv8,
                        const int32_t *block_tables, int32_t max_blocks_per_seq,
                        const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads,
                        int32_t max_context_len, float scale, float k_scale, float v_scale,
                        int32_t partition_size, void *workspace, size_t workspace_bytes,
-                       int32_t *d_status, pkv_stream_t stream) {
+                       int32_t *d_status, pkv_stream_t stream, const FaultSpec *fault = nullptr) {
   pkv_status st = check_cache_desc(cache);
   if (st != PKV_OK) return st;
   if (kv8 ? (cache.dtype != PKV_FP8_E4M3 || !is_16bit(act)) : !is_16bit(cache.dtype))
@@ -778,14 +860,23 @@ pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, 
   }
   if ((st = check_device()) != PKV_OK) return st;
 
-  CUtensorMap tmk, tmv;
-  if (kv8) {
-    if ((st = encode_fp8_k_map(&tmk, k_cache, cache)) != PKV_OK) return st;
-    if ((st = encode_fp8_v_map(&tmv, v_cache, cache)) != PKV_OK) return st;
-  } else {
-    if ((st = encode_cache_map(&tmk, k_cache, cache)) != PKV_OK) return st;
-    if ((st = encode_cache_map(&tmv, v_cache, cache)) != PKV_OK) return st;
+  // The two tensor maps depend only on the pools and their shape; a serving
+  // loop calls with the same pools every step, so the last pair encoded on
+  // this thread is kept and reused.
+  thread_local MapCache last;
+  if (!last.matches(k_cache, v_cache, cache, kv8)) {
+    last.valid = false;
+    if (kv8) {
+      if ((st = encode_fp8_k_map(&last.tmk, k_cache, cache)) != PKV_OK) return st;
+      if ((st = encode_fp8_v_map(&last.tmv, v_cache, cache)) != PKV_OK) return st;
+    } else {
+      if ((st = encode_cache_map(&last.tmk, k_cache, cache)) != PKV_OK) return st;
+      if ((st = encode_cache_map(&last.tmv, v_cache, cache)) != PKV_OK) return st;
+    }
+    last.set(k_cache, v_cache, cache, kv8);
   }
+  const CUtensorMap &tmk = last.tmk;
+  const CUtensorMap &tmv = last.tmv;
 
   DecodeArgs args{};
   args.query = query;
@@ -822,20 +913,26 @@ pkv_status decode_impl(void *out, float *lse, const void *query, pkv_dtype act, 
   args.max_parts = plan.max_parts;
   args.scale_log2 = scale * kLog2e * (kv8 ? k_scale : 1.f);
   args.out_scale = kv8 ? v_scale : 1.f;
+  args.fault_block = fault ? fault->block : -1;
+  args.fault_wait_ns = fault ? fault->wait_ns : kWaitLimitNs;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (split && !use_plan && cudaMemsetAsync(ws, 0, plan.ctrl_bytes, s) != cudaSuccess)
     return PKV_ERR_CUDA;
   if (use_plan) {  // the plan (which also zeroes the arrival counters)
-    decode_plan_kernel<<<1, kPlanThreads, 0, s>>>(
-        context_lens, num_seqs, cache.block_size, plan.part_blocks, plan.max_parts, args.len_limit,
-        reinterpret_cast<int2 *>(ws + plan.ctrl_bytes), const_cast<int32_t *>(args.unit_count),
-        args.counters, num_seqs * cache.num_kv_heads);
-    if ((st = launch_status()) != PKV_OK) return st;
+    if (launch_pdl(decode_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, context_lens, num_seqs,
+                   static_cast<int>(cache.block_size), plan.part_blocks, plan.max_parts, args.len_limit,
+                   reinterpret_cast<int2 *>(ws + plan.ctrl_bytes), const_cast<int32_t *>(args.unit_count),
+                   args.counters, num_seqs * cache.num_kv_heads) != cudaSuccess)
+      return PKV_ERR_CUDA;
   }
   const bool big = args.group > 8;
   const bool bf16 = act == PKV_BF16;
-  if (kv8)
+  if (fault != nullptr) {
+    // the one fault-injection instance: fp16 pools, head_dim 128, 16-token
+    // blocks, at most 8 query heads per kv head (checked by the caller)
+    st = launch_grid<__half, 128, 16, false, false, true>(tmk, tmv, args, s);
+  } else if (kv8)
     st = bf16 ? launch_decode_fp8<__nv_bfloat16>(cache.block_size, big, tmk, tmv, args, s)
               : launch_decode_fp8<__half>(cache.block_size, big, tmk, tmv, args, s);
   else if (cache.head_dim == 128)
@@ -923,18 +1020,40 @@ extern "C" pkv_status pkv_merge_attention_states(void *out, pkv_dtype out_dtype,
   pkv_status st = check_device();
   if (st != PKV_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const unsigned grid = static_cast<unsigned>((num_rows + 7) / 8);
+  const dim3 grid(static_cast<unsigned>((num_rows + 7) / 8));
   const bool bf16 = out_dtype == PKV_BF16;
-  if (head_dim == 128) {
-    if (bf16)
-      merge_states_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
-    else
-      merge_states_kernel<__half, 128><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
-  } else {
-    if (bf16)
-      merge_states_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
-    else
-      merge_states_kernel<__half, 64><<<grid, 256, 0, s>>>(out, states, state_stride, num_states, num_rows);
-  }
-  return launch_status();
+  cudaError_t err;
+  if (head_dim == 128)
+    err = bf16 ? launch_pdl(merge_states_kernel<__nv_bfloat16, 128>, grid, dim3(256), 0, s, out, states,
+                            state_stride, num_states, num_rows)
+               : launch_pdl(merge_states_kernel<__half, 128>, grid, dim3(256), 0, s, out, states, state_stride,
+                            num_states, num_rows);
+  else
+    err = bf16 ? launch_pdl(merge_states_kernel<__nv_bfloat16, 64>, grid, dim3(256), 0, s, out, states,
+                            state_stride, num_states, num_rows)
+               : launch_pdl(merge_states_kernel<__half, 64>, grid, dim3(256), 0, s, out, states, state_stride,
+                            num_states, num_rows);
+  return err == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+extern "C" pkv_status pkv_test_decode_withheld_load(
+    void *out, const void *query, const void *k_cache, const void *v_cache, pkv_cache_desc cache,
+    const int32_t *block_tables, int32_t max_blocks_per_seq, const int32_t *context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t max_context_len, float scale,
+    int32_t partition_size, void *workspace, size_t workspace_bytes, int32_t withheld_block,
+    uint32_t wait_limit_us, int32_t *d_status, pkv_stream_t stream) {
+  using namespace pkv;
+  if (cache.dtype != PKV_F16 || cache.head_dim != 128 || cache.block_size != 16 ||
+      cache.num_kv_heads < 1 || num_q_heads % cache.num_kv_heads != 0 ||
+      num_q_heads / cache.num_kv_heads > 8)
+    return PKV_ERR_BAD_SHAPE;
+  if (withheld_block < 0 || wait_limit_us < 1 || wait_limit_us > 1000000u) return PKV_ERR_BAD_SHAPE;
+  const int32_t part = pkv_paged_attention_partition_size(num_seqs, cache.num_kv_heads, 16,
+                                                          max_context_len, partition_size);
+  if (part < 0 || withheld_block >= part / 16) return PKV_ERR_BAD_PARTITION;
+  const FaultSpec fault{withheld_block, static_cast<uint64_t>(wait_limit_us) * 1000ull};
+  return decode_impl(out, nullptr, query, cache.dtype, k_cache, v_cache, cache, false,
+                     block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                     max_context_len, scale, 1.f, 1.f, partition_size, workspace, workspace_bytes,
+                     d_status, stream, &fault);
 }

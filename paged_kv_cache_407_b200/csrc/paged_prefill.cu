@@ -205,6 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 184);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 188);
 
+  pdl_trigger();
+  pdl_wait();  // before any global access and before taking tensor memory
   if (warp == 0) tc::tmem_alloc(holder, kTmemCols);
   if (tid == 0) {
 #pragma unroll
@@ -625,12 +627,9 @@ pkv_status launch_prefill_bs(int block_size, dim3 grid, const CUtensorMap &tq, c
                              const CUtensorMap &tv, const PrefillArgs &args, cudaStream_t stream) {
 #define PKV_PREFILL_CASE(BSV)                                                               \
   case BSV: {                                                                               \
-    auto kern = paged_prefill_kernel<T, BSV>;                                               \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,             \
-                             PrefillTune<T>::kSmem) != cudaSuccess)                         \
-      return PKV_ERR_CUDA;                                                                  \
-    kern<<<grid, kThreads, PrefillTune<T>::kSmem, stream>>>(tq, tk, tv, args);              \
-    return launch_status();                                                                 \
+    static std::atomic<uint64_t> smem_set{0};                                               \
+    return launch_with_smem(paged_prefill_kernel<T, BSV>, grid, dim3(kThreads),             \
+                            PrefillTune<T>::kSmem, stream, &smem_set, tq, tk, tv, args);    \
   }
   switch (block_size) {
     PKV_PREFILL_CASE(8)

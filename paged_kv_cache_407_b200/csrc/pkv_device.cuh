@@ -16,6 +16,16 @@ namespace pkv {
 // PKV_DEV_TIMEOUT and stops using the stage instead of spinning for ever.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 
+// Programmatic dependent launch.  Every kernel of the library is launched so
+// that it may start while the kernel before it in the stream is finishing;
+// it calls pdl_wait() before its first global memory access (read or write),
+// which returns once that kernel has completed and its writes are visible,
+// so stream order holds for memory exactly as without the overlap - only the
+// launch itself and the work before the wait are hidden.  pdl_trigger() lets
+// the next kernel in the stream be launched (it then waits likewise).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_flag(int32_t *d_status, int32_t bits) {
   if (d_status != nullptr) atomicOr(d_status, bits);
 }
@@ -70,15 +80,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false when
-// it has not completed after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// it has not completed after limit_ns (kWaitLimitNs unless a caller asks for
+// less).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -1,6 +1,7 @@
 // Host helpers: status strings, descriptor and device checks, tensor maps.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "pkv_host.h"
@@ -20,13 +21,38 @@ pkv_status check_cache_desc(const pkv_cache_desc &c) {
   return PKV_OK;
 }
 
+namespace {
+// Result of the compute-capability check per device ordinal (0 = not yet
+// asked, 1 = sm_100, 2 = another part); the answer cannot change while the
+// process runs.
+std::atomic<int8_t> g_device_kind[kMaxDevices];
+}  // namespace
+
 pkv_status check_device() {
-  int dev = 0, major = 0, minor = 0;
+  int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+  if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_DEVICE;
+  int8_t kind = g_device_kind[dev].load(std::memory_order_relaxed);
+  if (kind == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return PKV_ERR_CUDA;
+    kind = (major == 10 && minor == 0) ? 1 : 2;
+    g_device_kind[dev].store(kind, std::memory_order_relaxed);
+  }
+  return kind == 1 ? PKV_OK : PKV_ERR_DEVICE;
+}
+
+pkv_status set_smem_limit_once(const void *func, int bytes, std::atomic<uint64_t> *done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done->load(std::memory_order_acquire) & bit) != 0) return PKV_OK;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
     return PKV_ERR_CUDA;
-  return (major == 10 && minor == 0) ? PKV_OK : PKV_ERR_DEVICE;
+  if (bit != 0) done->fetch_or(bit, std::memory_order_release);
+  return PKV_OK;
 }
 
 namespace {

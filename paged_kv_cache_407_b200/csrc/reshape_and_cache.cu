@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(256)
                                  const int64_t *__restrict__ slot_mapping, int num_tokens,
                                  int num_kv_heads, int head_vecs, int block_size,
                                  int64_t num_slots, int32_t *d_status) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * head_vecs;
   const int64_t total = per_token * num_tokens;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -56,6 +58,8 @@ __global__ void __launch_bounds__(256)
                                   const int64_t *__restrict__ slot_mapping, int num_tokens,
                                   int num_kv_heads, int head_dim, int block_size,
                                   int64_t num_slots, int32_t *d_status) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * head_dim;
   const int64_t total = per_token * num_tokens;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -92,6 +96,8 @@ __global__ void __launch_bounds__(256)
                                  const int64_t *__restrict__ slot_mapping, int num_tokens,
                                  int num_kv_heads, int head_dim, int block_size, int64_t num_slots,
                                  float k_scale, float v_scale, int32_t *d_status) {
+  pdl_trigger();
+  pdl_wait();
   const int quads = head_dim / 4;
   const int64_t per_token = static_cast<int64_t>(num_kv_heads) * quads;
   const int64_t total = per_token * num_tokens;
@@ -180,12 +186,14 @@ extern "C" pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *val
   const bool vec = aligned(key, 8) && aligned(value, 8) && key_token_stride % 4 == 0 &&
                    value_token_stride % 4 == 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t err;
 #define PKV_FP8_WRITE(T, V)                                                                   \
-  reshape_and_cache_fp8_kernel<T, V><<<blocks, threads, 0, s>>>(                              \
-      static_cast<const T *>(key), static_cast<const T *>(value), key_token_stride,           \
-      value_token_stride, static_cast<uint8_t *>(k_cache), static_cast<uint8_t *>(v_cache),   \
-      slot_mapping, num_tokens, cache.num_kv_heads, cache.head_dim, cache.block_size,         \
-      num_slots, k_scale, v_scale, d_status)
+  err = launch_pdl(reshape_and_cache_fp8_kernel<T, V>, dim3(blocks), dim3(threads), 0, s,     \
+                   static_cast<const T *>(key), static_cast<const T *>(value),                \
+                   key_token_stride, value_token_stride, static_cast<uint8_t *>(k_cache),     \
+                   static_cast<uint8_t *>(v_cache), slot_mapping, num_tokens,                 \
+                   cache.num_kv_heads, cache.head_dim, cache.block_size, num_slots, k_scale,  \
+                   v_scale, d_status)
   if (input_dtype == PKV_BF16) {
     if (vec)
       PKV_FP8_WRITE(__nv_bfloat16, true);
@@ -198,7 +206,7 @@ extern "C" pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *val
       PKV_FP8_WRITE(__half, false);
   }
 #undef PKV_FP8_WRITE
-  return launch_status();
+  return err == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 extern "C" pkv_status pkv_reshape_and_cache(const void *key, const void *value,
@@ -227,23 +235,24 @@ extern "C" pkv_status pkv_reshape_and_cache(const void *key, const void *value,
                    value_token_stride % 8 == 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int threads = 256;
+  cudaError_t err;
   if (vec) {
     const int head_vecs = cache.head_dim / 8;
     const int64_t items = static_cast<int64_t>(num_tokens) * cache.num_kv_heads * head_vecs;
     const int blocks = static_cast<int>(std::min<int64_t>((items + threads - 1) / threads, 148 * 16));
-    reshape_and_cache_vec_kernel<<<blocks, threads, 0, s>>>(
-        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), key_token_stride / 8,
-        value_token_stride / 8, static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache),
-        slot_mapping, num_tokens, cache.num_kv_heads, head_vecs, cache.block_size, num_slots,
-        d_status);
+    err = launch_pdl(reshape_and_cache_vec_kernel, dim3(blocks), dim3(threads), 0, s,
+                     static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
+                     key_token_stride / 8, value_token_stride / 8, static_cast<uint4 *>(k_cache),
+                     static_cast<uint4 *>(v_cache), slot_mapping, num_tokens, cache.num_kv_heads,
+                     head_vecs, cache.block_size, num_slots, d_status);
   } else {
     const int64_t items = static_cast<int64_t>(num_tokens) * row;
     const int blocks = static_cast<int>(std::min<int64_t>((items + threads - 1) / threads, 148 * 16));
-    reshape_and_cache_elem_kernel<<<blocks, threads, 0, s>>>(
-        static_cast<const uint16_t *>(key), static_cast<const uint16_t *>(value), key_token_stride,
-        value_token_stride, static_cast<uint16_t *>(k_cache), static_cast<uint16_t *>(v_cache),
-        slot_mapping, num_tokens, cache.num_kv_heads, cache.head_dim, cache.block_size, num_slots,
-        d_status);
+    err = launch_pdl(reshape_and_cache_elem_kernel, dim3(blocks), dim3(threads), 0, s,
+                     static_cast<const uint16_t *>(key), static_cast<const uint16_t *>(value),
+                     key_token_stride, value_token_stride, static_cast<uint16_t *>(k_cache),
+                     static_cast<uint16_t *>(v_cache), slot_mapping, num_tokens, cache.num_kv_heads,
+                     cache.head_dim, cache.block_size, num_slots, d_status);
   }
-  return launch_status();
+  return err == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
