@@ -13,6 +13,12 @@ uniform on [128, 2048], pool = needed blocks + 10 %, shuffled).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--kv-dtype auto|e4m3]
 
+The same run also times a companion batch (default gqa_write, the GQA decode
++ cache-write batch) with the same step and protocol and reports it under
+"companion" with its own clocks and roofline.  Beside the back-to-back timed
+steps (inputs larger than L2), each batch's attention call is also timed
+--flush-reps times with L2 flushed before every call (median, p10, p90).
+
 Workloads prefill_llama7b and prefill_gqa_chunked time the chunked-prefill
 path instead (cache write of the chunks + tcgen05 prefill attention; metric
 TFLOP/s against the measured bf16 tensor peak).
@@ -67,6 +73,11 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    p.add_argument("--companion", default="gqa_write",
+                   help="second decode batch timed in the same run and reported under its own key "
+                        "(the other batch the ≥70%% HBM target names); 'none' to skip")
+    p.add_argument("--flush-reps", type=int, default=100,
+                   help="per-call timings with L2 flushed before each call (median, p10, p90)")
     return p.parse_args(argv)
 
 
@@ -243,31 +254,61 @@ def blas_threads():
         return 1
 
 
-def oracle_sample_rate(batch, seconds: float, f8=None):
+def host_cores() -> dict:
+    """Cores of the host: all it has, and those this process may run on."""
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count() or 1
+    return {"cpu_count": os.cpu_count() or 1, "usable": usable}
+
+
+def oracle_sample_rate(batch, seconds: float, f8=None, threads: int | None = None):
     """Time the oracle's decode over whole sequences of the batch (of its 8-bit
-    variant ``f8`` when given) until about ``seconds`` of CPU work; returns
-    (GB/s, description, cores, seconds)."""
+    variant ``f8`` when given) until about ``seconds`` of CPU work, with the
+    BLAS limited to ``threads`` threads when given; returns (GB/s,
+    description, threads used, seconds)."""
     import oracle as O
     from paged_kv_cache_407_b200 import accounting as A
 
-    order = np.random.default_rng(12345).permutation(batch.num_seqs)
-    done, t0 = [], time.perf_counter()
-    while len(done) < len(order) and time.perf_counter() - t0 < seconds:
-        s = int(order[len(done)])
-        if f8 is None:
-            O.decode_sequence(batch.q[s], batch.k_cache, batch.v_cache, batch.block_tables[s],
-                              int(batch.context_lens[s]), batch.block_size, batch.scale, batch.dtype)
-        else:
-            O.paged_attention_decode_fp8(batch.q, f8.k_cache, f8.v_cache, batch.block_tables, batch.context_lens,
-                                         batch.block_size, batch.scale, f8.k_scale, f8.v_scale, batch.dtype,
-                                         seqs=[s])
-        done.append(s)
-    dt = time.perf_counter() - t0
+    limit = None
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+
+        limit = threadpool_limits(limits=threads)
+    try:
+        used = blas_threads()
+        order = np.random.default_rng(12345).permutation(batch.num_seqs)
+        done, t0 = [], time.perf_counter()
+        while len(done) < len(order) and time.perf_counter() - t0 < seconds:
+            s = int(order[len(done)])
+            if f8 is None:
+                O.decode_sequence(batch.q[s], batch.k_cache, batch.v_cache, batch.block_tables[s],
+                                  int(batch.context_lens[s]), batch.block_size, batch.scale, batch.dtype)
+            else:
+                O.paged_attention_decode_fp8(batch.q, f8.k_cache, f8.v_cache, batch.block_tables,
+                                             batch.context_lens, batch.block_size, batch.scale, f8.k_scale,
+                                             f8.v_scale, batch.dtype, seqs=[s])
+            done.append(s)
+        dt = time.perf_counter() - t0
+    finally:
+        if limit is not None:
+            limit.unregister()
     b = A.decode_bytes(batch.context_lens[done], batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
                        batch.block_size, kv_elem_bytes=1 if f8 is not None else 2)["total"]
     desc = (f"oracle decode (fp64 NumPy) of {len(done)} of {batch.num_seqs} sequences of the "
             f"{batch.name} batch ({int(batch.context_lens[done].sum())} tokens), {dt:.1f} s")
-    return b / dt / 1e9, desc, blas_threads(), dt
+    return b / dt / 1e9, desc, used, dt
+
+
+def cpu_baseline_decode(batch, seconds: float, f8=None) -> dict:
+    """The oracle on every core the BLAS uses, then on one core; both on a
+    bounded sample of the batch (about ``seconds`` each)."""
+    rate, desc, used, _ = oracle_sample_rate(batch, seconds, f8=f8)
+    rate1, desc1, _, _ = oracle_sample_rate(batch, seconds, f8=f8, threads=1)
+    return {"value": round(rate, 4), "unit": "GB/s", "cores": used, "kind": "oracle", "sample": desc,
+            "blas_threads": used, **host_cores(),
+            "one_core": {"value": round(rate1, 4), "cores": 1, "sample": desc1}}
 
 
 def is_prefill(name: str) -> bool:
@@ -379,7 +420,8 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": workload_config(batch, args, 1),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": desc + "; each step a bounded sample of this workload"},
+                         "sample": desc + "; each step a bounded sample of this workload",
+                         "blas_threads": cores, **host_cores()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "decode_tokens_per_s": round(value * 1e9 / att["total"] * batch.num_seqs, 2),
     }
@@ -416,7 +458,8 @@ def run_reference_prefill(args):
         "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "config": prefill_config(b, 1),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": desc + "; each step a bounded sample of this workload"},
+                         "sample": desc + "; each step a bounded sample of this workload",
+                         "blas_threads": cores, **host_cores()},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -533,7 +576,8 @@ def run_prefill(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, desc, cores, _ = oracle_prefill_rate(b, args.cpu_seconds)
-        cpu = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+               "blas_threads": cores, **host_cores()}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -577,118 +621,203 @@ def run_prefill(args):
 
 
 # --------------------------------------------------------------------- ours
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
+L2_FLUSH_BYTES = 256 * 1024 * 1024  # twice the 126 MB L2
 
-    import paged_kv_cache_407_b200 as pkv
-    from paged_kv_cache_407_b200.build import build
-    from workloads.device import upload
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        from datetime import timedelta
+class DecodeRunner:
+    """One decode batch resident on the device, and the step the benchmark
+    times: copy-on-write pairs (if any), the cache write of the step's new
+    tokens, then decode attention (+ merge)."""
 
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if rank == 0:
-        build()
-    if world > 1:
-        dist.barrier()
-    pkv.library()
+    def __init__(self, batch, e4m3: bool, rank: int, dev, status, stream):
+        import torch
 
-    batch = build_workload(args.workload, rank)
-    e4m3 = args.kv_dtype == "e4m3"
-    f8 = None
-    if e4m3:
-        import workloads as W
-        from workloads.device import upload_fp8
+        import paged_kv_cache_407_b200 as pkv
+        from workloads.device import upload
 
-        f8 = W.fp8_variant(batch, 777 + rank)
-        db = upload_fp8(f8, dev)
-    else:
-        db = upload(batch, dev)
-    ws_bytes = pkv.workspace_size(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
-                                  batch.block_size, batch.max_context_len, batch.partition_size)
-    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    P = pkv.partition_size(batch.num_seqs, batch.num_kv_heads, batch.block_size, batch.max_context_len,
-                           batch.partition_size)
-    split = batch.max_context_len > P
-    nb_max = -(-batch.max_context_len // batch.block_size)
-    max_parts = -(-nb_max // (P // batch.block_size))
-    has_cow = batch.cow_pairs.shape[0] > 0
-    # cache write + attention kernel (+ merge kernel for splits of more than
-    # 32 partitions) (+ block copy)
-    launches_per_step = 2 + (1 if max_parts > 32 else 0) + (1 if has_cow else 0)
-
-    def step(q=db.q, out=db.out, key=db.key, value=db.value, slots=db.slot_mapping, tables=db.block_tables,
-             lens=db.context_lens, ev=None):
-        if has_cow:
-            pkv.copy_blocks(db.k_cache, db.v_cache, db.cow_pairs, d_status=status, stream=stream)
+        self.batch, self.e4m3, self.dev, self.status, self.stream = batch, e4m3, dev, status, stream
+        self.f8 = None
         if e4m3:
-            pkv.reshape_and_cache_fp8(key, value, db.k_cache, db.v_cache, slots, f8.k_scale, f8.v_scale,
-                                      d_status=status, stream=stream)
+            import workloads as W
+            from workloads.device import upload_fp8
+
+            self.f8 = W.fp8_variant(batch, 777 + rank)
+            self.db = upload_fp8(self.f8, dev)
         else:
-            pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=status, stream=stream)
-        if ev is not None:
-            ev[0].record(stream)
-        if e4m3:
-            pkv.paged_attention_decode_fp8(out, q, db.k_cache, db.v_cache, tables, lens, batch.max_context_len,
-                                           batch.scale, f8.k_scale, f8.v_scale,
-                                           partition_size=batch.partition_size, workspace=workspace,
-                                           d_status=status, stream=stream)
+            self.db = upload(batch, dev)
+        self.ws_bytes = pkv.workspace_size(batch.num_seqs, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                                           batch.block_size, batch.max_context_len, batch.partition_size)
+        self.workspace = torch.empty(max(self.ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.P = pkv.partition_size(batch.num_seqs, batch.num_kv_heads, batch.block_size, batch.max_context_len,
+                                    batch.partition_size)
+        self.split = batch.max_context_len > self.P
+        nb_max = -(-batch.max_context_len // batch.block_size)
+        self.max_parts = -(-nb_max // (self.P // batch.block_size))
+        self.has_cow = batch.cow_pairs.shape[0] > 0
+        # cache write + attention kernel (+ plan kernel for 3..32 partitions)
+        # (+ merge kernel for more than 32) (+ block copy)
+        self.launches_per_step = (2 + (1 if 3 <= self.max_parts <= 32 else 0) + (1 if self.max_parts > 32 else 0)
+                                  + (1 if self.has_cow else 0))
+
+    def attention(self, q=None, out=None, tables=None, lens=None):
+        import paged_kv_cache_407_b200 as pkv
+
+        db, b = self.db, self.batch
+        q = db.q if q is None else q
+        out = db.out if out is None else out
+        tables = db.block_tables if tables is None else tables
+        lens = db.context_lens if lens is None else lens
+        if self.e4m3:
+            pkv.paged_attention_decode_fp8(out, q, db.k_cache, db.v_cache, tables, lens, b.max_context_len,
+                                           b.scale, self.f8.k_scale, self.f8.v_scale,
+                                           partition_size=b.partition_size, workspace=self.workspace,
+                                           d_status=self.status, stream=self.stream)
         else:
-            pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, batch.max_context_len,
-                                       batch.scale, partition_size=batch.partition_size, workspace=workspace,
-                                       d_status=status, stream=stream)
+            pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, b.max_context_len,
+                                       b.scale, partition_size=b.partition_size, workspace=self.workspace,
+                                       d_status=self.status, stream=self.stream)
+
+    def step(self, q=None, out=None, key=None, value=None, slots=None, tables=None, lens=None, ev=None):
+        import paged_kv_cache_407_b200 as pkv
+
+        db = self.db
+        key = db.key if key is None else key
+        value = db.value if value is None else value
+        slots = db.slot_mapping if slots is None else slots
+        if self.has_cow:
+            pkv.copy_blocks(db.k_cache, db.v_cache, db.cow_pairs, d_status=self.status, stream=self.stream)
+        if self.e4m3:
+            pkv.reshape_and_cache_fp8(key, value, db.k_cache, db.v_cache, slots, self.f8.k_scale, self.f8.v_scale,
+                                      d_status=self.status, stream=self.stream)
+        else:
+            pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=self.status,
+                                  stream=self.stream)
         if ev is not None:
-            ev[1].record(stream)
+            ev[0].record(self.stream)
+        self.attention(q=q, out=out, tables=tables, lens=lens)
+        if ev is not None:
+            ev[1].record(self.stream)
 
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize(dev)
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+    def check_status(self, where):
+        if int(self.status.item()) != 0:
+            raise RuntimeError(f"device status {int(self.status.item())} {where}")
 
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:  # noqa: BLE001
-        pass
-    K = args.steps
-    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(uuid) as clocks:
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        wall0 = time.time()
-        t_start.record(stream)
-        for i in range(K):
-            step(ev=att_ev[i])
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-        clocks.mark(wall0, time.time())
-        if world > 1:
-            dist.barrier()
-    ms_total = t_start.elapsed_time(t_end)
-    att_ms = [a.elapsed_time(b) for a, b in att_ev]
-    clock = clocks.summary()
+    # ------------------------------------------------------------ timings
+    def timed_steps(self, K: int, warmup: int, world: int, uuid):
+        """K back-to-back steps (inputs larger than L2) bracketed by a barrier
+        and a synchronize; per-call attention events on the launching stream;
+        clocks sampled by nvidia-smi during the timed region."""
+        import torch
+        import torch.distributed as dist
 
-    # -------- end to end through the public API, host buffers -----------
-    # Every step copies its inputs from pinned host memory to the device and
-    # its output back.  As a serving loop would, the copies run on their own
-    # streams with double-buffered device tensors, so step i's upload and step
-    # i-1's read-back overlap step i-1's and step i's compute; every copy is
-    # inside the timed region.
-    e2e = None
-    if not args.no_e2e:
+        for _ in range(max(3, warmup)):
+            self.step()
+        torch.cuda.synchronize(self.dev)
+        self.check_status("during warm-up")
+        att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(uuid) as clocks:
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(self.dev)
+            wall0 = time.time()
+            t_start.record(self.stream)
+            for i in range(K):
+                self.step(ev=att_ev[i])
+            t_end.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            clocks.mark(wall0, time.time())
+            if world > 1:
+                dist.barrier()
+        self.check_status("in the timed region")
+        return t_start.elapsed_time(t_end), [a.elapsed_time(b) for a, b in att_ev], clocks.summary()
+
+    def flushed_calls(self, reps: int) -> dict:
+        """Per-call attention time with L2 flushed before every call (a write
+        of 256 MB between calls, outside the events): median, p10, p90."""
+        import torch
+
+        if reps <= 0:
+            return None
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=self.dev)
+        clean = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=self.dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps + 3):
+            # write 256 MB (evicts the inputs), then read another 256 MB so that
+            # the dirty lines are written back before the call, not during it
+            flush.fill_(i & 0xFF)
+            torch.amax(clean)
+            if i >= 3:
+                evs[i - 3][0].record(self.stream)
+            self.attention()
+            if i >= 3:
+                evs[i - 3][1].record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        self.check_status("in the L2-flushed calls")
+        ms = np.array([a.elapsed_time(b) for a, b in evs])
+        del flush, clean
+        return {"reps": reps, "l2_flushed": "256 MB written, then 256 MB read, before every call",
+                "median_ms": round(float(np.median(ms)), 5),
+                "p10_ms": round(float(np.percentile(ms, 10)), 5), "p90_ms": round(float(np.percentile(ms, 90)), 5),
+                "mean_ms": round(float(ms.mean()), 5)}
+
+    def host_submit_us(self, calls: int = 400) -> dict:
+        """Host time per decode call: the Python binding (argument checks,
+        marshalling, the C call) and the bare C-ABI call with arguments
+        marshalled once; CPU wall clock around the calls, no synchronisation
+        inside (the GPU drains them afterwards)."""
+        import ctypes
+
+        import torch
+
+        import paged_kv_cache_407_b200 as pkv
+        from paged_kv_cache_407_b200 import binding as bd
+
+        torch.cuda.synchronize(self.dev)
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            self.attention()
+        t_binding = (time.perf_counter() - t0) / calls * 1e6
+        torch.cuda.synchronize(self.dev)
+        db, b = self.db, self.batch
+        lib = pkv.library()
+        stream = ctypes.c_void_p(self.stream.cuda_stream)
+        ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        ws = ctypes.c_size_t(self.workspace.numel())
+        if self.e4m3:
+            desc = bd.fp8_cache_desc(db.k_cache, db.v_cache)
+            fn = lib.pkv_paged_attention_decode_fp8
+            argv = (ptr(db.out), ptr(db.q), bd._DTYPES[db.q.dtype], ptr(db.k_cache), ptr(db.v_cache), desc,
+                    ptr(db.block_tables), db.block_tables.shape[1], ptr(db.context_lens), b.num_seqs,
+                    b.num_q_heads, b.max_context_len, ctypes.c_float(b.scale), ctypes.c_float(self.f8.k_scale),
+                    ctypes.c_float(self.f8.v_scale), b.partition_size, ptr(self.workspace), ws, ptr(self.status),
+                    stream)
+        else:
+            desc = bd.cache_desc(db.k_cache)
+            fn = lib.pkv_paged_attention_decode
+            argv = (ptr(db.out), ptr(db.q), ptr(db.k_cache), ptr(db.v_cache), desc, ptr(db.block_tables),
+                    db.block_tables.shape[1], ptr(db.context_lens), b.num_seqs, b.num_q_heads, b.max_context_len,
+                    ctypes.c_float(b.scale), b.partition_size, ptr(self.workspace), ws, ptr(self.status), stream)
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            if fn(*argv) != 0:
+                raise RuntimeError("decode call failed while timing the host submit")
+        t_cabi = (time.perf_counter() - t0) / calls * 1e6
+        torch.cuda.synchronize(self.dev)
+        self.check_status("while timing the host submit")
+        return {"binding": round(t_binding, 2), "c_abi": round(t_cabi, 2), "calls": calls}
+
+    def e2e(self, K: int, warmup: int, world: int) -> dict:
+        """End to end through the public API from host buffers.  Every step
+        copies its inputs from pinned host memory to the device and its output
+        back.  As a serving loop would, the copies run on their own streams
+        with double-buffered device tensors, so step i's upload and step
+        i-1's read-back overlap step i-1's and step i's compute; every copy
+        is inside the timed region."""
+        import torch
+        import torch.distributed as dist
+
+        db, dev, stream = self.db, self.dev, self.stream
         names = ("q", "key", "value", "slots", "tables", "lens")
         srcs = (db.q, db.key, db.value, db.slot_mapping, db.block_tables, db.context_lens)
         h_in = {n: t.detach().cpu().pin_memory() for n, t in zip(names, srcs)}
@@ -711,15 +840,15 @@ def run_ours(args):
                 ev_in[b].record(up)
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_out[b])  # step i-2's output has been read back
-            step(q=d_in[b]["q"], out=d_out[b], key=d_in[b]["key"], value=d_in[b]["value"],
-                 slots=d_in[b]["slots"], tables=d_in[b]["tables"], lens=d_in[b]["lens"])
+            self.step(q=d_in[b]["q"], out=d_out[b], key=d_in[b]["key"], value=d_in[b]["value"],
+                      slots=d_in[b]["slots"], tables=d_in[b]["tables"], lens=d_in[b]["lens"])
             ev_done[b].record(stream)
             down.wait_event(ev_done[b])
             with torch.cuda.stream(down):
                 h_out[b].copy_(d_out[b], non_blocking=True)
                 ev_out[b].record(down)
 
-        for i in range(max(3, args.warmup)):
+        for i in range(max(3, warmup)):
             e2e_step(i)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -735,10 +864,80 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         if not torch.equal(h_out[(K - 1) % 2].view(torch.int16), db.out.view(torch.int16).cpu()):
             raise RuntimeError("end-to-end output differs from the device-resident run")
-        e2e = {"ms": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h}
+        self.check_status("in the end-to-end run")
+        # the same copies with no kernel between them: the host link's share
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        up.wait_event(c0)
+        down.wait_event(c0)
+        for i in range(K):
+            b = i % 2
+            with torch.cuda.stream(up):
+                for n in names:
+                    d_in[b][n].copy_(h_in[n], non_blocking=True)
+            with torch.cuda.stream(down):
+                h_out[b].copy_(d_out[b], non_blocking=True)
+        stream.wait_stream(up)
+        stream.wait_stream(down)
+        c1.record(stream)
+        torch.cuda.synchronize(dev)
+        return {"ms": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h, "copies_ms": c0.elapsed_time(c1)}
 
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+def decode_roofline(att_bytes_total: float, att_ms: float, e4m3: bool, workload: str) -> dict:
+    peak, peak_kind = measured_peak()
+    achieved = att_bytes_total / (att_ms * 1e-3) / 1e9
+    return {
+        "bound": "hbm",
+        "kernel": "paged_attention_decode (attention kernel + log-sum-exp merge, timed together)",
+        "achieved": round(achieved, 1),
+        "peak": peak,
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": profiled_traffic(workload, "e4m3" if e4m3 else "f16"),
+    }
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_407_b200 as pkv
+    from paged_kv_cache_407_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    pkv.library()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        pass
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    e4m3 = args.kv_dtype == "e4m3"
+    K = args.steps
+
+    batch = build_workload(args.workload, rank)
+    run = DecodeRunner(batch, e4m3, rank, dev, status, stream)
+    ms_total, att_ms, clock = run.timed_steps(K, args.warmup, world, uuid)
+    flushed = run.flushed_calls(args.flush_reps)
+    host_us = run.host_submit_us()
+    e2e = None if args.no_e2e else run.e2e(K, args.warmup, world)
 
     att_bytes, write_bytes, copy_bytes = step_bytes(batch, kv_bytes=1 if e4m3 else 2)
     att_ms_mean = float(np.mean(att_ms))
@@ -746,10 +945,36 @@ def run_ours(args):
         [ms_total, att_ms_mean, e2e["ms"] if e2e else 0.0], [att_bytes["total"], batch.num_seqs], dev)
     ms_step = ms_total / K
 
+    # the companion batch: same step, same protocol, its own clocks and roofline
+    companion = None
+    if args.companion not in ("none", "", args.workload):
+        cb = build_workload(args.companion, rank)
+        crun = DecodeRunner(cb, e4m3, rank, dev, status, stream)
+        c_total, c_att, c_clock = crun.timed_steps(K, args.warmup, world, uuid)
+        c_flushed = crun.flushed_calls(args.flush_reps)
+        c_att_bytes, c_write, _ = step_bytes(cb, kv_bytes=1 if e4m3 else 2)
+        (c_total, c_att_max), (c_bytes_all, c_seqs_all) = reduce_across_ranks(
+            [c_total, float(np.mean(c_att))], [c_att_bytes["total"], cb.num_seqs], dev)
+        c_step = c_total / K
+        companion = {
+            "workload": cb.name,
+            "value": round(c_bytes_all / (c_step * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(c_step, 5),
+            "decode_tokens_per_s": round(c_seqs_all / (c_step * 1e-3), 1),
+            "attention_ms_per_call": round(c_att_max, 5),
+            "bytes_per_step": {"attention": c_att_bytes["total"], "cache_write": c_write},
+            "config": workload_config(cb, args, world),
+            "split_k": {"partition_tokens": crun.P, "split": bool(crun.split), "workspace_bytes": crun.ws_bytes},
+            "roofline": decode_roofline(c_att_bytes["total"], c_att_max, e4m3, cb.name),
+            "per_call_l2_flushed": c_flushed,
+            "clocks": c_clock,
+            "gpu_launches": crun.launches_per_step * K,
+        }
+        del crun
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, cores, _ = oracle_sample_rate(batch, args.cpu_seconds, f8=f8)
-        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = cpu_baseline_decode(batch, args.cpu_seconds, f8=run.f8)
 
     if world > 1:
         dist.barrier()
@@ -757,15 +982,11 @@ def run_ours(args):
     if rank != 0:
         return 0
 
-    peak, peak_kind = measured_peak()
-    total_att_bytes = bytes_all  # every rank's own batch, summed
-    value = total_att_bytes / (ms_step * 1e-3) / 1e9
-    achieved = att_bytes["total"] / (att_ms_max * 1e-3) / 1e9
-    traffic = profiled_traffic(batch.name, "e4m3" if e4m3 else "f16")
+    value = bytes_all / (ms_step * 1e-3) / 1e9  # every rank's own batch, summed
     config = workload_config(batch, args, world)
     config["kv_cache_dtype"] = "e4m3 (8-bit pools, fp16 MMA operands)" if e4m3 else batch.dtype
     if e4m3:
-        config["pool_bytes"] = int(f8.k_cache.nbytes + f8.v_cache.nbytes)
+        config["pool_bytes"] = int(run.f8.k_cache.nbytes + run.f8.v_cache.nbytes)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -785,30 +1006,26 @@ def run_ours(args):
         "bytes_per_step": {"attention": att_bytes["total"], "attention_kv": att_bytes["kv"],
                            "cache_write": write_bytes, "block_copy": copy_bytes},
         "attention_ms_per_call": round(att_ms_max, 5),
+        "per_call_l2_flushed": flushed,
+        "host_submit_us_per_call": host_us,
         "kv_accounting": decode_accounting(batch, 1 if e4m3 else 2, ms_step),
-        "split_k": {"partition_tokens": P, "split": bool(split), "workspace_bytes": ws_bytes,
-                    "partials_bytes_moved": split_partials_bytes(batch, P)},
-        "roofline": {
-            "bound": "hbm",
-            "kernel": "paged_attention_decode (attention kernel + log-sum-exp merge, timed together)",
-            "achieved": round(achieved, 1),
-            "peak": peak,
-            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4),
-            "traffic": traffic,
-        },
+        "split_k": {"partition_tokens": run.P, "split": bool(run.split), "workspace_bytes": run.ws_bytes,
+                    "partials_bytes_moved": split_partials_bytes(batch, run.P)},
+        "roofline": decode_roofline(att_bytes["total"], att_ms_max, e4m3, batch.name),
         "clocks": clock,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": run.launches_per_step * K,
     }
     if e2e:
-        line["e2e"] = {"value": round(total_att_bytes / (e2e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
+        line["e2e"] = {"value": round(bytes_all / (e2e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": round(e2e_ms / K, 5),
+                       "copies_only_ms_per_step": round(e2e["copies_ms"] / K, 5),
                        "pipelining": "inputs uploaded and outputs read back on two copy streams, "
                                      "double-buffered, overlapping compute of neighbouring steps"}
     if cpu:
         line["cpu_baseline"] = cpu
+    if companion:
+        line["companion"] = companion
     print(json.dumps(line), flush=True)
     return 0
 
