@@ -656,8 +656,8 @@ class DecodeRunner:
         self.has_cow = batch.cow_pairs.shape[0] > 0
         # cache write + attention kernel (+ plan kernel for 3..32 partitions)
         # (+ merge kernel for more than 32) (+ block copy)
-        self.launches_per_step = (2 + (1 if 3 <= self.max_parts <= 32 else 0) + (1 if self.max_parts > 32 else 0)
-                                  + (1 if self.has_cow else 0))
+        self.attention_launches = 1 + (1 if 3 <= self.max_parts <= 32 else 0) + (1 if self.max_parts > 32 else 0)
+        self.launches_per_step = 1 + self.attention_launches + (1 if self.has_cow else 0)
 
     def attention(self, q=None, out=None, tables=None, lens=None):
         import paged_kv_cache_407_b200 as pkv
@@ -677,7 +677,7 @@ class DecodeRunner:
                                        b.scale, partition_size=b.partition_size, workspace=self.workspace,
                                        d_status=self.status, stream=self.stream)
 
-    def step(self, q=None, out=None, key=None, value=None, slots=None, tables=None, lens=None, ev=None):
+    def step(self, q=None, out=None, key=None, value=None, slots=None, tables=None, lens=None):
         import paged_kv_cache_407_b200 as pkv
 
         db = self.db
@@ -692,11 +692,7 @@ class DecodeRunner:
         else:
             pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=self.status,
                                   stream=self.stream)
-        if ev is not None:
-            ev[0].record(self.stream)
         self.attention(q=q, out=out, tables=tables, lens=lens)
-        if ev is not None:
-            ev[1].record(self.stream)
 
     def check_status(self, where):
         if int(self.status.item()) != 0:
@@ -704,9 +700,14 @@ class DecodeRunner:
 
     # ------------------------------------------------------------ timings
     def timed_steps(self, K: int, warmup: int, world: int, uuid):
-        """K back-to-back steps (inputs larger than L2) bracketed by a barrier
-        and a synchronize; per-call attention events on the launching stream;
-        clocks sampled by nvidia-smi during the timed region."""
+        """Two timed regions, each bracketed by a barrier and a synchronize,
+        with clocks sampled by nvidia-smi over both: K back-to-back steps
+        (inputs larger than L2), then K back-to-back attention calls alone.
+        Only the regions' ends carry CUDA events: an event recorded between
+        two kernels would stop the second from launching while the first
+        finishes (programmatic dependent launch), so per-call events would
+        time the launch gap too.  Returns (ms of the K steps, ms per
+        attention call, clocks)."""
         import torch
         import torch.distributed as dist
 
@@ -714,23 +715,30 @@ class DecodeRunner:
             self.step()
         torch.cuda.synchronize(self.dev)
         self.check_status("during warm-up")
-        att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_start, a_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(uuid) as clocks:
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize(self.dev)
             wall0 = time.time()
             t_start.record(self.stream)
-            for i in range(K):
-                self.step(ev=att_ev[i])
+            for _ in range(K):
+                self.step()
             t_end.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            if world > 1:
+                dist.barrier()
+            a_start.record(self.stream)
+            for _ in range(K):
+                self.attention()
+            a_end.record(self.stream)
             torch.cuda.synchronize(self.dev)
             clocks.mark(wall0, time.time())
             if world > 1:
                 dist.barrier()
-        self.check_status("in the timed region")
-        return t_start.elapsed_time(t_end), [a.elapsed_time(b) for a, b in att_ev], clocks.summary()
+        self.check_status("in the timed regions")
+        return t_start.elapsed_time(t_end), a_start.elapsed_time(a_end) / K, clocks.summary()
 
     def flushed_calls(self, reps: int) -> dict:
         """Per-call attention time with L2 flushed before every call (a write
@@ -889,7 +897,7 @@ def decode_roofline(att_bytes_total: float, att_ms: float, e4m3: bool, workload:
     achieved = att_bytes_total / (att_ms * 1e-3) / 1e9
     return {
         "bound": "hbm",
-        "kernel": "paged_attention_decode (attention kernel + log-sum-exp merge, timed together)",
+        "kernel": "paged_attention_decode (planning + attention + merge kernels of one call; calls back to back)",
         "achieved": round(achieved, 1),
         "peak": peak,
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
@@ -940,9 +948,8 @@ def run_ours(args):
     e2e = None if args.no_e2e else run.e2e(K, args.warmup, world)
 
     att_bytes, write_bytes, copy_bytes = step_bytes(batch, kv_bytes=1 if e4m3 else 2)
-    att_ms_mean = float(np.mean(att_ms))
     (ms_total, att_ms_max, e2e_ms), (bytes_all, seqs_all) = reduce_across_ranks(
-        [ms_total, att_ms_mean, e2e["ms"] if e2e else 0.0], [att_bytes["total"], batch.num_seqs], dev)
+        [ms_total, att_ms, e2e["ms"] if e2e else 0.0], [att_bytes["total"], batch.num_seqs], dev)
     ms_step = ms_total / K
 
     # the companion batch: same step, same protocol, its own clocks and roofline
@@ -954,7 +961,7 @@ def run_ours(args):
         c_flushed = crun.flushed_calls(args.flush_reps)
         c_att_bytes, c_write, _ = step_bytes(cb, kv_bytes=1 if e4m3 else 2)
         (c_total, c_att_max), (c_bytes_all, c_seqs_all) = reduce_across_ranks(
-            [c_total, float(np.mean(c_att))], [c_att_bytes["total"], cb.num_seqs], dev)
+            [c_total, c_att], [c_att_bytes["total"], cb.num_seqs], dev)
         c_step = c_total / K
         companion = {
             "workload": cb.name,
@@ -969,6 +976,7 @@ def run_ours(args):
             "per_call_l2_flushed": c_flushed,
             "clocks": c_clock,
             "gpu_launches": crun.launches_per_step * K,
+            "gpu_launches_attention_region": crun.attention_launches * K,
         }
         del crun
 
@@ -1014,6 +1022,7 @@ def run_ours(args):
         "roofline": decode_roofline(att_bytes["total"], att_ms_max, e4m3, batch.name),
         "clocks": clock,
         "gpu_launches": run.launches_per_step * K,
+        "gpu_launches_attention_region": run.attention_launches * K,
     }
     if e2e:
         line["e2e"] = {"value": round(bytes_all / (e2e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",

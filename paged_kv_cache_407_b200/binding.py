@@ -180,6 +180,18 @@ def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, d_status=None,
     _check(st, "pkv_reshape_and_cache")
 
 
+def _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, device):
+    """The caller's workspace and its size in bytes, or, when the caller gave
+    none and one is needed, a fresh torch allocation (the library itself
+    never allocates)."""
+    if workspace is not None:
+        return workspace, workspace.numel() * workspace.element_size()
+    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
+    if need == 0:
+        return None, 0
+    return torch.empty(need, dtype=torch.uint8, device=device), need
+
+
 def workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
                    partition_size=0) -> int:
     return int(library().pkv_paged_attention_workspace_size(
@@ -211,10 +223,7 @@ def paged_attention_decode(out, query, k_cache, v_cache, block_tables, context_l
         raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
     if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
         raise ValueError("context_lens must be a contiguous int32 [S] tensor")
-    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    workspace, ws_bytes = _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, query.device)
     st = library().pkv_paged_attention_decode(
         _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
@@ -243,10 +252,7 @@ def paged_attention_decode_lse(out, lse, query, k_cache, v_cache, block_tables, 
         raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
     if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
         raise ValueError("context_lens must be a contiguous int32 [S] tensor")
-    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    workspace, ws_bytes = _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, query.device)
     st = library().pkv_paged_attention_decode_lse(
         _ptr(out), _ptr(lse), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
@@ -324,10 +330,7 @@ def test_decode_withheld_load(out, query, k_cache, v_cache, block_tables, contex
     S, Hq, D = query.shape
     if out.shape != query.shape or out.dtype != k_cache.dtype or query.dtype != k_cache.dtype:
         raise ValueError("query/out must be [S, Hq, head_dim] in the cache dtype")
-    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    workspace, ws_bytes = _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, query.device)
     st = library().pkv_test_decode_withheld_load(
         _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables), block_tables.shape[1],
         _ptr(context_lens), S, Hq, int(max_context_len), float(scale), int(partition_size), _ptr(workspace),
@@ -428,10 +431,7 @@ def paged_attention_decode_fp8(out, query, k_cache, v_cache, block_tables, conte
         raise ValueError("block_tables must be a contiguous int32 [S, max_blocks_per_seq] tensor")
     if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
         raise ValueError("context_lens must be a contiguous int32 [S] tensor")
-    need = workspace_size(S, Hq, desc.num_kv_heads, D, desc.block_size, max_context_len, partition_size)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=query.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    workspace, ws_bytes = _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, query.device)
     st = library().pkv_paged_attention_decode_fp8(
         _ptr(out), _ptr(query), _DTYPES[query.dtype], _ptr(k_cache), _ptr(v_cache), desc,
         _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len),
