@@ -187,3 +187,25 @@ def test_fp8_calls_validate_on_the_host(lib):
     assert need > 0
     assert decode(P=256, maxlen=1024) == 5
     assert decode(P=256, maxlen=1024, ws=A, ws_bytes=need - 1) == 5
+
+
+def test_withheld_load_entry_validates_on_the_host(lib):
+    """The fault-injection entry point accepts only its one kernel instance
+    (fp16 pools, head_dim 128, 16-token blocks, up to 8 query heads per kv
+    head), a wait limit of 1 us .. 1 s and a withheld block inside the first
+    partition; each rule is checked before any device work."""
+    null = None
+    A = ctypes.c_void_p(0x10000)
+    fn = lib.pkv_test_decode_withheld_load
+
+    def call(desc=None, Hq=8, maxlen=300, P=512, block=3, wait_us=3000):
+        return fn(A, A, A, A, desc or _desc(N=64, B=16, H=2, D=128), A, 32, A, 4, Hq, maxlen,
+                  ctypes.c_float(0.1), P, null, 0, block, wait_us, null, null)
+
+    assert call(desc=_desc(N=64, B=16, H=2, D=128, dt=1)) == 3   # bf16 pools
+    assert call(desc=_desc(N=64, B=32, H=2, D=128)) == 3         # 32-token blocks
+    assert call(desc=_desc(N=64, B=16, H=2, D=64)) == 3          # head_dim 64
+    assert call(Hq=2 * 16) == 3                                  # 16 query heads per kv head
+    assert call(wait_us=0) == 3 and call(wait_us=2_000_000) == 3
+    assert call(block=-1) == 3
+    assert call(block=32) == 6                                   # past the first 512-token partition
