@@ -658,41 +658,47 @@ class DecodeRunner:
         # (+ merge kernel for more than 32) (+ block copy)
         self.attention_launches = 1 + (1 if 3 <= self.max_parts <= 32 else 0) + (1 if self.max_parts > 32 else 0)
         self.launches_per_step = 1 + self.attention_launches + (1 if self.has_cow else 0)
+        self._calls, self._att = self.prepare()
 
-    def attention(self, q=None, out=None, tables=None, lens=None):
+    def prepare(self, q=None, out=None, key=None, value=None, slots=None, tables=None, lens=None):
+        """The step's library calls on these buffers (default: the batch's
+        own), each prepared once through the public API: (calls of the whole
+        step, the attention call).  A serving loop that reuses its buffers
+        calls the library this way."""
         import paged_kv_cache_407_b200 as pkv
 
         db, b = self.db, self.batch
         q = db.q if q is None else q
         out = db.out if out is None else out
-        tables = db.block_tables if tables is None else tables
-        lens = db.context_lens if lens is None else lens
-        if self.e4m3:
-            pkv.paged_attention_decode_fp8(out, q, db.k_cache, db.v_cache, tables, lens, b.max_context_len,
-                                           b.scale, self.f8.k_scale, self.f8.v_scale,
-                                           partition_size=b.partition_size, workspace=self.workspace,
-                                           d_status=self.status, stream=self.stream)
-        else:
-            pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, b.max_context_len,
-                                       b.scale, partition_size=b.partition_size, workspace=self.workspace,
-                                       d_status=self.status, stream=self.stream)
-
-    def step(self, q=None, out=None, key=None, value=None, slots=None, tables=None, lens=None):
-        import paged_kv_cache_407_b200 as pkv
-
-        db = self.db
         key = db.key if key is None else key
         value = db.value if value is None else value
         slots = db.slot_mapping if slots is None else slots
+        tables = db.block_tables if tables is None else tables
+        lens = db.context_lens if lens is None else lens
+        kw = dict(d_status=self.status, stream=self.stream, prepare=True)
+        calls = []
         if self.has_cow:
-            pkv.copy_blocks(db.k_cache, db.v_cache, db.cow_pairs, d_status=self.status, stream=self.stream)
+            calls.append(pkv.copy_blocks(db.k_cache, db.v_cache, db.cow_pairs, **kw))
         if self.e4m3:
-            pkv.reshape_and_cache_fp8(key, value, db.k_cache, db.v_cache, slots, self.f8.k_scale, self.f8.v_scale,
-                                      d_status=self.status, stream=self.stream)
+            calls.append(pkv.reshape_and_cache_fp8(key, value, db.k_cache, db.v_cache, slots, self.f8.k_scale,
+                                                   self.f8.v_scale, **kw))
+            att = pkv.paged_attention_decode_fp8(out, q, db.k_cache, db.v_cache, tables, lens, b.max_context_len,
+                                                 b.scale, self.f8.k_scale, self.f8.v_scale,
+                                                 partition_size=b.partition_size, workspace=self.workspace, **kw)
         else:
-            pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, d_status=self.status,
-                                  stream=self.stream)
-        self.attention(q=q, out=out, tables=tables, lens=lens)
+            calls.append(pkv.reshape_and_cache(key, value, db.k_cache, db.v_cache, slots, **kw))
+            att = pkv.paged_attention_decode(out, q, db.k_cache, db.v_cache, tables, lens, b.max_context_len,
+                                             b.scale, partition_size=b.partition_size, workspace=self.workspace,
+                                             **kw)
+        calls.append(att)
+        return tuple(calls), att
+
+    def attention(self):
+        self._att()
+
+    def step(self):
+        for c in self._calls:
+            c()
 
     def check_status(self, where):
         if int(self.status.item()) != 0:
@@ -771,9 +777,10 @@ class DecodeRunner:
 
     def host_submit_us(self, calls: int = 400) -> dict:
         """Host time per decode call: the Python binding (argument checks,
-        marshalling, the C call) and the bare C-ABI call with arguments
-        marshalled once; CPU wall clock around the calls, no synchronisation
-        inside (the GPU drains them afterwards)."""
+        marshalling, the C call), the binding's prepared call (checks and
+        marshalling done once; what the timed steps use) and the bare C-ABI
+        call; CPU wall clock around the calls, no synchronisation inside (the
+        GPU drains them afterwards)."""
         import ctypes
 
         import torch
@@ -781,13 +788,27 @@ class DecodeRunner:
         import paged_kv_cache_407_b200 as pkv
         from paged_kv_cache_407_b200 import binding as bd
 
+        db, b = self.db, self.batch
         torch.cuda.synchronize(self.dev)
         t0 = time.perf_counter()
         for _ in range(calls):
-            self.attention()
+            if self.e4m3:
+                pkv.paged_attention_decode_fp8(db.out, db.q, db.k_cache, db.v_cache, db.block_tables,
+                                               db.context_lens, b.max_context_len, b.scale, self.f8.k_scale,
+                                               self.f8.v_scale, partition_size=b.partition_size,
+                                               workspace=self.workspace, d_status=self.status,
+                                               stream=self.stream)
+            else:
+                pkv.paged_attention_decode(db.out, db.q, db.k_cache, db.v_cache, db.block_tables, db.context_lens,
+                                           b.max_context_len, b.scale, partition_size=b.partition_size,
+                                           workspace=self.workspace, d_status=self.status, stream=self.stream)
         t_binding = (time.perf_counter() - t0) / calls * 1e6
         torch.cuda.synchronize(self.dev)
-        db, b = self.db, self.batch
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            self._att()
+        t_prepared = (time.perf_counter() - t0) / calls * 1e6
+        torch.cuda.synchronize(self.dev)
         lib = pkv.library()
         stream = ctypes.c_void_p(self.stream.cuda_stream)
         ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
@@ -813,7 +834,8 @@ class DecodeRunner:
         t_cabi = (time.perf_counter() - t0) / calls * 1e6
         torch.cuda.synchronize(self.dev)
         self.check_status("while timing the host submit")
-        return {"binding": round(t_binding, 2), "c_abi": round(t_cabi, 2), "calls": calls}
+        return {"binding": round(t_binding, 2), "binding_prepared": round(t_prepared, 2),
+                "c_abi": round(t_cabi, 2), "calls": calls}
 
     def e2e(self, K: int, warmup: int, world: int) -> dict:
         """End to end through the public API from host buffers.  Every step
@@ -839,6 +861,10 @@ class DecodeRunner:
         ev_done = [torch.cuda.Event() for _ in range(2)]
         ev_out = [torch.cuda.Event() for _ in range(2)]
 
+        steps = [self.prepare(q=d_in[b]["q"], out=d_out[b], key=d_in[b]["key"], value=d_in[b]["value"],
+                              slots=d_in[b]["slots"], tables=d_in[b]["tables"], lens=d_in[b]["lens"])[0]
+                 for b in range(2)]
+
         def e2e_step(i):
             b = i % 2
             up.wait_event(ev_done[b])  # step i-2 has consumed input buffer b
@@ -848,8 +874,8 @@ class DecodeRunner:
                 ev_in[b].record(up)
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_out[b])  # step i-2's output has been read back
-            self.step(q=d_in[b]["q"], out=d_out[b], key=d_in[b]["key"], value=d_in[b]["value"],
-                      slots=d_in[b]["slots"], tables=d_in[b]["tables"], lens=d_in[b]["lens"])
+            for c in steps[b]:
+                c()
             ev_done[b].record(stream)
             down.wait_event(ev_done[b])
             with torch.cuda.stream(down):

@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     DEV_TIMEOUT,
     LIB_PATH,
     PkvError,
+    PreparedCall,
     cache_desc,
     copy_blocks,
     fp8_cache_desc,

@@ -137,6 +137,33 @@ def _check(status: int, where: str) -> None:
         raise PkvError(status, where)
 
 
+class PreparedCall:
+    """One library call whose arguments were checked and marshalled once
+    (``prepare=True`` on the calls that accept it): calling it issues the C
+    call again with the same tensors, scalars and stream, and raises on a
+    non-zero status as the plain call does.  It keeps the tensors it refers
+    to alive.  For loops that repeat a call on fixed buffers, where the
+    per-call argument checks would cost more host time than the launch."""
+
+    __slots__ = ("_fn", "_argv", "_where", "_keep", "result")
+
+    def __init__(self, fn, argv, where, keep, result):
+        self._fn, self._argv, self._where, self._keep, self.result = fn, argv, where, keep, result
+
+    def __call__(self):
+        st = self._fn(*self._argv)
+        if st != OK:
+            raise PkvError(st, self._where)
+        return self.result
+
+
+def _invoke(fn, argv, where, prepare, keep=(), result=None):
+    if prepare:
+        return PreparedCall(fn, tuple(argv), where, keep, result)
+    _check(fn(*argv), where)
+    return result
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -162,7 +189,7 @@ def _same_pool(k_cache, v_cache):
         raise ValueError("k_cache and v_cache must have the same shape, dtype and layout")
 
 
-def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, d_status=None, stream=None):
+def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, d_status=None, stream=None, prepare=False):
     """Write new tokens ``key/value [T, Hkv, D]`` into the slots ``slot_mapping [T]`` (int64)."""
     desc = cache_desc(k_cache)
     _same_pool(k_cache, v_cache)
@@ -174,10 +201,10 @@ def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, d_status=None,
             raise ValueError("key/value heads and dims must be contiguous within a token")
     if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T or not slot_mapping.is_contiguous():
         raise ValueError("slot_mapping must be a contiguous int64 tensor with one entry per token")
-    st = library().pkv_reshape_and_cache(
-        _ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(k_cache), _ptr(v_cache), desc,
-        _ptr(slot_mapping), T, _ptr(d_status), _stream(stream, k_cache.device))
-    _check(st, "pkv_reshape_and_cache")
+    return _invoke(library().pkv_reshape_and_cache,
+                   (_ptr(key), _ptr(value), key.stride(0), value.stride(0), _ptr(k_cache), _ptr(v_cache), desc,
+                    _ptr(slot_mapping), T, _ptr(d_status), _stream(stream, k_cache.device)),
+                   "pkv_reshape_and_cache", prepare, (key, value, k_cache, v_cache, slot_mapping, d_status))
 
 
 def _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, device):
@@ -204,7 +231,7 @@ def partition_size(num_seqs, num_kv_heads, block_size, max_context_len, partitio
 
 
 def paged_attention_decode(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
-                           scale, partition_size=0, workspace=None, d_status=None, stream=None):
+                           scale, partition_size=0, workspace=None, d_status=None, stream=None, prepare=False):
     """Decode attention: ``out [S, Hq, D] = attention(query [S, Hq, D], paged K/V)``.
 
     ``workspace``: a device tensor of at least ``workspace_size(...)`` bytes;
@@ -224,12 +251,12 @@ def paged_attention_decode(out, query, k_cache, v_cache, block_tables, context_l
     if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
         raise ValueError("context_lens must be a contiguous int32 [S] tensor")
     workspace, ws_bytes = _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, query.device)
-    st = library().pkv_paged_attention_decode(
-        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
-        block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
-        int(partition_size), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device))
-    _check(st, "pkv_paged_attention_decode")
-    return out
+    return _invoke(library().pkv_paged_attention_decode,
+                   (_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
+                    block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len), float(scale),
+                    int(partition_size), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device)),
+                   "pkv_paged_attention_decode", prepare,
+                   (out, query, k_cache, v_cache, block_tables, context_lens, workspace, d_status), out)
 
 
 def paged_attention_decode_lse(out, lse, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
@@ -291,7 +318,7 @@ def merge_attention_states(out, states, stream=None):
 
 
 def paged_prefill(out, query, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len, scale,
-                  d_status=None, stream=None):
+                  d_status=None, stream=None, prepare=False):
     """Causal attention of chunks of new tokens over their sequences' paged
     K/V: ``query``/``out`` ``[T, Hq, 128]``; sequence s owns rows
     ``query_start[s] .. query_start[s+1]`` (its last tokens, already written
@@ -310,12 +337,12 @@ def paged_prefill(out, query, k_cache, v_cache, block_tables, query_start, conte
     for t, n in ((query_start, S + 1), (context_lens, S)):
         if t.dtype != torch.int32 or t.numel() != n or not t.is_contiguous():
             raise ValueError("query_start / context_lens must be contiguous int32 [S + 1] / [S] tensors")
-    st = library().pkv_paged_prefill(
-        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables), block_tables.shape[1],
-        _ptr(query_start), _ptr(context_lens), S, T, int(max_query_len), Hq, float(scale), _ptr(d_status),
-        _stream(stream, query.device))
-    _check(st, "pkv_paged_prefill")
-    return out
+    return _invoke(library().pkv_paged_prefill,
+                   (_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
+                    block_tables.shape[1], _ptr(query_start), _ptr(context_lens), S, T, int(max_query_len), Hq,
+                    float(scale), _ptr(d_status), _stream(stream, query.device)),
+                   "pkv_paged_prefill", prepare,
+                   (out, query, k_cache, v_cache, block_tables, query_start, context_lens, d_status), out)
 
 
 def test_decode_withheld_load(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
@@ -394,7 +421,7 @@ def fp8_cache_desc(k_cache: torch.Tensor, v_cache: torch.Tensor) -> CacheDesc:
 
 
 def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, d_status=None,
-                          stream=None):
+                          stream=None, prepare=False):
     """Quantising write of new tokens ``key/value [T, Hkv, D]`` (fp16/bf16) into
     8-bit pools: codes e4m3(x / scale)."""
     desc = fp8_cache_desc(k_cache, v_cache)
@@ -408,16 +435,16 @@ def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v
         raise ValueError("key and value must have the same dtype")
     if slot_mapping.dtype != torch.int64 or slot_mapping.numel() != T or not slot_mapping.is_contiguous():
         raise ValueError("slot_mapping must be a contiguous int64 tensor with one entry per token")
-    st = library().pkv_reshape_and_cache_fp8(
-        _ptr(key), _ptr(value), key.stride(0), value.stride(0), _DTYPES[key.dtype], _ptr(k_cache),
-        _ptr(v_cache), desc, _ptr(slot_mapping), T, float(k_scale), float(v_scale), _ptr(d_status),
-        _stream(stream, k_cache.device))
-    _check(st, "pkv_reshape_and_cache_fp8")
+    return _invoke(library().pkv_reshape_and_cache_fp8,
+                   (_ptr(key), _ptr(value), key.stride(0), value.stride(0), _DTYPES[key.dtype], _ptr(k_cache),
+                    _ptr(v_cache), desc, _ptr(slot_mapping), T, float(k_scale), float(v_scale), _ptr(d_status),
+                    _stream(stream, k_cache.device)),
+                   "pkv_reshape_and_cache_fp8", prepare, (key, value, k_cache, v_cache, slot_mapping, d_status))
 
 
 def paged_attention_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
                                scale, k_scale, v_scale, partition_size=0, workspace=None, d_status=None,
-                               stream=None):
+                               stream=None, prepare=False):
     """Decode attention over 8-bit pools (K, V read back as code * scale);
     query/out fp16 or bf16 ``[S, Hq, D]``."""
     desc = fp8_cache_desc(k_cache, v_cache)
@@ -432,16 +459,16 @@ def paged_attention_decode_fp8(out, query, k_cache, v_cache, block_tables, conte
     if context_lens.dtype != torch.int32 or context_lens.numel() != S or not context_lens.is_contiguous():
         raise ValueError("context_lens must be a contiguous int32 [S] tensor")
     workspace, ws_bytes = _workspace(workspace, S, Hq, desc, D, max_context_len, partition_size, query.device)
-    st = library().pkv_paged_attention_decode_fp8(
-        _ptr(out), _ptr(query), _DTYPES[query.dtype], _ptr(k_cache), _ptr(v_cache), desc,
-        _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len),
-        float(scale), float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
-        _ptr(d_status), _stream(stream, query.device))
-    _check(st, "pkv_paged_attention_decode_fp8")
-    return out
+    return _invoke(library().pkv_paged_attention_decode_fp8,
+                   (_ptr(out), _ptr(query), _DTYPES[query.dtype], _ptr(k_cache), _ptr(v_cache), desc,
+                    _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), S, Hq, int(max_context_len),
+                    float(scale), float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
+                    _ptr(d_status), _stream(stream, query.device)),
+                   "pkv_paged_attention_decode_fp8", prepare,
+                   (out, query, k_cache, v_cache, block_tables, context_lens, workspace, d_status), out)
 
 
-def copy_blocks(k_cache, v_cache, block_pairs, d_status=None, stream=None):
+def copy_blocks(k_cache, v_cache, block_pairs, d_status=None, stream=None, prepare=False):
     """Copy-on-write: block ``pairs[i, 1]`` of both pools becomes a copy of
     ``pairs[i, 0]`` (fp16/bf16 pools, or 8-bit pools)."""
     if k_cache.dtype in _FP8_DTYPES:
@@ -452,9 +479,10 @@ def copy_blocks(k_cache, v_cache, block_pairs, d_status=None, stream=None):
     if block_pairs.dtype != torch.int64 or block_pairs.dim() != 2 or block_pairs.shape[1] != 2 \
             or not block_pairs.is_contiguous():
         raise ValueError("block_pairs must be a contiguous int64 [num_pairs, 2] tensor")
-    st = library().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), desc, _ptr(block_pairs),
-                                   block_pairs.shape[0], _ptr(d_status), _stream(stream, k_cache.device))
-    _check(st, "pkv_copy_blocks")
+    return _invoke(library().pkv_copy_blocks,
+                   (_ptr(k_cache), _ptr(v_cache), desc, _ptr(block_pairs), block_pairs.shape[0], _ptr(d_status),
+                    _stream(stream, k_cache.device)),
+                   "pkv_copy_blocks", prepare, (k_cache, v_cache, block_pairs, d_status))
 
 
 def version() -> int:

@@ -270,3 +270,32 @@ def test_runs_on_a_side_stream():
     side.synchronize()
     kc, vc = oracle_caches(b)
     compare(bits(db.out), oracle_out(b, kc, vc), W.BF16, "side stream")
+
+
+def test_prepared_calls_match_plain_calls():
+    """A prepared call (arguments checked and marshalled once) reissued on
+    the same buffers gives the plain call's result bit for bit, and reflects
+    new contents of those buffers (here: a changed query)."""
+    b = W.small_case(88, num_seqs=7, num_q_heads=16, num_kv_heads=4, head_dim=128, block_size=16,
+                     dtype=W.BF16, max_len=1200, partition_size=256)
+    db = upload(b)
+    st = status_tensor()
+    write = pkv.reshape_and_cache(db.key, db.value, db.k_cache, db.v_cache, db.slot_mapping, d_status=st,
+                                  prepare=True)
+    out = torch.empty_like(db.q)
+    dec = pkv.paged_attention_decode(out, db.q, db.k_cache, db.v_cache, db.block_tables, db.context_lens,
+                                     b.max_context_len, b.scale, partition_size=256, d_status=st, prepare=True)
+    write()
+    assert dec() is out
+    ref = pkv.paged_attention_decode(torch.empty_like(db.q), db.q, db.k_cache, db.v_cache, db.block_tables,
+                                     db.context_lens, b.max_context_len, b.scale, partition_size=256)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    db.q.mul_(0.5)
+    dec()
+    ref2 = pkv.paged_attention_decode(torch.empty_like(db.q), db.q, db.k_cache, db.v_cache, db.block_tables,
+                                      db.context_lens, b.max_context_len, b.scale, partition_size=256)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
+    assert not torch.equal(ref.view(torch.int16), ref2.view(torch.int16))
