@@ -918,6 +918,27 @@ class DecodeRunner:
         return {"ms": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h, "copies_ms": c0.elapsed_time(c1)}
 
 
+def read_stream_gbs(dev, nbytes: int = 2 << 30, reps: int = 10) -> float:
+    """Context for the roofline: the rate of a plain read-only stream (a
+    torch max-reduction over a 2 GiB buffer, one read per byte), beside the
+    copy rate the roofline uses as its peak."""
+    import torch
+
+    buf = torch.zeros(nbytes // 4, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        torch.amax(buf)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record()
+    for _ in range(reps):
+        torch.amax(buf)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    del buf
+    return nbytes / (ms * 1e-3) / 1e9
+
+
 def decode_roofline(att_bytes_total: float, att_ms: float, e4m3: bool, workload: str) -> dict:
     peak, peak_kind = measured_peak()
     achieved = att_bytes_total / (att_ms * 1e-3) / 1e9
@@ -971,6 +992,7 @@ def run_ours(args):
     ms_total, att_ms, clock = run.timed_steps(K, args.warmup, world, uuid)
     flushed = run.flushed_calls(args.flush_reps)
     host_us = run.host_submit_us()
+    read_gbs = read_stream_gbs(dev)
     e2e = None if args.no_e2e else run.e2e(K, args.warmup, world)
 
     att_bytes, write_bytes, copy_bytes = step_bytes(batch, kv_bytes=1 if e4m3 else 2)
@@ -1042,6 +1064,7 @@ def run_ours(args):
         "attention_ms_per_call": round(att_ms_max, 5),
         "per_call_l2_flushed": flushed,
         "host_submit_us_per_call": host_us,
+        "context_read_stream_gbs": round(read_gbs, 1),
         "kv_accounting": decode_accounting(batch, 1 if e4m3 else 2, ms_step),
         "split_k": {"partition_tokens": run.P, "split": bool(run.split), "workspace_bytes": run.ws_bytes,
                     "partials_bytes_moved": split_partials_bytes(batch, run.P)},
