@@ -70,6 +70,18 @@ constexpr uint32_t kTmemCols = 512;          // S buffers [0, 256), O of half 0 
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
 
+// One 32-bit word from global to shared memory, asynchronously (no register
+// is written, so nothing waits on it until cp_async_wait).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Until at most N of this thread's most recent groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // max(a, b, c) in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -87,7 +99,9 @@ template <typename T>
 struct PrefillTune {
   static constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
   static constexpr uint32_t kBarOff = kXOff + 2u * kRows * 8u;
-  static constexpr uint32_t kSmem = kBarOff + 192u + 1024u;
+  // block-id rings of the two load warps: [warp][3 tiles][16 entries]
+  static constexpr uint32_t kTabOff = kBarOff + 192u;
+  static constexpr uint32_t kSmem = kTabOff + 2u * 3u * 16u * 4u + 1024u;
 };
 
 struct PrefillArgs {
@@ -276,49 +290,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const int32_t *trow = a.block_tables + static_cast<size_t>(it.s) * a.max_blocks_per_seq;
-      auto ids_of = [&](int j) -> int {
-        const int lb = j * kBlocksPerTile + lane;
-        return (j < it.ntiles && lane < kBlocksPerTile && lb < it.nb) ? __ldg(trow + lb) : -1;
+      // The block ids of tile t reach slot t % 3 of this warp's ring by
+      // cp.async two tiles before use, so the Block Table's latency stays
+      // off this loop.  Lane b < kBlocksPerTile owns entry b of every slot:
+      // it copies that entry in and reads it back itself, so no other
+      // lane's copy needs ordering.
+      int32_t *ring = reinterpret_cast<int32_t *>(smem + TN::kTabOff) + (is_k ? 0 : 3 * 16);
+      auto fetch = [&](int t) {
+        const int lb = t * kBlocksPerTile + lane;
+        if (t < it.ntiles && lane < kBlocksPerTile && lb < it.nb)
+          cp_async_4(smem_addr(ring + (t % 3) * 16 + lane), trow + lb);
+        cp_async_commit();  // a group per tile, empty or not
       };
-      int ids = ids_of(0);
+      fetch(0);
+      fetch(1);
       for (int j = 0; j < it.ntiles; ++j, ++jt) {
         const int st = jt & 1;
-        const int next = ids_of(j + 1);  // in flight while this tile is issued
+        fetch(j + 2);  // slot (j + 2) % 3 was read back at tile j - 1
         if (jt >= 2 && !(run = wait(empty + 8 * st, ((jt - 2) >> 1) & 1))) break;
-        uint32_t bytes = 0;
-        int idv[kBlocksPerTile];
-#pragma unroll
-        for (int bi = 0; bi < kBlocksPerTile; ++bi) {
-          idv[bi] = __shfl_sync(kFullMask, ids, bi);
-          const int lb = j * kBlocksPerTile + bi;
-          if (lb < it.nb) {
-            if (static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
-              bytes += 2u * 64u * BS * 2u;
-            else if (lane == 0)
-              raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
-          }
-        }
+        cp_async_wait<2>();  // this lane's entry of tile j is in
+        const bool in_tile = lane < kBlocksPerTile && j * kBlocksPerTile + lane < it.nb;
+        const int id = in_tile ? ring[(j % 3) * 16 + lane] : -1;
+        const bool ok = in_tile && static_cast<unsigned>(id) < static_cast<unsigned>(a.num_blocks);
+        if (in_tile && !ok) raise_flag(a.d_status, PKV_DEV_BAD_BLOCK);
+        // one vote instead of a shuffle per block: this warp shares its
+        // sub-partition's MIO queue with two softmax warps' exponentials, and
+        // every shuffle waits its turn there
+        const uint32_t bytes = static_cast<uint32_t>(__popc(__ballot_sync(kFullMask, ok))) * (256u * BS);
+        const uint32_t bar = full + 8 * st;
         if (lane == 0) {
-          const uint32_t bar = full + 8 * st;
-          const uint32_t dst = stage0 + st * kTile;
           fence_proxy_async_smem();
-          if (bytes == 0) {
-            mbar_arrive(bar);
-          } else {
-            mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-            for (int bi = 0; bi < kBlocksPerTile; ++bi) {
-              const int lb = j * kBlocksPerTile + bi;
-              if (lb < it.nb && static_cast<unsigned>(idv[bi]) < static_cast<unsigned>(a.num_blocks))
-                tma_load_5d(dst + bi * (BS / 8) * kGroupBytes, map, bar, 0, 0, 0, 0,
-                            idv[bi] * a.num_kv_heads + it.g, policy);
-            }
-          }
+          if (bytes == 0) mbar_arrive(bar);
+          else mbar_arrive_expect_tx(bar, bytes);
         }
-        ids = next;
+        __syncwarp();
+        // lane b issues block b's box: one TMA instruction for the tile
+        // instead of kBlocksPerTile issued one after another
+        if (ok)
+          tma_load_5d(stage0 + st * kTile + lane * (BS / 8) * kGroupBytes, map, bar, 0, 0, 0, 0,
+                      id * a.num_kv_heads + it.g, policy);
       }
       ++n;
     }
+    cp_async_wait<0>();  // no copy into the ring outlives the loop
   } else if (warp == kMmaWarp || warp == kPvWarp) {
     // --------------------------------------------------------- MMA issuers
     // Two issuing warps feed the one tensor pipe, so that neither kind of
