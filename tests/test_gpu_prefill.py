@@ -165,6 +165,18 @@ def test_long_chunks_sampled_rows_and_repeat_calls_bit_identical():
     compare(bits(outs[0])[rows], ref, W.BF16, "long chunks, sampled rows")
 
 
+def test_one_long_context_short_chunk():
+    """A 64-token chunk at the end of a 40000-token context (313 K/V tiles, the
+    last one ragged) and a second sequence of 3 tokens: the load warps' block-id
+    ring, the stage counters and every barrier phase wrap hundreds of times
+    inside one item.  Every output element against the oracle."""
+    b = W.prefill_batch(83, dtype=W.BF16, num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+                        context_lens=[40000, 3], chunk_lens=[64, 3])
+    out, st = _run(b)
+    assert st == 0
+    compare(bits(out), _oracle(b), W.BF16, "prefill 40000-token context, 64-token chunk")
+
+
 @pytest.mark.parametrize("name", sorted(W.PREFILL_WORKLOADS))
 def test_bench_prefill_workloads_sampled_rows(name):
     """The bench's prefill batches at full size, in the launch the bench times:
