@@ -50,6 +50,8 @@ METRIC = "paged decode attention KV GB/s and tokens/s on 1 B200; % of HBM roofli
 PREFILL_METRIC = "paged prefill attention TFLOP/s (causal, algorithmic FLOPs) on 1 B200; % of tensor roofline"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0       # HBM3e, 8 TB/s per GPU (the figure the roofline is also quoted against)
+NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 / fp16 tensor rate per GPU
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["paged_kv_cache_407_b200/csrc/pkv_host.cu",
                   "paged_kv_cache_407_b200/csrc/paged_attention.cu",
@@ -606,6 +608,8 @@ def run_prefill(args):
                             if peak_kind == "measured" else "fallback"),
             "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
             "traffic": profiled_traffic(b.name, kernel="paged_prefill_kernel"),
+            "nominal": NOMINAL_BF16_TFLOPS,
+            "frac_of_nominal": round(achieved / NOMINAL_BF16_TFLOPS, 4),
         },
         "clocks": clock,
         "gpu_launches": 2 * K,
@@ -951,6 +955,8 @@ def decode_roofline(att_bytes_total: float, att_ms: float, e4m3: bool, workload:
         "unit": "GB/s",
         "frac": round(achieved / peak, 4),
         "traffic": profiled_traffic(workload, "e4m3" if e4m3 else "f16"),
+        "nominal": NOMINAL_HBM_GBS,
+        "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
     }
 
 
