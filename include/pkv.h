@@ -26,8 +26,19 @@
  *     not NULL (an int32 in device memory, to be read after the stream
  *     synchronises; the library never clears it).  Kernels never trap: an
  *     offending element is skipped or masked and the flag is raised.
- *   - The library keeps no mutable global state apart from a once-only lookup
- *     of the driver's tensor-map encoder; calls are thread-safe.
+ *   - Mutable global state is limited to caches filled on first use (the
+ *     driver's tensor-map encoder; per device, its compute capability and each
+ *     kernel's shared-memory limit; per host thread, recently encoded tensor
+ *     maps) and the built-in scratch of pkv_paged_attention_decode_noalloc.
+ *     The caches are atomic or per thread, so calls are thread-safe.
+ *   - Calls can be captured in a CUDA graph (stream capture): they allocate
+ *     nothing, never synchronise and queue only kernels (launched with
+ *     programmatic dependent launch) plus at most one cudaMemsetAsync.  Make
+ *     one call of each entry point per device before capturing, so that the
+ *     first-use set-up above happens outside the capture.  A captured call
+ *     keeps the pointers, sizes and max_context_len it was captured with; the
+ *     contents of the device arrays (inputs, lengths, tables, slots) may
+ *     change between replays.
  *
  * Cache layout ("HND"): k_cache and v_cache are separate pools, each
  *   [num_blocks][num_kv_heads][block_size][head_dim] row-major, element type
