@@ -19,8 +19,8 @@ The same run also times a companion batch (default gqa_write, the GQA decode
 steps (inputs larger than L2), each batch's attention call is also timed
 --flush-reps times with L2 flushed before every call (median, p10, p90).
 
-Workloads prefill_llama7b and prefill_gqa_chunked time the chunked-prefill
-path instead (cache write of the chunks + tcgen05 prefill attention; metric
+Workloads prefill_llama7b, prefill_gqa_chunked and prefill_mixed time the
+chunked-prefill path instead (cache write of the chunks + tcgen05 prefill attention; metric
 TFLOP/s against the measured bf16 tensor peak).
 
 Under torchrun every rank runs its own batch (weak scaling, seed + rank);
@@ -322,7 +322,7 @@ def is_prefill(name: str) -> bool:
 def build_prefill(name: str, rank: int):
     import workloads as W
 
-    base = {"prefill_llama7b": 6, "prefill_gqa_chunked": 7}[name]
+    base = {"prefill_llama7b": 6, "prefill_gqa_chunked": 7, "prefill_mixed": 11}[name]
     return W.PREFILL_WORKLOADS[name](seed=base + 1000 * rank)
 
 
@@ -498,6 +498,8 @@ def run_prefill(args):
     db = upload_prefill(b, dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    from paged_kv_cache_407_b200 import binding as bd
+    prefill_ws = torch.empty(bd.PREFILL_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)  # the item counter
 
     def step(q=db.q, out=db.out, key=db.key, value=db.value, slots=db.slot_mapping, tables=db.block_tables,
              qs=db.query_start, lens=db.context_lens, ev=None):
@@ -505,7 +507,7 @@ def run_prefill(args):
         if ev is not None:
             ev[0].record(stream)
         pkv.paged_prefill(out, q, db.k_cache, db.v_cache, tables, qs, lens, b.max_query_len, b.scale,
-                          d_status=status, stream=stream)
+                          d_status=status, stream=stream, workspace=prefill_ws)
         if ev is not None:
             ev[1].record(stream)
 

@@ -68,7 +68,8 @@ typedef enum {
   PKV_ERR_BAD_DTYPE = 2,      /* dtype is not PKV_F16 / PKV_BF16 */
   PKV_ERR_BAD_SHAPE = 3,      /* unsupported head_dim / block_size / head counts / negative size */
   PKV_ERR_MISALIGNED = 4,     /* a pointer or stride breaks the stated alignment */
-  PKV_ERR_WORKSPACE = 5,      /* workspace NULL or smaller than pkv_paged_attention_workspace_size */
+  PKV_ERR_WORKSPACE = 5,      /* workspace NULL or smaller than pkv_paged_attention_workspace_size
+                                 (pkv_paged_prefill: smaller than PKV_PREFILL_WORKSPACE_BYTES) */
   PKV_ERR_BAD_PARTITION = 6,  /* partition_size not a positive multiple of block_size */
   PKV_ERR_TOO_LARGE = 7,      /* a size exceeds what the kernels index (see each call) */
   PKV_ERR_CUDA = 8,           /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
@@ -331,6 +332,15 @@ PKV_API pkv_status pkv_paged_attention_decode_fp8(
  * head_dim 128; num_q_heads / num_kv_heads in {1, 2, 4, 8, 16}.
  * Runs on tcgen05 tensor cores: 128-row query tiles x 128-token K/V tiles,
  * fp32 accumulation in tensor memory; a persistent grid of one CTA per SM.
+ * workspace  : NULL, or at least PKV_PREFILL_WORKSPACE_BYTES of 4-byte-aligned
+ *              device memory owned by the caller (PKV_ERR_WORKSPACE if
+ *              smaller).  Given one, the call zeroes an item counter in it
+ *              (cudaMemsetAsync on `stream`) and the CTAs take the work items
+ *              (query tile, kv head, sequence) in order from it, each as it
+ *              frees up, which keeps them evenly loaded when the chunks'
+ *              lengths differ; two calls in flight at once need two
+ *              workspaces.  NULL: a fixed assignment of items to CTAs.  The
+ *              outputs are the same either way, bit for bit.
  * Device-detected errors: a sequence whose lengths break the rules above is
  * skipped with PKV_DEV_BAD_LEN; a block id outside the pool raises
  * PKV_DEV_BAD_BLOCK (that block's tokens are garbage); a wait past ~1 s
@@ -341,8 +351,11 @@ PKV_API pkv_status pkv_paged_prefill(void *out, const void *query, const void *k
                                      const int32_t *block_tables, int32_t max_blocks_per_seq,
                                      const int32_t *query_start, const int32_t *context_lens,
                                      int32_t num_seqs, int32_t num_tokens, int32_t max_query_len,
-                                     int32_t num_q_heads, float scale, int32_t *d_status,
-                                     pkv_stream_t stream);
+                                     int32_t num_q_heads, float scale, void *workspace,
+                                     size_t workspace_bytes, int32_t *d_status, pkv_stream_t stream);
+
+/* Workspace of pkv_paged_prefill (its item counter, with room to spare). */
+#define PKV_PREFILL_WORKSPACE_BYTES 16
 
 /*
  * pkv_paged_attention_decode_lse - decode attention over a part of each

@@ -10,6 +10,7 @@ from .binding import (  # noqa: F401
     DEV_BAD_SLOT,
     DEV_TIMEOUT,
     LIB_PATH,
+    PREFILL_WORKSPACE_BYTES,
     PkvError,
     PreparedCall,
     cache_desc,

@@ -81,7 +81,7 @@ SIGNATURES = {
                                                   _c_void_p]),
     "pkv_paged_prefill": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc, _c_void_p, _i32,
                                          _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _f32, _c_void_p,
-                                         _c_void_p]),
+                                         ctypes.c_size_t, _c_void_p, _c_void_p]),
     "pkv_test_decode_withheld_load": (ctypes.c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, CacheDesc,
                                                      _c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _f32, _i32,
                                                      _c_void_p, _size_t, _i32, ctypes.c_uint32, _c_void_p,
@@ -318,11 +318,16 @@ def merge_attention_states(out, states, stream=None):
 
 
 def paged_prefill(out, query, k_cache, v_cache, block_tables, query_start, context_lens, max_query_len, scale,
-                  d_status=None, stream=None, prepare=False):
+                  d_status=None, stream=None, prepare=False, dynamic=True, workspace=None):
     """Causal attention of chunks of new tokens over their sequences' paged
     K/V: ``query``/``out`` ``[T, Hq, 128]``; sequence s owns rows
     ``query_start[s] .. query_start[s+1]`` (its last tokens, already written
-    to the cache); ``context_lens`` counts them."""
+    to the cache); ``context_lens`` counts them.
+
+    ``dynamic``: the CTAs take the work items from a counter in ``workspace``
+    (a device tensor of at least PREFILL_WORKSPACE_BYTES; allocated with
+    torch when None), which keeps them evenly loaded when the chunks differ
+    in length; False: a fixed assignment (no workspace).  Same outputs."""
     desc = cache_desc(k_cache)
     _same_pool(k_cache, v_cache)
     T, Hq, D = query.shape
@@ -337,12 +342,17 @@ def paged_prefill(out, query, k_cache, v_cache, block_tables, query_start, conte
     for t, n in ((query_start, S + 1), (context_lens, S)):
         if t.dtype != torch.int32 or t.numel() != n or not t.is_contiguous():
             raise ValueError("query_start / context_lens must be contiguous int32 [S + 1] / [S] tensors")
+    if dynamic and workspace is None:
+        workspace = torch.empty(PREFILL_WORKSPACE_BYTES, dtype=torch.uint8, device=query.device)
+    if not dynamic:
+        workspace = None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     return _invoke(library().pkv_paged_prefill,
                    (_ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), desc, _ptr(block_tables),
                     block_tables.shape[1], _ptr(query_start), _ptr(context_lens), S, T, int(max_query_len), Hq,
-                    float(scale), _ptr(d_status), _stream(stream, query.device)),
+                    float(scale), _ptr(workspace), ws_bytes, _ptr(d_status), _stream(stream, query.device)),
                    "pkv_paged_prefill", prepare,
-                   (out, query, k_cache, v_cache, block_tables, query_start, context_lens, d_status), out)
+                   (out, query, k_cache, v_cache, block_tables, query_start, context_lens, d_status, workspace), out)
 
 
 def test_decode_withheld_load(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
@@ -365,6 +375,9 @@ def test_decode_withheld_load(out, query, k_cache, v_cache, block_tables, contex
     _check(st, "pkv_test_decode_withheld_load")
     return out
 
+
+# Workspace of pkv_paged_prefill's dynamic item order (PKV_PREFILL_WORKSPACE_BYTES).
+PREFILL_WORKSPACE_BYTES = 16
 
 # Capacity of the library's built-in split-K scratch (PKV_NOALLOC_SCRATCH_BYTES).
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024

@@ -100,7 +100,7 @@ struct PrefillTune {
   static constexpr bool kSplit = std::is_same<T, __nv_bfloat16>::value;
   static constexpr uint32_t kBarOff = kXOff + 2u * kRows * 8u;
   // block-id rings of the two load warps: [warp][3 tiles][16 entries]
-  static constexpr uint32_t kTabOff = kBarOff + 192u;
+  static constexpr uint32_t kTabOff = kBarOff + 320u;
   static constexpr uint32_t kSmem = kTabOff + 2u * 3u * 16u * 4u + 1024u;
 };
 
@@ -120,6 +120,10 @@ struct PrefillArgs {
   int qtiles;      // query tiles of the longest chunk
   int items;       // qtiles * num_kv_heads * num_seqs work items
   float scale_log2;
+  // Non-null: CTAs take items in index order from this counter (zeroed
+  // before the launch), each as it frees up.  Null: the static order of
+  // item_index.
+  unsigned int *ticket;
 };
 
 // One work item: a 128-row query tile of one (sequence, kv head).  Items are
@@ -218,6 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t holder = bars + 184;
   volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 184);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 188);
+  // The CTA's item sequence: the K-load warp takes each item (from the
+  // ticket counter, or the static order) and publishes its index in slot
+  // k % 4 of a ring; every other role reads it there, so all walk the same
+  // items.  [4] index published (1 arrival) / read by every other role.
+  const uint32_t bar_item = bars + 192;
+  const uint32_t bar_itemfree = bars + 224;
+  constexpr int kItemReaders = 3 + kSoftmaxWarps;  // V-load, S-issue, P V-issue and softmax warps
+  volatile int *item_ring = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 256);
 
   pdl_trigger();
   pdl_wait();  // before any global access and before taking tensor memory
@@ -239,6 +251,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_end, 1);
     mbar_init(bar_x, kSoftmaxWarps);
     mbar_init(bar_done, 2);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(bar_item + 8 * i, 1);
+      mbar_init(bar_itemfree + 8 * i, kItemReaders);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -254,6 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (mbar_wait(bar, parity)) return true;
     *abort_flag = 1;
     return false;
+  };
+  // The k-th item of this CTA as the roles other than the K-load warp see
+  // it: false if a wait ran out; i = -1 past the last item.
+  auto read_item = [&](int k, int &i) -> bool {
+    const int slot = k & 3;
+    if (!wait(bar_item + 8 * slot, (k >> 2) & 1)) return false;
+    i = item_ring[slot];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_itemfree + 8 * slot);
+    return true;
   };
 
   if (warp == kLoadKWarp || warp == kLoadVWarp) {
@@ -272,7 +299,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0;   // items so far
     int jt = 0;  // K/V tiles so far
     for (int k = 0; run; ++k) {
-      const int i = item_index(a, k);
+      int i;
+      if (is_k) {
+        // take the CTA's k-th item and publish it to the other roles, once
+        // they have all read the index the slot held four items back
+        const int slot = k & 3;
+        if (k >= 4 && !(run = wait(bar_itemfree + 8 * slot, ((k - 4) >> 2) & 1))) break;
+        int idx = 0;
+        if (lane == 0) {
+          idx = a.ticket != nullptr ? static_cast<int>(min(atomicAdd(a.ticket, 1u), 0x7fffffffu))
+                                    : item_index(a, k);
+          if (idx >= a.items) idx = -1;
+          item_ring[slot] = idx;
+          mbar_arrive(bar_item + 8 * slot);
+        }
+        i = __shfl_sync(kFullMask, idx, 0);
+      } else if (!(run = read_item(k, i))) {
+        break;
+      }
       if (i < 0) break;
       Item it;
       if (!item_at<BS>(a, i, it, false)) continue;
@@ -346,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0;
     int jt = 0;
     for (int k = 0; run; ++k) {
-      const int i = item_index(a, k);
+      int i;
+      if (!(run = read_item(k, i))) break;
       if (i < 0) break;
       Item it;
       if (!item_at<BS>(a, i, it, false)) continue;
@@ -420,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0;
     int jt = 0;
     for (int k = 0; run; ++k) {
-      const int i = item_index(a, k);
+      int i;
+      if (!(run = read_item(k, i))) break;
       if (i < 0) break;
       Item it;
       if (!item_at<BS>(a, i, it, tid == 0)) continue;
@@ -664,6 +710,7 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
                                         const int32_t *query_start, const int32_t *context_lens,
                                         int32_t num_seqs, int32_t num_tokens,
                                         int32_t max_query_len, int32_t num_q_heads, float scale,
+                                        void *workspace, size_t workspace_bytes,
                                         int32_t *d_status, pkv_stream_t stream) {
   using namespace pkv;
   pkv_status st = check_cache_desc(cache);
@@ -682,8 +729,10 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
   if (!out || !query || !k_cache || !v_cache || !block_tables || !query_start || !context_lens)
     return PKV_ERR_NULL_POINTER;
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(query, 16) || !aligned(out, 16) ||
-      !aligned(block_tables, 4) || !aligned(query_start, 4) || !aligned(context_lens, 4))
+      !aligned(block_tables, 4) || !aligned(query_start, 4) || !aligned(context_lens, 4) ||
+      !aligned(workspace, 4))
     return PKV_ERR_MISALIGNED;
+  if (workspace != nullptr && workspace_bytes < PKV_PREFILL_WORKSPACE_BYTES) return PKV_ERR_WORKSPACE;
   const long long qtiles = (static_cast<long long>(max_query_len) * G + kRows - 1) / kRows;
   const long long items = qtiles * cache.num_kv_heads * num_seqs;
   if (items > 2147483647ll) return PKV_ERR_TOO_LARGE;
@@ -718,6 +767,11 @@ extern "C" pkv_status pkv_paged_prefill(void *out, const void *query, const void
     return PKV_ERR_CUDA;
   dim3 grid(static_cast<unsigned>(items < sms ? items : sms));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (workspace != nullptr) {
+    // the item counter starts at zero for this launch
+    if (cudaMemsetAsync(workspace, 0, sizeof(unsigned int), s) != cudaSuccess) return PKV_ERR_CUDA;
+    args.ticket = static_cast<unsigned int *>(workspace);
+  }
   return cache.dtype == PKV_BF16 ? launch_prefill_bs<__nv_bfloat16>(cache.block_size, grid, tq, tk, tv, args, s)
                                  : launch_prefill_bs<__half>(cache.block_size, grid, tq, tk, tv, args, s);
 }

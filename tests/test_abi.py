@@ -114,9 +114,9 @@ def test_prefill_host_validation_without_device(lib):
     pre = lib.pkv_paged_prefill
 
     def call(desc=None, out=A, q=A, k=A, v=A, tables=A, qs=A, lens=A, S=2, T=64, maxq=32, Hq=8,
-             scale=0.125):
+             scale=0.125, ws=null, ws_bytes=0):
         return pre(out, q, k, v, desc or _desc(N=64, B=16, H=4, D=128), tables, 8, qs, lens, S, T, maxq, Hq,
-                   ctypes.c_float(scale), null, null)
+                   ctypes.c_float(scale), ws, ws_bytes, null, null)
 
     assert call(desc=_desc(D=64)) == 3                 # head_dim must be 128
     assert call(desc=_desc(D=128, dt=2)) == 2          # 8-bit pools: not for prefill
@@ -128,6 +128,8 @@ def test_prefill_host_validation_without_device(lib):
     assert call(S=0) == 0 and call(T=0) == 0 and call(maxq=0) == 0  # nothing to do
     assert call(q=null) == 1 and call(lens=null) == 1 and call(qs=null) == 1
     assert call(k=odd) == 4 and call(out=odd) == 4     # pools and rows must be 16-byte aligned
+    assert call(ws=ctypes.c_void_p(0x10002), ws_bytes=16) == 4   # workspace: 4-byte aligned
+    assert call(ws=A, ws_bytes=bd.PREFILL_WORKSPACE_BYTES - 1) == 5  # workspace too small
     # query tiles x kv heads x sequences beyond 2^31 - 1
     assert call(S=40, maxq=2**31 - 1, Hq=4) == 7
 

@@ -165,6 +165,46 @@ def test_long_chunks_sampled_rows_and_repeat_calls_bit_identical():
     compare(bits(outs[0])[rows], ref, W.BF16, "long chunks, sampled rows")
 
 
+def test_dynamic_and_static_item_orders_agree_bitwise():
+    """The work items (query tile, kv head, sequence) taken from the item
+    counter in the workspace, or in the fixed order without one: each item
+    is computed whole by one CTA either way, so the outputs must agree bit
+    for bit, on a batch whose chunks differ in length; and they match the
+    oracle on sampled rows.  Two calls with the same workspace reuse its
+    counter."""
+    b = W.prefill_mixed()
+    db = upload_prefill(b)
+    st = status_tensor()
+    pkv.reshape_and_cache(db.key, db.value, db.k_cache, db.v_cache, db.slot_mapping, d_status=st)
+    ws = torch.full((pkv.PREFILL_WORKSPACE_BYTES,), 0xAB, dtype=torch.uint8, device="cuda")  # not zero: the call zeroes it
+    outs = []
+    for dynamic in (False, True, True):
+        out = torch.full_like(db.q, float("nan"))
+        pkv.paged_prefill(out, db.q, db.k_cache, db.v_cache, db.block_tables, db.query_start, db.context_lens,
+                          b.max_query_len, b.scale, d_status=st, dynamic=dynamic, workspace=ws if dynamic else None)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    assert torch.equal(outs[1].view(torch.int16), outs[2].view(torch.int16))
+    kc, vc = O.reshape_and_cache(b.k_cache, b.v_cache, b.key, b.value, b.slot_mapping, b.block_size)
+    qs = np.asarray(b.query_start)
+    rows = np.arange(0, b.num_tokens, 211)
+    Hq, Hkv = b.q.shape[1], kc.shape[1]
+    ref = np.zeros((len(rows),) + b.q.shape[1:])
+    for i, t in enumerate(rows):
+        s = int(np.searchsorted(qs, t, side="right") - 1)
+        L, C = int(b.context_lens[s]), int(qs[s + 1] - qs[s])
+        K = O.decode_bits(O.materialize(kc, b.block_tables[s], L, b.block_size), b.dtype)
+        V = O.decode_bits(O.materialize(vc, b.block_tables[s], L, b.block_size), b.dtype)
+        p = L - C + (t - qs[s])
+        q = O.decode_bits(b.q[t], b.dtype)
+        for g in range(Hkv):
+            hs = [h for h in range(Hq) if O.kv_head_of(h, Hq, Hkv) == g]
+            ref[i, hs] = O.attend(q[hs], K[g, : p + 1], V[g, : p + 1], b.scale)
+    compare(bits(outs[1])[rows], ref, b.dtype, "prefill mixed batch, dynamic order, sampled rows")
+
+
 def test_one_long_context_short_chunk():
     """A 64-token chunk at the end of a 40000-token context (313 K/V tiles, the
     last one ragged) and a second sequence of 3 tokens: the load warps' block-id

@@ -4,7 +4,9 @@ kernel (``csrc/paged_prefill.cu``), run on the CPU.
 Roles are generators that wait and arrive exactly as the kernel's warps do:
 the K and V load warps (Q tiles into two buffers, K/V tiles into two stages),
 the S-issuing and the P V-issuing MMA warps, and eight softmax warps (with a
-random lazy rescale of O and the per-item epilogue).  mbarriers complete a
+random lazy rescale of O and the per-item epilogue).  The K-load warp takes
+every item (empty ones included) and publishes its index in a four-slot ring,
+which the eleven other warps read before they start the item.  mbarriers complete a
 phase when their expected arrivals are in; a wait is the parity test the
 hardware does.  tcgen05 work runs on one in-order pipe, a commit arrives once
 everything its thread issued before it is done; TMA loads land in any order.
@@ -51,6 +53,10 @@ def run_model(ntiles_per_item, seed, drop=None):
     bar("o")
     bar("end")
     bar("x", 8)
+    for i in range(4):
+        bar(f"item{i}")
+        bar(f"itemfree{i}", 11)
+    ring = {}
     pipe, loads = [], []
     pending = {}          # resource -> list of async ops reading it
     s_ops = {}            # global tile -> S op
@@ -72,9 +78,45 @@ def run_model(ntiles_per_item, seed, drop=None):
 
     items = [n for n in ntiles_per_item]
 
+    def publish(k):
+        """The K-load warp takes item k (len(items): the end) and publishes its
+        index in slot k % 4, once the eleven readers have read what the slot
+        held four items back."""
+        if k >= 4 and drop != "itemfree":
+            yield from wait(f"itemfree{k % 4}", (k - 4) >> 2)
+        ring[k % 4] = k
+        bars[f"item{k % 4}"].arrive()
+        yield
+
+    def read_items():
+        """Another warp's view of the item sequence: item k's tile count, then
+        None at the end."""
+        for k in range(len(items) + 1):
+            yield from wait(f"item{k % 4}", k >> 2)
+            assert ring[k % 4] == k, "a warp read another item's index"
+            bars[f"itemfree{k % 4}"].arrive()
+            yield ("item", items[k] if k < len(items) else None)
+
+    def walk(gen):
+        """The tile counts of the items, as read from the ring (waits pass
+        through)."""
+        for x in gen:
+            if isinstance(x, tuple):
+                return x[1]
+            yield x
+        return None
+
     def producer(kind):
         n = jt = 0
-        for nt in items:
+        src = None if kind == "K" else read_items()
+        for k in range(len(items) + 1):
+            if kind == "K":
+                yield from publish(k)
+                nt = items[k] if k < len(items) else None
+            else:
+                nt = yield from walk(src)
+            if nt is None:
+                break
             if nt == 0:
                 continue
             if kind == "K":
@@ -95,7 +137,11 @@ def run_model(ntiles_per_item, seed, drop=None):
 
     def s_issuer():
         n = jt = 0
-        for nt in items:
+        src = read_items()
+        while True:
+            nt = yield from walk(src)
+            if nt is None:
+                break
             if nt == 0:
                 continue
             qb = n & 1
@@ -118,7 +164,11 @@ def run_model(ntiles_per_item, seed, drop=None):
 
     def pv_issuer():
         n = jt = 0
-        for nt in items:
+        src = read_items()
+        while True:
+            nt = yield from walk(src)
+            if nt is None:
+                break
             if nt == 0:
                 continue
             for j in range(nt):
@@ -139,7 +189,11 @@ def run_model(ntiles_per_item, seed, drop=None):
 
     def softmax():
         n = jt = 0
-        for nt in items:
+        src = read_items()
+        while True:
+            nt = yield from walk(src)
+            if nt is None:
+                break
             if nt == 0:
                 continue
             for j in range(nt):
@@ -212,11 +266,11 @@ def test_protocol_holds_on_random_schedules():
         run_model(_items(seed), seed)
 
 
-@pytest.mark.parametrize("drop", ["qfree", "pfree", "end"])
+@pytest.mark.parametrize("drop", ["qfree", "pfree", "end", "itemfree"])
 def test_each_synchronisation_is_needed(drop):
-    """Removing the Q-buffer release, the S-buffer release (P V done) or the
+    """Removing the Q-buffer release, the S-buffer release (P V done), the
     one-phase final barrier (falling back to a parity wait on the per-tile
-    P V barrier) breaks some schedule."""
+    P V barrier) or the item ring's release breaks some schedule."""
     failures = 0
     for seed in range(300):
         try:

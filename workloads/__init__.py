@@ -618,7 +618,21 @@ def prefill_gqa_chunked(seed: int = 7) -> PrefillBatch:
                          context_lens=[8192] * 8, chunk_lens=[1024] * 8, name="prefill_gqa_chunked")
 
 
+def prefill_mixed(seed: int = 11) -> PrefillBatch:
+    """A mixed serving batch: 16 sequences whose chunks are 64..2048 tokens
+    (uniform) on top of 0..6000 cached tokens (uniform), 32 q / 8 kv heads,
+    head_dim 128, 16-token blocks, bf16.  The work per (sequence, kv head)
+    differs by up to ~100x, which is what an even spread of work over the
+    SMs has to absorb."""
+    r = np.random.default_rng(seed)
+    C = r.integers(64, 2049, 16)
+    L = C + r.integers(0, 6001, 16)
+    return prefill_batch(seed, dtype=BF16, num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                         context_lens=[int(x) for x in L], chunk_lens=[int(x) for x in C], name="prefill_mixed")
+
+
 PREFILL_WORKLOADS = {
     "prefill_llama7b": prefill_llama7b,
     "prefill_gqa_chunked": prefill_gqa_chunked,
+    "prefill_mixed": prefill_mixed,
 }
