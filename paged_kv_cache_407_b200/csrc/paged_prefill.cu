@@ -229,7 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_item = bars + 192;
   const uint32_t bar_itemfree = bars + 224;
   constexpr int kItemReaders = 3 + kSoftmaxWarps;  // V-load, S-issue, P V-issue and softmax warps
-  volatile int *item_ring = reinterpret_cast<volatile int *>(smem + TN::kBarOff + 256);
+  // [4] int32 slots.  Its address is derived from the shared window's base
+  // where it is used, so no register holds it through the other roles' loops.
+  auto item_slot = [&](int slot) -> uint32_t {
+    return ((smem_addr(smem_raw) + 1023u) & ~1023u) + TN::kBarOff + 256u + 4u * static_cast<uint32_t>(slot);
+  };
 
   pdl_trigger();
   pdl_wait();  // before any global access and before taking tensor memory
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto read_item = [&](int k, int &i) -> bool {
     const int slot = k & 3;
     if (!wait(bar_item + 8 * slot, (k >> 2) & 1)) return false;
-    i = item_ring[slot];
+    asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(i) : "r"(item_slot(slot)) : "memory");
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_itemfree + 8 * slot);
     return true;
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           idx = a.ticket != nullptr ? static_cast<int>(min(atomicAdd(a.ticket, 1u), 0x7fffffffu))
                                     : item_index(a, k);
           if (idx >= a.items) idx = -1;
-          item_ring[slot] = idx;
+          asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(item_slot(slot)), "r"(idx) : "memory");
           mbar_arrive(bar_item + 8 * slot);
         }
         i = __shfl_sync(kFullMask, idx, 0);
