@@ -8,7 +8,9 @@ serves every step while the sequences grow.  Each replay is compared with the
 oracle's attention over every sequence's logical history (no paging at all).
 
 Cases: three partitions at the capacity (the planning kernel clears the split
-counters) and two (an asynchronous memset does, captured as a graph node)."""
+counters) and two (an asynchronous memset does, captured as a graph node).  A
+chunked prefill of a mixed batch is captured and replayed too (its item
+counter reset is a memset node)."""
 
 import numpy as np
 import pytest
@@ -131,4 +133,37 @@ def test_decode_step_replayed_from_a_cuda_graph(dtype, B, Hq, Hkv, D, lens, P, s
         check(q, f"graph case, replay {t + 1}")
     assert int(st.item()) == 0
     assert max(len(h) for h in hist_k) <= cap
+    del graph
+
+
+def test_prefill_replayed_from_a_cuda_graph():
+    """The chunked prefill of a mixed batch (cache write of the chunks, then
+    prefill with its item counter zeroed by a memset node) captured once and
+    replayed twice: each replay's output equals the eagerly issued call's bit
+    for bit (every work item is computed whole by one CTA, whatever order
+    the CTAs take the items in)."""
+    from workloads.device import upload_prefill
+    b = W.prefill_mixed()
+    db = upload_prefill(b)
+    st = status_tensor()
+    ws = torch.empty(pkv.PREFILL_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step(out):
+        pkv.reshape_and_cache(db.key, db.value, db.k_cache, db.v_cache, db.slot_mapping, d_status=st)
+        pkv.paged_prefill(out, db.q, db.k_cache, db.v_cache, db.block_tables, db.query_start, db.context_lens,
+                          b.max_query_len, b.scale, d_status=st, workspace=ws)
+
+    eager = torch.full_like(db.q, float("nan"))
+    step(eager)
+    torch.cuda.synchronize()
+    out = torch.full_like(db.q, float("nan"))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(out)
+    for _ in range(2):
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    assert int(st.item()) == 0
     del graph
