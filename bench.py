@@ -782,8 +782,14 @@ class DecodeRunner:
 
         torch.cuda.synchronize(self.dev)
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step()
+        try:
+            # thread-local capture: other threads' CUDA calls (NCCL's
+            # watchdog under torchrun) do not break it
+            with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+                step()
+        except RuntimeError as e:
+            torch.cuda.synchronize(self.dev)
+            return {"unavailable": f"capture failed: {str(e).splitlines()[0][:160]}"}
         for _ in range(3):
             graph.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
