@@ -8,10 +8,11 @@
 //
 // A work item is a (128-row query tile, kv head, sequence); a tile row is one
 // (token, query head of the group) pair, so 128 / G tokens per tile.  The
-// grid is persistent (one CTA per SM), each CTA walking a fixed share of the
-// items, so that the next item's Q tile and first K/V tiles load while the
-// current one finishes.  Roles (warp-specialised, synchronised only through
-// mbarriers):
+// grid is persistent (one CTA per SM): each CTA takes its next item from a
+// counter in the caller's workspace as it frees up (or, without one, walks a
+// fixed share of the items), so that the next item's Q tile and first K/V
+// tiles load while the current one finishes.  Roles (warp-specialised,
+// synchronised only through mbarriers):
 //   warps 0-7  softmax, two threads per row, each owning one 64-token half of
 //              every K/V tile with its own running max, sum and O
 //              accumulator (merged once at the end): tcgen05.ld of its TMEM
@@ -20,13 +21,15 @@
 //              is rescaled, after P V(j-1) is done), P written back into the
 //              same TMEM columns (fp16, or bf16 high + bf16 residual, since
 //              bf16 alone would round P by 2^-9), finally the merged O / l;
-//   warp 8     TMA: the Q tiles (rank-3 map over [T][Hq][D], two buffers)
-//              and the K tiles,
-//              128 tokens gathered through the Block Table, one TMA box per
-//              block (a rank-5 view of [N][Hkv][B][D] that lands the block
-//              as groups of 8 rows, so that the tile's 8-row groups sit at
-//              one fixed stride for the tensor core), two stages;
-//   warp 9     TMA: the V tiles, two stages;
+//   warp 8     takes the items and publishes each index to the other warps
+//              (a four-slot ring in shared memory); TMA: the Q tiles (rank-3
+//              map over [T][Hq][D], two buffers) and the K tiles, 128 tokens
+//              gathered through the Block Table, one TMA box per block (a
+//              rank-5 view of [N][Hkv][B][D] that lands the block as groups of
+//              8 rows, so that the tile's 8-row groups sit at one fixed stride
+//              for the tensor core), lane b issuing block b's box, the block
+//              ids read ahead by cp.async; two stages;
+//   warp 9     TMA: the V tiles, the same way, two stages;
 //   warp 10    tcgen05.mma, one thread: S(j) = Q K(j)^T (128x128x128) into
 //              one of two TMEM buffers, once P V(j-2) has read that buffer;
 //   warp 11    tcgen05.mma, one thread: O_h += P_h(j) V_h(j) with P read from
