@@ -13,14 +13,15 @@
 // fixed share of the items), so that the next item's Q tile and first K/V
 // tiles load while the current one finishes.  Roles (warp-specialised,
 // synchronised only through mbarriers):
-//   warps 0-7  softmax, two threads per row, each owning one 64-token half of
-//              every K/V tile with its own running max, sum and O
-//              accumulator (merged once at the end): tcgen05.ld of its TMEM
-//              lane of S, causal mask, lazy rescaling (the reference max moves
-//              only when the row max grows by more than 2^8; then O_h in TMEM
-//              is rescaled, after P V(j-1) is done), P written back into the
-//              same TMEM columns (fp16, or bf16 high + bf16 residual, since
-//              bf16 alone would round P by 2^-9), finally the merged O / l;
+//   warps 0-7  softmax, 16 rows per warp: read with the 16-lane tcgen05.ld
+//              shape, a row's 128 scores of a tile sit with the four threads
+//              of one quad (32 each, two rows per thread), so the row max and
+//              sum are two shuffles and one O accumulator serves the row.
+//              Causal mask, lazy rescaling (the reference max moves only when
+//              the row max grows by more than 2^8; then O in TMEM is rescaled,
+//              after P V(j-1) is done), P written back into the S buffer as
+//              the A operand (fp16, or bf16 high + bf16 residual, since bf16
+//              alone would round P by 2^-9), finally O / l;
 //   warp 8     takes the items and publishes each index to the other warps
 //              (a four-slot ring in shared memory); TMA: the Q tiles (rank-3
 //              map over [T][Hq][D], two buffers) and the K tiles, 128 tokens
@@ -31,10 +32,10 @@
 //              ids read ahead by cp.async; two stages;
 //   warp 9     TMA: the V tiles, the same way, two stages;
 //   warp 10    tcgen05.mma, one thread: S(j) = Q K(j)^T (128x128x128) into
-//              one of two TMEM buffers, once P V(j-2) has read that buffer;
-//   warp 11    tcgen05.mma, one thread: O_h += P_h(j) V_h(j) with P read from
-//              tensor memory (the S buffer) and V from shared memory
-//              (MN-major).  Two issuers, because a thread that has just
+//              one of three TMEM buffers, once P V(j-3) has read that buffer;
+//   warp 11    tcgen05.mma, one thread: O += P(j) V(j) with P read from tensor
+//              memory (the S buffer) and V from shared memory (MN-major).
+//              Two issuers, because a thread that has just
 //              issued a batch of MMAs waits for the tensor pipe to take them
 //              before its next barrier test completes: with one issuer every
 //              operand wait sat on the pipe's critical path.
@@ -62,14 +63,14 @@ constexpr int kLoadVWarp = 9;     // TMA loads of V tiles
 constexpr int kMmaWarp = 10;      // issues the S = Q K^T MMAs
 constexpr int kPvWarp = 11;       // issues the O += P V MMAs
 constexpr int kThreads = 32 * 12;
-constexpr int kHalf = 64;         // tokens of a K/V tile per softmax half
 constexpr uint32_t kChunk = 128u * 128u;  // [128 rows][64 elements] of 16-bit: 16 KB
 constexpr uint32_t kTile = 2u * kChunk;   // [128][128] of 16-bit: 32 KB
 constexpr uint32_t kQOff = 0;               // two Q buffers (this item's, the next one's)
 constexpr uint32_t kKOff = 2u * kTile;       // two K stages
 constexpr uint32_t kVOff = 4u * kTile;       // two V stages
 constexpr uint32_t kXOff = 6u * kTile;       // final (m, l) exchange of the softmax halves
-constexpr uint32_t kTmemCols = 512;          // S buffers [0, 256), O of half 0 / 1 [256, 512)
+constexpr int kSBufs = 3;                    // S buffers in tensor memory
+constexpr uint32_t kTmemCols = 512;          // S buffers [0, 384), O [384, 512)
 constexpr float kLazyRescale = 8.f;               // log2 of the largest P allowed
 constexpr uint32_t kFullMask = 0xffffffffu;
 
@@ -208,19 +209,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_kfree = bars + 48;   // [2] K stage read by S (MMA commit)
   const uint32_t bar_v = bars + 64;       // [2] V stage loaded
   const uint32_t bar_vfree = bars + 80;   // [2] V stage read by P V
-  const uint32_t bar_s = bars + 96;       // [2] S buffer written (MMA commit)
+  const uint32_t bar_s = bars + 96;       // [3] S buffer written (MMA commit)
   // P-ready comes one per S buffer: a softmax warp may arrive for tile j+1
   // before a slower one arrives for tile j, and those arrivals must not
   // count towards the same phase.
-  const uint32_t bar_p = bars + 112;      // [2] P in TMEM, O rescaled (one arrival per softmax warp)
-  const uint32_t bar_pfree = bars + 128;  // [2] P in the S buffer read by P V (MMA commit)
-  const uint32_t bar_o = bars + 144;      // P V done (MMA commit)
-  // The item's last P V done (MMA commit).  The final read of O cannot use
-  // bar_o: when the softmax warps finish their last tile, P V(n-2) may still
-  // be running as well as P V(n-1), and a parity wait cannot tell two
-  // outstanding phases from none.
-  const uint32_t bar_end = bars + 152;
-  const uint32_t bar_x = bars + 168;      // softmax halves' final (m, l) exchanged
+  const uint32_t bar_p = bars + 120;      // [3] P in TMEM, O rescaled (one arrival per softmax warp)
+  // [3] P V of the buffer's tile done (MMA commit): frees the S buffer, and
+  // tells the softmax that O holds that tile's product (for the rescale, and
+  // for the epilogue after an item's last tile).  A wait on it cannot be
+  // ambiguous: its next phase needs P of three tiles on, which the waiting
+  // warp has not written.
+  const uint32_t bar_pfree = bars + 144;
   const uint32_t bar_done = bars + 176;   // drain on the error path
   const uint32_t holder = bars + 184;
   volatile uint32_t *holder_ptr = reinterpret_cast<volatile uint32_t *>(smem + TN::kBarOff + 184);
@@ -250,13 +249,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_kfree + 8 * i, 1);
       mbar_init(bar_v + 8 * i, 1);
       mbar_init(bar_vfree + 8 * i, 1);
+    }
+#pragma unroll
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar_s + 8 * i, 1);
       mbar_init(bar_p + 8 * i, kSoftmaxWarps);
       mbar_init(bar_pfree + 8 * i, 1);
     }
-    mbar_init(bar_o, 1);
-    mbar_init(bar_end, 1);
-    mbar_init(bar_x, kSoftmaxWarps);
     mbar_init(bar_done, 2);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -270,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *holder_ptr;
-  const uint32_t tO = tmem + 2 * kKv;  // O of half h at tO + h * kDim
+  const uint32_t tO = tmem + kSBufs * kKv;  // O [128 rows][128 columns]
 
   // A wait that gives up after ~1 s (then every role stops).
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
@@ -407,12 +406,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(run = wait(bar_q + 8 * qb, (n >> 1) & 1))) break;
         const uint32_t qbase = sb + kQOff + qb * kTile;
         for (int j = 0; j < it.ntiles; ++j, ++jt) {
-          const int b = jt & 1;
-          if (jt >= 2 && !(run = wait(bar_pfree + 8 * b, ((jt - 2) >> 1) & 1))) break;
-          if (!(run = wait(bar_k + 8 * b, (jt >> 1) & 1))) break;
+          const int b = jt % kSBufs;  // S buffer
+          const int ks = jt & 1;      // K stage
+          if (jt >= kSBufs && !(run = wait(bar_pfree + 8 * b, (jt / kSBufs - 1) & 1))) break;
+          if (!(run = wait(bar_k + 8 * ks, (jt >> 1) & 1))) break;
           if (lane == 0) {
             tc::fence_after_sync();
-            const uint32_t kb = sb + kKOff + b * kTile;
+            const uint32_t kb = sb + kKOff + ks * kTile;
 #pragma unroll
             for (int kk = 0; kk < kDim / 16; ++kk) {
               const uint32_t qoff = (kk >> 2) * kChunk + (kk & 3) * 32u;
@@ -421,37 +421,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                              tc::smem_desc_sw128(kb + koff, 16u, kGroupBytes), kIdescS, kk > 0 ? 1u : 0u);
             }
             tc::commit(bar_s + 8 * b);
-            tc::commit(bar_kfree + 8 * b);
+            tc::commit(bar_kfree + 8 * ks);
             if (j == it.ntiles - 1) tc::commit(bar_qfree + 8 * qb);
           }
           __syncwarp();
         }
       } else {
         for (int j = 0; j < it.ntiles; ++j, ++jt) {
-          const int b = jt & 1;
-          if (!(run = wait(bar_v + 8 * b, (jt >> 1) & 1))) break;
-          if (!(run = wait(bar_p + 8 * b, (jt >> 1) & 1))) break;
+          const int b = jt % kSBufs;  // S buffer holding P
+          const int vs = jt & 1;      // V stage
+          if (!(run = wait(bar_v + 8 * vs, (jt >> 1) & 1))) break;
+          if (!(run = wait(bar_p + 8 * b, (jt / kSBufs) & 1))) break;
           // The first P V of an item overwrites O.  It needs P from every
           // softmax warp, which each writes only after reading out the
           // previous item's O, so bar_p orders that too.
           if (lane == 0) {
             tc::fence_after_sync();
-            const uint32_t vb = sb + kVOff + b * kTile;
-            // O_h += P_h V_h: P_h sits in the S buffer's columns of half h
-            // (high part in its first 32 columns, bf16 residual in the next
-            // 32), V_h is V rows 64h .. 64h + 63.
+            const uint32_t vb = sb + kVOff + vs * kTile;
+            // O += P V: P of tokens 16kk .. 16kk + 15 sits in columns 8kk ..
+            // 8kk + 7 of the S buffer (bf16 residuals 64 columns on) and meets
+            // V rows 16kk .. 16kk + 15.
 #pragma unroll
             for (int kk = 0; kk < kKv / 16; ++kk) {
-              const uint32_t h = kk >> 2;
-              const uint32_t pcol = tmem + b * kKv + h * kHalf + (kk & 3) * 8u;
+              const uint32_t pcol = tmem + b * kKv + kk * 8u;
               const uint64_t vdesc = tc::smem_desc_sw128(vb + kk * 2u * kGroupBytes, 1024u, kGroupBytes);
-              tc::mma_f16_ts(tO + h * kDim, pcol, vdesc, kIdescO, (j > 0 || (kk & 3) > 0) ? 1u : 0u);
-              if constexpr (kSplit) tc::mma_f16_ts(tO + h * kDim, pcol + 32u, vdesc, kIdescO, 1u);
+              tc::mma_f16_ts(tO, pcol, vdesc, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+              if constexpr (kSplit) tc::mma_f16_ts(tO, pcol + 64u, vdesc, kIdescO, 1u);
             }
-            tc::commit(bar_o);
-            tc::commit(bar_vfree + 8 * b);
+            tc::commit(bar_vfree + 8 * vs);
             tc::commit(bar_pfree + 8 * b);
-            if (j == it.ntiles - 1) tc::commit(bar_end);
           }
           __syncwarp();
         }
@@ -459,15 +457,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++n;
     }
   } else if (warp < kSoftmaxWarps) {
-    // ------------------------------------- softmax, (row, token half) per thread
-    // Each half of the threads runs its own online softmax over its half of
-    // every K/V tile, with its own O accumulator in TMEM; the two partial
-    // states of a row are merged once at the end of the item (split-K
-    // identity).
-    const int row = tid & (kRows - 1);
-    const int half = tid >> 7;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tOh = tO + half * kDim;
+    // -------------------------- softmax, 16 rows per warp, 2 rows per thread
+    // Warp w reads TMEM lanes (tile rows) 32 (w % 4) + 16 (w / 4) .. + 15
+    // with the 16-lane shapes: thread t holds rows r0 = base + t/4 and
+    // r1 = r0 + 8, columns 2c, 2c + 1 (c = t % 4) of every 8-column group.
+    // The four threads of a row are one quad of the warp, so the row max and
+    // sum are two shuffles, one O accumulator serves the row and tensor
+    // memory holds three S buffers.  P of the token pair (8i + 2c, + 1) goes
+    // to column c + 4i (the A-operand layout), with the 16x128b shape.
+    const int base = 32 * (warp & 3) + 16 * (warp >> 2);
+    const int c = lane & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(base) << 16;
     bool run = true;
     int n = 0;
     int jt = 0;
@@ -477,104 +477,123 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i < 0) break;
       Item it;
       if (!item_at<BS>(a, i, it, tid == 0)) continue;
-      const int t_row = it.tok0 + row / G;  // chunk token of the row
-      const int h_row = row % G;
-      const bool row_valid = t_row < it.C;
-      const int p_row = it.L - it.C + t_row;  // >= L for rows past the chunk
-      float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
-      float l_sum = 0.f;
+      int t_row[2], h_row[2], p_row[2];
+      bool row_valid[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = base + (lane >> 2) + 8 * r;
+        t_row[r] = it.tok0 + row / G;  // chunk token of the row
+        h_row[r] = row % G;
+        row_valid[r] = t_row[r] < it.C;
+        p_row[r] = it.L - it.C + t_row[r];  // >= L for rows past the chunk
+      }
+      float m_ref[2] = {-INFINITY, -INFINITY};  // reference maxima (log2 units)
+      float l_sum[2] = {0.f, 0.f};              // this thread's 32 columns of each row
       for (int j = 0; j < it.ntiles; ++j, ++jt) {
-        const int b = jt & 1;
-        if (!(run = wait(bar_s + 8 * b, (jt >> 1) & 1))) break;
+        const int b = jt % kSBufs;
+        if (!(run = wait(bar_s + 8 * b, (jt / kSBufs) & 1))) break;
         tc::fence_after_sync();
-        float x[kHalf];
+        float x[64];  // x[4g + 2r + e]: row r, token 8g + 2c + e
         {
-          uint32_t r0[32], r1[32];  // both loads in flight, one wait
-          const uint32_t col = tmem + b * kKv + (lane_off | static_cast<uint32_t>(half * kHalf));
-          tc::ld_32x32b_x32(col, r0);
-          tc::ld_32x32b_x32(col + 32u, r1);
+          uint32_t rr[64];
+          tc::ld_16x256b_x16(tmem + b * kKv + lane_off, rr);
           tc::wait_ld();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            x[q] = __uint_as_float(r0[q]);
-            x[32 + q] = __uint_as_float(r1[q]);
+          for (int q = 0; q < 64; ++q) x[q] = __uint_as_float(rr[q]);
+        }
+        int lim[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) lim[r] = min(p_row[r] + 1, it.L) - j * kKv;  // tokens < lim are visible
+        if (lim[0] < kKv || lim[1] < kKv) {
+#pragma unroll
+          for (int g = 0; g < 16; ++g)
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+                x[4 * g + 2 * r + e] = 8 * g + 2 * c + e < lim[r] ? x[4 * g + 2 * r + e] : -INFINITY;
+        }
+        float alpha[2] = {1.f, 1.f};
+        bool move_any = false;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          float m0 = fmaxf(x[2 * r], x[2 * r + 1]), m1 = fmaxf(x[4 + 2 * r], x[4 + 2 * r + 1]);
+#pragma unroll
+          for (int g = 2; g < 16; g += 2) {
+            m0 = max3(m0, x[4 * g + 2 * r], x[4 * g + 2 * r + 1]);
+            m1 = max3(m1, x[4 * g + 4 + 2 * r], x[4 * g + 4 + 2 * r + 1]);
+          }
+          float mt = fmaxf(m0, m1);
+          mt = fmaxf(mt, __shfl_xor_sync(kFullMask, mt, 1));
+          mt = fmaxf(mt, __shfl_xor_sync(kFullMask, mt, 2));
+          mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
+          if (mt > m_ref[r] + kLazyRescale) {
+            alpha[r] = fast_exp2(m_ref[r] - mt);  // 0 while m_ref is -inf
+            m_ref[r] = mt;
+            l_sum[r] *= alpha[r];
+            move_any = true;
           }
         }
-        const int lim = min(p_row + 1, it.L) - (j * kKv + half * kHalf);  // columns < lim are visible
-        if (lim < kHalf) {
-#pragma unroll
-          for (int c = 0; c < kHalf; ++c) x[c] = c < lim ? x[c] : -INFINITY;
-        }
-        float mp[8];  // eight independent partial maxima, two columns per step
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mp[q] = x[q];
-#pragma unroll
-        for (int c = 8; c < kHalf; c += 2) mp[(c >> 1) & 7] = max3(mp[(c >> 1) & 7], x[c], x[c + 1]);
-        float mt = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
-        mt *= a.scale_log2;  // scale > 0: the max of the scaled scores
-        const bool move = mt > m_ref + kLazyRescale;
-        float alpha = 1.f;
-        if (move) {
-          alpha = fast_exp2(m_ref - mt);  // 0 while m_ref is -inf
-          m_ref = mt;
-          l_sum *= alpha;
-        }
-        if (j > 0 && __any_sync(kFullMask, move)) {
-          // O_h must hold P V(j-1) before it is rescaled.  P V(j-2) is done
-          // (S(j) waited for it) and P V(j) needs this warp's P(j), so
-          // exactly one phase of bar_o can be outstanding here.
-          if (!(run = wait(bar_o, (jt - 1) & 1))) break;
+        if (j > 0 && __any_sync(kFullMask, move_any)) {
+          // O must hold P V(j-1) before it is rescaled; P V(j) needs this
+          // warp's P(j), so nothing else writes O meanwhile.
+          const int jp = jt - 1;
+          if (!(run = wait(bar_pfree + 8 * (jp % kSBufs), (jp / kSBufs) & 1))) break;
           tc::fence_after_sync();
 #pragma unroll
-          for (int cc = 0; cc < 4; cc += 2) {
-            uint32_t r0[32], r1[32];
-            const uint32_t col = tOh + (lane_off | static_cast<uint32_t>(cc * 32));
-            tc::ld_32x32b_x32(col, r0);
-            tc::ld_32x32b_x32(col + 32u, r1);
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[16];
+            tc::ld_16x256b_x4(tO + lane_off + 32u * ch, o);
             tc::wait_ld();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              r0[q] = __float_as_uint(__uint_as_float(r0[q]) * alpha);
-              r1[q] = __float_as_uint(__uint_as_float(r1[q]) * alpha);
-            }
-            tc::st_32x32b_x32(col, r0);
-            tc::st_32x32b_x32(col + 32u, r1);
+            for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[(q >> 1) & 1]);
+            tc::st_16x256b_x4(tO + lane_off + 32u * ch, o);
           }
           tc::wait_st();
         }
-        // P of this half into the S buffer's columns of the half (A operand
-        // of P V in tensor memory): high part, then the bf16 residual
-        const float mref = m_ref == -INFINITY ? 0.f : m_ref;  // no visible token yet: P = 0
-        {
-          uint32_t hi[32], lo[32];
-          // column pairs in packed fp32 arithmetic (one instruction per pair)
-          const float2 sc = make_float2(a.scale_log2, a.scale_log2);
-          const float2 nm = make_float2(-mref, -mref);
-          float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // independent partial sums
+        // P into the S buffer (A operand of P V in tensor memory): high parts
+        // in columns 0 .. 63, bf16 residuals in 64 .. 127; two halves of the
+        // token range, so fewer values are live at once
+        const float2 sc = make_float2(a.scale_log2, a.scale_log2);
+        float2 nm[2];
 #pragma unroll
-          for (int e = 0; e < kHalf / 2; ++e) {
-            const float2 t = __ffma2_rn(make_float2(x[2 * e], x[2 * e + 1]), sc, nm);
-            const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-            ls[e & 1] = __fadd2_rn(ls[e & 1], p);
-            hi[e] = Pack<T>::pack(p.x, p.y);
-            if constexpr (kSplit) {
-              const float2 r = __ffma2_rn(Pack<T>::unpack(hi[e]), make_float2(-1.f, -1.f), p);
-              lo[e] = Pack<T>::pack(r.x, r.y);
+        for (int r = 0; r < 2; ++r) {
+          const float mr = m_ref[r] == -INFINITY ? 0.f : m_ref[r];  // no visible token yet: P = 0
+          nm[r] = make_float2(-mr, -mr);
+        }
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t hi[16], lo[16];  // [2 g' + r]: group 8 hf + g', row r
+#pragma unroll
+          for (int g2 = 0; g2 < 8; ++g2) {
+            const int g = 8 * hf + g2;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const float2 t = __ffma2_rn(make_float2(x[4 * g + 2 * r], x[4 * g + 2 * r + 1]), sc, nm[r]);
+              const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+              ls[r] = __fadd2_rn(ls[r], p);
+              hi[2 * g2 + r] = Pack<T>::pack(p.x, p.y);
+              if constexpr (kSplit) {
+                const float2 q2 = __ffma2_rn(Pack<T>::unpack(hi[2 * g2 + r]), make_float2(-1.f, -1.f), p);
+                lo[2 * g2 + r] = Pack<T>::pack(q2.x, q2.y);
+              }
             }
           }
-          const float2 lsum = __fadd2_rn(ls[0], ls[1]);
-          l_sum += lsum.x + lsum.y;
-          const uint32_t pcol = tmem + b * kKv + half * kHalf;
-          tc::st_32x32b_x32(pcol + lane_off, hi);
-          if constexpr (kSplit) tc::st_32x32b_x32(pcol + 32u + lane_off, lo);
-          tc::wait_st();
+          const uint32_t pcol = tmem + b * kKv + lane_off + 32u * hf;
+          tc::st_16x128b_x8(pcol, hi);
+          if constexpr (kSplit) tc::st_16x128b_x8(pcol + 64u, lo);
         }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) l_sum[r] += ls[r].x + ls[r].y;
+        tc::wait_st();
         // V(j) landed; tokens past the context get zero rows, so that P = 0
         // never meets a NaN in stale shared memory
         const int valid_tok = min(kKv, it.L - j * kKv);
         if (valid_tok < kKv) {
-          if (!(run = wait(bar_v + 8 * b, (jt >> 1) & 1))) break;
-          uint8_t *vt = smem + kVOff + b * kTile;
+          const int vs = jt & 1;
+          if (!(run = wait(bar_v + 8 * vs, (jt >> 1) & 1))) break;
+          uint8_t *vt = smem + kVOff + vs * kTile;
           for (int u = valid_tok * 16 + tid; u < kKv * 16; u += kSoftmaxThreads) {
             const int r = u >> 4, w = u & 15;  // token row, 16-byte unit of its 256 bytes
             *reinterpret_cast<uint4 *>(vt + (r >> 3) * kGroupBytes + (w >> 3) * 1024 + (r & 7) * 128 +
@@ -587,49 +606,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar_p + 8 * b);
       }
       if (!run) break;
-      // ---- epilogue of the item: merge the two halves' states of the row
-      if (!(run = wait(bar_end, n & 1))) break;
+      // ---- epilogue of the item: row sums over the quad, O / l, once the
+      // item's last P V is done
+      const int jl = jt - 1;
+      if (!(run = wait(bar_pfree + 8 * (jl % kSBufs), (jl / kSBufs) & 1))) break;
       tc::fence_after_sync();
-      float2 *xch = reinterpret_cast<float2 *>(smem + kXOff);
-      xch[half * kRows + row] = make_float2(m_ref, l_sum);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_x);
-      if (!(run = wait(bar_x, n & 1))) break;
-      const float2 o0 = xch[row];
-      const float2 o1 = xch[kRows + row];
-      const float M = fmaxf(o0.x, o1.x);
-      const float w0 = o0.x == -INFINITY ? 0.f : fast_exp2(o0.x - M);
-      const float w1 = o1.x == -INFINITY ? 0.f : fast_exp2(o1.x - M);
-      const float Ls = w0 * o0.y + w1 * o1.y;
-      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-      const float c0 = w0 * inv, c1 = w1 * inv;
-      // this thread writes output columns half*64 .. half*64 + 63
-      T *orow = static_cast<T *>(a.out) +
-                (static_cast<size_t>(it.t_begin + t_row) * a.num_q_heads + it.g * G + h_row) * kDim + half * kHalf;
+      float inv[2];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t r0[32], r1[32];
-        const uint32_t col = static_cast<uint32_t>(half * kHalf + cc * 32);
-        tc::ld_32x32b_x32(tO + (lane_off | col), r0);
-        tc::ld_32x32b_x32(tO + kDim + (lane_off | col), r1);
+      for (int r = 0; r < 2; ++r) {
+        float L = l_sum[r];
+        L += __shfl_xor_sync(kFullMask, L, 1);
+        L += __shfl_xor_sync(kFullMask, L, 2);
+        inv[r] = L > 0.f ? 1.f / L : 0.f;
+      }
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[16];  // [4 g' + 2 r + e]: row r, column 32 ch + 8 g' + 2c + e
+        tc::ld_16x256b_x4(tO + lane_off + 32u * ch, o);
         tc::wait_ld();
-        if (row_valid) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            float v[8];
+        for (int r = 0; r < 2; ++r) {
+          if (!row_valid[r]) continue;
+          T *orow = static_cast<T *>(a.out) +
+                    (static_cast<size_t>(it.t_begin + t_row[r]) * a.num_q_heads + it.g * G + h_row[r]) * kDim;
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const int q = q4 * 8 + e;
-              const float2 w = __ffma2_rn(make_float2(__uint_as_float(r0[q]), __uint_as_float(r0[q + 1])),
-                                          make_float2(c0, c0),
-                                          __fmul2_rn(make_float2(__uint_as_float(r1[q]), __uint_as_float(r1[q + 1])),
-                                                     make_float2(c1, c1)));
-              v[e] = w.x;
-              v[e + 1] = w.y;
-            }
-            *reinterpret_cast<uint4 *>(orow + cc * 32 + q4 * 8) =
-                make_uint4(Pack<T>::pack(v[0], v[1]), Pack<T>::pack(v[2], v[3]), Pack<T>::pack(v[4], v[5]),
-                           Pack<T>::pack(v[6], v[7]));
+          for (int g2 = 0; g2 < 4; ++g2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[4 * g2 + 2 * r]), __uint_as_float(o[4 * g2 + 2 * r + 1])),
+                                        make_float2(inv[r], inv[r]));
+            *reinterpret_cast<uint32_t *>(orow + 32 * ch + 8 * g2 + 2 * c) = Pack<T>::pack(v.x, v.y);
           }
         }
       }

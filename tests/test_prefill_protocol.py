@@ -4,19 +4,22 @@ kernel (``csrc/paged_prefill.cu``), run on the CPU.
 Roles are generators that wait and arrive exactly as the kernel's warps do:
 the K and V load warps (Q tiles into two buffers, K/V tiles into two stages),
 the S-issuing and the P V-issuing MMA warps, and eight softmax warps (with a
-random lazy rescale of O and the per-item epilogue).  The K-load warp takes
-every item (empty ones included) and publishes its index in a four-slot ring,
-which the eleven other warps read before they start the item.  mbarriers complete a
-phase when their expected arrivals are in; a wait is the parity test the
-hardware does.  tcgen05 work runs on one in-order pipe, a commit arrives once
-everything its thread issued before it is done; TMA loads land in any order.
+random lazy rescale of O and the per-item epilogue).  S goes through three
+tensor-memory buffers; P overwrites S in its buffer; one O accumulator.  The
+K-load warp takes every item (empty ones included) and publishes its index in
+a four-slot ring, which the eleven other warps read before they start the
+item.  mbarriers complete a phase when their expected arrivals are in; a wait
+is the parity test the hardware does.  tcgen05 work runs on one in-order pipe,
+a commit arrives once everything its thread issued before it is done; TMA
+loads land in any order.
 
 Checked on every schedule: no deadlock; every parity wait releases exactly on
 the phase it means (a wait that could be satisfied by an older or a newer
 phase is a bug even when the schedule happens to be benign); no buffer (Q, K
 and V stages, S buffers in tensor memory, O) is rewritten while an
 asynchronous reader is pending, or read before its writer completed.  Each
-synchronisation the kernel relies on, removed, makes some schedule fail.
+synchronisation the kernel relies on, removed or pointed at the wrong tile,
+makes some schedule fail.
 """
 
 import random
@@ -24,6 +27,8 @@ import random
 import pytest
 
 pytestmark = pytest.mark.filterwarnings("ignore")
+
+NS = 3  # S buffers in tensor memory
 
 
 class Bar:
@@ -39,7 +44,8 @@ class Bar:
 
 def run_model(ntiles_per_item, seed, drop=None):
     """ntiles_per_item: K/V tiles of each item of one CTA (0 = an empty item,
-    skipped by every role).  drop: name of one synchronisation to remove."""
+    skipped by every role).  drop: name of one synchronisation to remove (or,
+    for "rescale" / "epilogue", to point at the tile before the right one)."""
     rnd = random.Random(seed)
     bars = {}
 
@@ -47,20 +53,20 @@ def run_model(ntiles_per_item, seed, drop=None):
         bars[name] = Bar(name, count)
 
     for i in range(2):
-        for nm in ("q", "qfree", "k", "kfree", "v", "vfree", "s", "pfree"):
+        for nm in ("q", "qfree", "k", "kfree", "v", "vfree"):
             bar(f"{nm}{i}")
+    for i in range(NS):
+        bar(f"s{i}")
+        bar(f"pfree{i}")
         bar(f"p{i}", 8)
-    bar("o")
-    bar("end")
-    bar("x", 8)
     for i in range(4):
         bar(f"item{i}")
         bar(f"itemfree{i}", 11)
     ring = {}
     pipe, loads = [], []
-    pending = {}          # resource -> list of async ops reading it
+    pending = {}          # resource -> list of async ops reading (or writing) it
     s_ops = {}            # global tile -> S op
-    st = {"pv_item": -1, "o_readers": 0}
+    st = {"pv_item": -1, "o_readers": 0, "s_readers": {}}
 
     def wait(name, phase):
         b = bars[name]
@@ -76,7 +82,7 @@ def run_model(ntiles_per_item, seed, drop=None):
         for r in res:
             pending.setdefault(r, []).append(op)
 
-    items = [n for n in ntiles_per_item]
+    items = list(ntiles_per_item)
 
     def publish(k):
         """The K-load warp takes item k (len(items): the end) and publishes its
@@ -98,8 +104,8 @@ def run_model(ntiles_per_item, seed, drop=None):
             yield ("item", items[k] if k < len(items) else None)
 
     def walk(gen):
-        """The tile counts of the items, as read from the ring (waits pass
-        through)."""
+        """The next item's tile count as read from the ring (waits pass
+        through); None at the end."""
         for x in gen:
             if isinstance(x, tuple):
                 return x[1]
@@ -147,15 +153,16 @@ def run_model(ntiles_per_item, seed, drop=None):
             qb = n & 1
             yield from wait(f"q{qb}", n >> 1)
             for j in range(nt):
-                b = jt & 1
-                if jt >= 2 and drop != "pfree":
-                    yield from wait(f"pfree{b}", (jt - 2) >> 1)
-                yield from wait(f"k{b}", jt >> 1)
+                b, ks = jt % NS, jt & 1
+                if jt >= NS and drop != "pfree":
+                    yield from wait(f"pfree{b}", jt // NS - 1)
+                yield from wait(f"k{ks}", jt >> 1)
                 assert not busy(f"S{b}"), "S buffer rewritten while P V reads P"
-                op = {"done": False}
-                read(op, f"Q{qb}", f"K{b}")
+                assert st["s_readers"].get(b, 0) == 0, "S buffer rewritten while the softmax reads it"
+                op = {"done": False, "tile": jt}
+                read(op, f"Q{qb}", f"K{ks}")
                 s_ops[jt] = op
-                pipe.extend([("op", op), ("commit", f"s{b}"), ("commit", f"kfree{b}")])
+                pipe.extend([("op", op), ("commit", f"s{b}"), ("commit", f"kfree{ks}")])
                 if j == nt - 1:
                     pipe.append(("commit", f"qfree{qb}"))
                 jt += 1
@@ -172,17 +179,14 @@ def run_model(ntiles_per_item, seed, drop=None):
             if nt == 0:
                 continue
             for j in range(nt):
-                b = jt & 1
-                yield from wait(f"v{b}", jt >> 1)
-                yield from wait(f"p{b}", jt >> 1)
+                b, vs = jt % NS, jt & 1
+                yield from wait(f"v{vs}", jt >> 1)
+                yield from wait(f"p{b}", jt // NS)
                 assert st["o_readers"] == 0, "P V writes O while a softmax warp reads it"
-                op = {"done": False}
-                read(op, f"V{b}", f"S{b}")
-                pending.setdefault("O", []).append(op)
+                op = {"done": False, "tile": jt}
+                read(op, f"V{vs}", f"S{b}", "O")
                 st["pv_item"] = max(st["pv_item"], n)
-                pipe.extend([("op", op), ("commit", "o"), ("commit", f"vfree{b}"), ("commit", f"pfree{b}")])
-                if j == nt - 1 and drop != "end":
-                    pipe.append(("commit", "end"))
+                pipe.extend([("op", op), ("commit", f"vfree{vs}"), ("commit", f"pfree{b}")])
                 jt += 1
                 yield
             n += 1
@@ -197,17 +201,23 @@ def run_model(ntiles_per_item, seed, drop=None):
             if nt == 0:
                 continue
             for j in range(nt):
-                b = jt & 1
-                yield from wait(f"s{b}", jt >> 1)
+                b = jt % NS
+                yield from wait(f"s{b}", jt // NS)
                 assert s_ops[jt]["done"], "S read before its MMA completed"
+                st["s_readers"][b] = st["s_readers"].get(b, 0) + 1
+                yield
+                st["s_readers"][b] -= 1
                 if j == nt - 1 and rnd.random() < 0.5:
                     # the item's last tile reaches past the context: this warp
                     # zeroes the tail rows of the V stage before arriving on P
-                    yield from wait(f"v{b}", jt >> 1)
-                    assert not busy(f"V{b}"), "V stage zeroed while a P V reads it"
-                    assert not any(name == f"v{b}" for name, _ in loads), "V stage zeroed under a landing load"
+                    vs = jt & 1
+                    yield from wait(f"v{vs}", jt >> 1)
+                    assert not busy(f"V{vs}"), "V stage zeroed while a P V reads it"
+                    assert not any(name == f"v{vs}" for name, _ in loads), "V stage zeroed under a landing load"
                 if j > 0 and rnd.random() < 0.3:
-                    yield from wait("o", jt - 1)
+                    jp = jt - 1 if drop != "rescale" else jt - 2
+                    if jp >= 0:
+                        yield from wait(f"pfree{jp % NS}", jp // NS)
                     assert not busy("O"), "O rescaled while a P V is pending"
                     st["o_readers"] += 1
                     yield
@@ -215,13 +225,10 @@ def run_model(ntiles_per_item, seed, drop=None):
                 yield
                 bars[f"p{b}"].arrive()
                 jt += 1
-            if drop == "end":
-                yield from wait("o", jt - 1)
-            else:
-                yield from wait("end", n)
+            jl = jt - 1 if drop != "epilogue" else jt - 2
+            if jl >= 0:
+                yield from wait(f"pfree{jl % NS}", jl // NS)
             assert not busy("O"), "epilogue reads O with a P V pending"
-            bars["x"].arrive()
-            yield from wait("x", n)
             st["o_readers"] += 1
             yield
             assert st["pv_item"] <= n, "next item's P V issued while O is read out"
@@ -266,11 +273,11 @@ def test_protocol_holds_on_random_schedules():
         run_model(_items(seed), seed)
 
 
-@pytest.mark.parametrize("drop", ["qfree", "pfree", "end", "itemfree"])
+@pytest.mark.parametrize("drop", ["qfree", "pfree", "itemfree", "rescale", "epilogue"])
 def test_each_synchronisation_is_needed(drop):
-    """Removing the Q-buffer release, the S-buffer release (P V done), the
-    one-phase final barrier (falling back to a parity wait on the per-tile
-    P V barrier) or the item ring's release breaks some schedule."""
+    """Removing the Q-buffer release, the S-buffer release (P V done) or the
+    item ring's release, or pointing the rescale's or the epilogue's wait at
+    the tile before the one it must wait for, breaks some schedule."""
     failures = 0
     for seed in range(300):
         try:
