@@ -25,7 +25,10 @@
 // arrives with those eight tokens on consecutive shared-memory rows
 // (row 8t + i of tile half u = token 16t + 4(i/2) + i%2 + 2u), and the V tile
 // as rows of 128 bytes, so both ldmatrix patterns are free of bank conflicts
-// under the 128-byte swizzle.
+// under the 128-byte swizzle.  With at most eight query heads per kv head the
+// 8-bit pools use DecodeState8T instead (end of this file): the same tiles and
+// the same fragments read as the other operand, with the tokens on M, half the
+// MMAs and half the accumulator registers.
 #pragma once
 
 #include <type_traits>
@@ -380,6 +383,209 @@ struct DecodeState {
           mm[r + 8] = m1;
           ml[r + 8] = l1;
         }
+      }
+    }
+  }
+};
+
+// 8-bit pools with at most 8 query heads per kv head: the same computation
+// with the tokens on the MMA's M dimension and the heads on N, so one
+// m16n8k16 covers 16 tokens for all (up to eight) heads of the group
+// instead of a 16-row query tile that is mostly padding.  Per 16 tokens:
+//   S[16 slots x 8 heads] = K[16 slots x D] . Q^T          (8 MMAs)
+//   O^T[D x 8 heads]     += V^T[D x 16 slots] . P^T        (8 MMAs)
+// The K tile's rows are already in the permuted token order of the 8-bit
+// layout: 16-token group tp of a block sits in rows tp*8 .. tp*8 + 7 and
+// B/2 + tp*8 .. + 7, and slot s of a group (s < 8 the first run, s >= 8 the
+// second) holds token 16tp + 4((s & 7) >> 1) + 2(s >> 3) + (s & 1).  That
+// order is what makes the A fragments line up: ldmatrix gives lane (g, t) the
+// four codes 4t .. 4t + 3 of slot g's 16-dimension chunk (k-slots 2t, 2t + 1
+// and 2t + 8, 2t + 9 in the head-dimension order that load_q uses for Q), and
+// of dimension g's row of V^T the tokens 16tp + 4t .. + 3, which are exactly
+// the group's slots 2t, 2t + 1, 2t + 8, 2t + 9.  P moves from the accumulator
+// layout of S (slot rows) to the B layout of P^T (head rows) with two 8x8
+// transposes per group.
+template <typename T, int D, int BS>
+struct DecodeState8T {
+  static_assert(BS % 16 == 0, "blocks of whole 16-token groups");
+  static constexpr int kTP = BS / 16;  // 16-token groups per block
+  static constexpr int kMT = D / 16;   // 16-dimension m-tiles of O^T
+  static constexpr int kKS = D / 16;   // 16-deep steps of the score product
+  using MMA = Mma<__half>;
+  using PK = Pack<__half>;
+
+  uint32_t qb0[kKS], qb1[kKS];  // Q^T as B fragments (head g = lane / 4)
+  float ma, mb, la, lb;         // running max / sum of heads 2t and 2t + 1
+  float o[kMT][4];              // O^T: dims g, g + 8 of each m-tile x heads 2t, 2t + 1
+
+  static __device__ __forceinline__ uint32_t q_pair(const T *p) {
+    if constexpr (std::is_same<T, __half>::value) {
+      return *reinterpret_cast<const uint32_t *>(p);
+    } else {
+      const float2 f = Pack<T>::unpack(*reinterpret_cast<const uint32_t *>(p));
+      return Pack<__half>::pack(f.x, f.y);
+    }
+  }
+
+  // B fragment of step kk for head g: k-slots {2t, 2t + 1} are dims
+  // 16kk + 4t + {0, 1}, k-slots {2t + 8, 2t + 9} dims 16kk + 4t + {2, 3}.
+  __device__ __forceinline__ void load_q(const T *q, int G, int lane) {
+    const int g = lane >> 2;
+    const int c4 = (lane & 3) * 4;
+#pragma unroll
+    for (int kk = 0; kk < kKS; ++kk) {
+      qb0[kk] = g < G ? q_pair(q + g * D + 16 * kk + c4) : 0u;
+      qb1[kk] = g < G ? q_pair(q + g * D + 16 * kk + c4 + 2) : 0u;
+    }
+  }
+
+  __device__ __forceinline__ void reset() {
+    ma = mb = -INFINITY;
+    la = lb = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  }
+
+  static __device__ __forceinline__ uint32_t transpose8x8(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+  }
+
+  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int nv, float scale_log2, int lane) {
+    const int mi = lane >> 3;  // ldmatrix: which 8x8 matrix this lane addresses
+    const int ri = lane & 7;   // ldmatrix: which row of it
+    const int g = lane >> 2;
+    const int t = lane & 3;
+
+    // ---- S[16 slots x 8 heads] per group = K . Q^T; even and odd steps in
+    // two chains
+    float s[kTP][4];
+#pragma unroll
+    for (int tp = 0; tp < kTP; ++tp) {
+      float s2[4] = {0.f, 0.f, 0.f, 0.f};
+      s[tp][0] = s[tp][1] = s[tp][2] = s[tp][3] = 0.f;
+#pragma unroll
+      for (int kk2 = 0; kk2 < kKS / 2; ++kk2) {
+        // matrices: slots 0-7 / 8-15 of chunk 2 kk2, then of chunk 2 kk2 + 1
+        uint32_t r0, r1, r2, r3;
+        const int row = (mi & 1) * (BS / 2) + tp * 8 + ri;
+        const int chunk = 2 * kk2 + (mi >> 1);
+        ldsm_x4(kb + row * 128 + ((chunk ^ ri) << 4), r0, r1, r2, r3);
+        uint32_t lo_g, hi_g, lo_g8, hi_g8;
+        e4m3x4_to_f16x2x2(r0, lo_g, hi_g);
+        e4m3x4_to_f16x2x2(r1, lo_g8, hi_g8);
+        MMA::k16(s[tp], lo_g, lo_g8, hi_g, hi_g8, qb0[2 * kk2], qb1[2 * kk2]);
+        e4m3x4_to_f16x2x2(r2, lo_g, hi_g);
+        e4m3x4_to_f16x2x2(r3, lo_g8, hi_g8);
+        MMA::k16(s2, lo_g, lo_g8, hi_g, hi_g8, qb0[2 * kk2 + 1], qb1[2 * kk2 + 1]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[tp][j] += s2[j];
+    }
+    // s[tp][0], [1]: slot g x heads 2t, 2t + 1; [2], [3]: slot g + 8
+    const bool partial = nv < BS;
+    const int tok_g = ((g >> 1) << 2) + (g & 1);  // token of slot g in its group; slot g + 8: + 2
+    float mxa = -INFINITY, mxb = -INFINITY;
+#pragma unroll
+    for (int tp = 0; tp < kTP; ++tp) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float v = s[tp][j] * scale_log2;
+        if (partial && 16 * tp + tok_g + ((j >> 1) << 1) >= nv) v = -INFINITY;
+        s[tp][j] = v;
+      }
+      mxa = fmaxf(mxa, fmaxf(s[tp][0], s[tp][2]));
+      mxb = fmaxf(mxb, fmaxf(s[tp][1], s[tp][3]));
+    }
+#pragma unroll
+    for (int d = 4; d < 32; d <<= 1) {
+      mxa = fmaxf(mxa, __shfl_xor_sync(kFullMask, mxa, d));
+      mxb = fmaxf(mxb, __shfl_xor_sync(kFullMask, mxb, d));
+    }
+    const float mna = fmaxf(ma, mxa), mnb = fmaxf(mb, mxb);
+    const float ba = mna == -INFINITY ? 0.f : mna, bb = mnb == -INFINITY ? 0.f : mnb;
+    const float ala = fast_exp2(ma - ba), alb = fast_exp2(mb - bb);
+    ma = mna;
+    mb = mnb;
+    float rsa = 0.f, rsb = 0.f;
+    uint32_t pb0[kTP], pb1[kTP];  // P^T as B operands: k-slots 2t, 2t + 1 / 2t + 8, 2t + 9 of head g
+#pragma unroll
+    for (int tp = 0; tp < kTP; ++tp) {
+      const float p0 = fast_exp2(s[tp][0] - ba), p1 = fast_exp2(s[tp][1] - bb);
+      const float p2 = fast_exp2(s[tp][2] - ba), p3 = fast_exp2(s[tp][3] - bb);
+      rsa += p0 + p2;
+      rsb += p1 + p3;
+      pb0[tp] = transpose8x8(PK::pack(p0, p1));
+      pb1[tp] = transpose8x8(PK::pack(p2, p3));
+    }
+    la = la * ala + rsa;
+    lb = lb * alb + rsb;
+    if (__any_sync(kFullMask, ala != 1.f || alb != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt) {
+        o[mt][0] *= ala;
+        o[mt][1] *= alb;
+        o[mt][2] *= ala;
+        o[mt][3] *= alb;
+      }
+    }
+
+    // ---- O^T[D x 8] += V^T . P^T per group; lane t's codes of group tp are
+    // tokens 16tp + 4t .. + 3
+#pragma unroll
+    for (int tp = 0; tp < kTP; ++tp) {
+      const int t0 = 16 * tp + 4 * t;
+      const bool vmask = partial && (16 * tp + 16 > nv);
+      const uint32_t bmask = (t0 < nv ? 0x000000ffu : 0u) | (t0 + 1 < nv ? 0x0000ff00u : 0u) |
+                             (t0 + 2 < nv ? 0x00ff0000u : 0u) | (t0 + 3 < nv ? 0xff000000u : 0u);
+#pragma unroll
+      for (int dq = 0; dq < D / 32; ++dq) {
+        uint32_t v[4];  // dims 32dq + 8j + (lane's row) for matrix j
+        ldsm_x4(vb + v8_off<BS>(32 * dq + 8 * mi + ri, tp), v[0], v[1], v[2], v[3]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t lo_g, hi_g, lo_g8, hi_g8;
+          e4m3x4_to_f16x2x2(vmask ? (v[2 * h] & bmask) : v[2 * h], lo_g, hi_g);
+          e4m3x4_to_f16x2x2(vmask ? (v[2 * h + 1] & bmask) : v[2 * h + 1], lo_g8, hi_g8);
+          MMA::k16(o[2 * dq + h], lo_g, lo_g8, hi_g, hi_g8, pb0[tp], pb1[tp]);
+        }
+      }
+    }
+  }
+
+  // Sum l over the eight lanes that share a head pair.
+  __device__ __forceinline__ void reduce_l() {
+#pragma unroll
+    for (int d = 4; d < 32; d <<= 1) {
+      la += __shfl_xor_sync(kFullMask, la, d);
+      lb += __shfl_xor_sync(kFullMask, lb, d);
+    }
+  }
+
+  // Rows < G of the state to shared memory as DecodeState::store_rows does.
+  __device__ __forceinline__ void store_rows(float *mo, float *mm, float *ml, int G, int lane) const {
+    const int g = lane >> 2;
+    const int ha = 2 * (lane & 3), hb = ha + 1;
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt) {
+      if (ha < G) {
+        mo[ha * D + 16 * mt + g] = o[mt][0];
+        mo[ha * D + 16 * mt + g + 8] = o[mt][2];
+      }
+      if (hb < G) {
+        mo[hb * D + 16 * mt + g] = o[mt][1];
+        mo[hb * D + 16 * mt + g + 8] = o[mt][3];
+      }
+    }
+    if (g == 0) {
+      if (ha < G) {
+        mm[ha] = ma;
+        ml[ha] = la;
+      }
+      if (hb < G) {
+        mm[hb] = mb;
+        ml[hb] = lb;
       }
     }
   }

@@ -291,7 +291,8 @@ __global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2, SHOR
                              const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
   using TN = GridTune<D, BS, KV8 ? 1 : 2, SHORT>;
   constexpr int kStageBytes = 2 * BS * D * (KV8 ? 1 : 2);
-  using State = DecodeState<T, D, BS, BIG, KV8>;
+  using State = typename std::conditional<KV8 && !BIG, DecodeState8T<T, D, BS>,
+                                          DecodeState<T, D, BS, BIG, KV8>>::type;
   pdl_trigger();
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
