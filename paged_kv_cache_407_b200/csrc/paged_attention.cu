@@ -259,19 +259,27 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap *tmk,
 // GQA batch (1024-token partitions): 94.8 -> 89.2 us (16-bit), 66.4 -> 58.6
 // us (8-bit); on the 7B batch (whole 2048-token sequences) the same shape
 // is 5-8 % slower, whose longer units make the last wave longer.
-template <int D, int BS, int ESZ = 2, bool SHORT = false>
+// LEAN: the 8-bit instances with the tokens on M (DecodeState8T, at most
+// eight query heads per kv head), which need 128 registers per thread, so one
+// more CTA per SM fits once the stages shrink: for 16-token blocks four CTAs
+// of four warps x three stages (7B batch 99.8 -> 98.4 us per call), or eight
+// of two warps x three stages for short units (GQA batch 53.4 -> 51.1 us).
+template <int D, int BS, int ESZ = 2, bool SHORT = false, bool LEAN = false>
 struct GridTune {
   static constexpr int kStage = 2 * BS * D * ESZ;
   // 8-bit pools with 32-token blocks: two warps with three stages each (four
   // CTAs per SM) measured best; four warps spill under the register cap.
   static constexpr bool kKv8Bs32 = ESZ == 1 && BS == 32;
   static constexpr bool kShort = SHORT && BS == 16;
+  static constexpr bool kLean16 = LEAN && BS == 16;
   static constexpr int kWarps = kShort ? 2 : (kKv8Bs32 ? 2 : (kStage >= 16384 ? 2 : 4));
-  static constexpr int kFit = kShort ? (ESZ == 1 ? 4 : 2) : (kKv8Bs32 ? 3 : 65536 / (kWarps * kStage));
+  static constexpr int kFit = kShort ? (ESZ == 1 ? (LEAN ? 3 : 4) : 2)
+                                     : (kKv8Bs32 || kLean16 ? 3 : 65536 / (kWarps * kStage));
   static constexpr int kStages = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
   // Three CTAs per SM fit in shared memory; ask the register allocation for
-  // three as well (at most 168 registers with four warps); six of two warps.
-  static constexpr int kMinBlocks = kShort ? 6 : 3;
+  // three as well (at most 168 registers with four warps); six of two warps
+  // (LEAN: four and eight, at most 128 registers).
+  static constexpr int kMinBlocks = kShort ? (kLean16 ? 8 : 6) : (kLean16 ? 4 : 3);
   static constexpr int kRing = kWarps * kStages * kStage;
   static constexpr int kMerge = kWarps * 16 * (D + 2) * 4;
   static constexpr int kData = kRing > kMerge ? kRing : kMerge;
@@ -286,10 +294,10 @@ struct GridTune {
 // FAULT = false and none of its code.
 template <typename T, int D, int BS, int WARPS, int NST, bool BIG, bool KV8, bool FAULT = false,
           bool SHORT = false>
-__global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2, SHORT>::kMinBlocks))
+__global__ void __launch_bounds__(WARPS * 32, (GridTune<D, BS, KV8 ? 1 : 2, SHORT, KV8 && !BIG>::kMinBlocks))
     paged_decode_grid_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
-  using TN = GridTune<D, BS, KV8 ? 1 : 2, SHORT>;
+  using TN = GridTune<D, BS, KV8 ? 1 : 2, SHORT, KV8 && !BIG>;
   constexpr int kStageBytes = 2 * BS * D * (KV8 ? 1 : 2);
   using State = typename std::conditional<KV8 && !BIG, DecodeState8T<T, D, BS>,
                                           DecodeState<T, D, BS, BIG, KV8>>::type;
@@ -712,7 +720,7 @@ bool make_plan(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int3
 template <typename T, int D, int BS, bool BIG, bool KV8, bool FAULT = false, bool SHORT = false>
 pkv_status launch_grid(const CUtensorMap &tmk, const CUtensorMap &tmv, const DecodeArgs &args,
                        cudaStream_t stream) {
-  using TN = GridTune<D, BS, KV8 ? 1 : 2, SHORT>;
+  using TN = GridTune<D, BS, KV8 ? 1 : 2, SHORT, KV8 && !BIG>;
   auto kern = paged_decode_grid_kernel<T, D, BS, TN::kWarps, TN::kStages, BIG, KV8, FAULT, SHORT>;
   static std::atomic<uint64_t> smem_set{0};  // per device, this instance
   dim3 grid = args.units == nullptr
