@@ -110,6 +110,10 @@ FP8_CASES = [
     (W.F16, 64, 8, 1, 600, 128),
     (W.BF16, 16, 32, 2, 500, 0),   # 16 query heads per kv head
     (W.BF16, 16, 4, 4, 1200, 16),  # one block per partition, merge kernel path
+    # groups that are not powers of two
+    (W.F16, 16, 12, 4, 900, 0),     # GQA 3: tokens on M, five idle head columns
+    (W.BF16, 32, 28, 4, 1500, 512),  # GQA 7
+    (W.F16, 64, 24, 2, 700, 64),    # GQA 12: query-rows form
 ]
 
 

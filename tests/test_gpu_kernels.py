@@ -124,6 +124,11 @@ DECODE_CASES = [
     (W.BF16, 64, 32, 32, 2, 400, 0),     # GQA 16 (rows 8..15 of the MMA)
     (W.F16, 128, 64, 32, 2, 700, 256),   # GQA 16, 64-token blocks
     (W.BF16, 128, 16, 2, 2, 1200, 16),   # one block per partition
+    # groups that are not powers of two: rows G..15 of the MMA idle
+    (W.F16, 128, 16, 12, 4, 600, 0),     # GQA 3
+    (W.BF16, 128, 32, 28, 4, 900, 256),  # GQA 7
+    (W.F16, 64, 16, 24, 2, 500, 64),     # GQA 12 (rows 8..11 of the second half)
+    (W.BF16, 128, 8, 10, 2, 400, 0),     # GQA 5, 8-token blocks
 ]
 
 

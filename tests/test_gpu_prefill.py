@@ -54,6 +54,8 @@ CASES = [
     (W.F16, 8, 16, 1, [333], [100]),
     (W.BF16, 64, 16, 8, [1000, 5, 70], [0, 5, 64]),
     (W.F16, 16, 4, 2, [128, 256, 129], [128, 128, 1]),
+    (W.BF16, 16, 32, 4, [513, 90, 1000], [513, 17, 300]),  # 8 query heads per kv head: 16 tokens a tile
+    (W.F16, 32, 16, 2, [64, 777], [64, 129]),
 ]
 
 
