@@ -39,6 +39,15 @@
  *     keeps the pointers, sizes and max_context_len it was captured with; the
  *     contents of the device arrays (inputs, lengths, tables, slots) may
  *     change between replays.
+ *   - Check build (PKV_CHECK).  The same sources compiled with PKV_CHECK
+ *     defined give libpkv_check.so (`python -m paged_kv_cache_407_b200.build
+ *     --check`), a debugging build that also verifies the caller guarantees
+ *     the kernels cannot see cheaply: no slot repeats in one cache write, no
+ *     copy destination repeats or is also a source.  Those calls then copy
+ *     the index array to the host and synchronise the stream before queuing
+ *     anything, so a check build cannot be captured in a CUDA graph (the call
+ *     returns PKV_ERR_CUDA while its stream is capturing).  pkv_check_build()
+ *     tells the two builds apart.
  *
  * Cache layout ("HND"): k_cache and v_cache are separate pools, each
  *   [num_blocks][num_kv_heads][block_size][head_dim] row-major, element type
@@ -75,7 +84,9 @@ typedef enum {
   PKV_ERR_CUDA = 8,           /* a CUDA runtime/driver call failed (launch, attribute, tensor map) */
   PKV_ERR_DEVICE = 9,         /* current device is not compute capability 10.0 (B200 / sm_100a) */
   PKV_ERR_NO_BLOCKS = 10,     /* block manager: the free pool cannot supply the blocks asked for */
-  PKV_ERR_BAD_SEQUENCE = 11   /* block manager: unknown, repeated or already present sequence id */
+  PKV_ERR_BAD_SEQUENCE = 11,  /* block manager: unknown, repeated or already present sequence id */
+  PKV_ERR_ALIAS = 12          /* check build only: a slot repeats within one cache write, or a
+                                 copy pair's dst repeats or is also a src (see PKV_CHECK below) */
 } pkv_status;
 
 /* Device-side error bits OR-ed into *d_status. */
@@ -131,7 +142,8 @@ typedef struct {
  * Errors: NULL pointers (when num_tokens > 0), bad desc or 8-bit pools
  *   -> status; a slot >= num_blocks*B -> PKV_DEV_BAD_SLOT, that token skipped.
  *   Two tokens with the same slot in one call race (caller error, result
- *   unspecified).
+ *   unspecified); a check build returns PKV_ERR_ALIAS instead, before
+ *   writing anything (negative slots may repeat).
  */
 PKV_API pkv_status pkv_reshape_and_cache(const void *key, const void *value, int64_t key_token_stride,
                                  int64_t value_token_stride, void *k_cache, void *v_cache,
@@ -232,7 +244,9 @@ PKV_API pkv_status pkv_paged_attention_decode(void *out, const void *query, cons
  * block_pairs  device, int64 [num_pairs][2] = (src, dst).
  * Errors: a src or dst outside [0, num_blocks) -> PKV_DEV_BAD_BLOCK and that
  *   pair is skipped.  A dst that repeats, or that is also a src in the same
- *   call, races (caller error, result unspecified).
+ *   call (its own included), races (caller error, result unspecified); a
+ *   check build returns PKV_ERR_ALIAS instead, before copying anything
+ *   (pairs the kernel would skip are left out of that check).
  */
 PKV_API pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_desc cache,
                            const int64_t *block_pairs, int32_t num_pairs, int32_t *d_status,
@@ -278,7 +292,7 @@ PKV_API pkv_status pkv_paged_attention_decode_noalloc(
  * k_cache[p / B][h][p % B][:] and V codes to v_cache[p / B][h][:][p % B].
  * key, value: fp16 or bf16 (input_dtype), same layout and strides as
  * pkv_reshape_and_cache; cache.dtype must be PKV_FP8_E4M3; k_scale, v_scale > 0.
- * Errors as pkv_reshape_and_cache.
+ * Errors as pkv_reshape_and_cache (PKV_ERR_ALIAS included).
  */
 PKV_API pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *value,
                                              int64_t key_token_stride, int64_t value_token_stride,
@@ -431,6 +445,9 @@ PKV_API const char *pkv_status_string(pkv_status status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 PKV_API int32_t pkv_version(void);
+
+/* 1 in a check build (PKV_CHECK defined: libpkv_check.so), 0 otherwise. */
+PKV_API int32_t pkv_check_build(void);
 
 #ifdef __cplusplus
 }

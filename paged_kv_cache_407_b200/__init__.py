@@ -9,11 +9,14 @@ from .binding import (  # noqa: F401
     DEV_BAD_LEN,
     DEV_BAD_SLOT,
     DEV_TIMEOUT,
+    CHECK_LIB_PATH,
+    ERR_ALIAS,
     LIB_PATH,
     PREFILL_WORKSPACE_BYTES,
     PkvError,
     PreparedCall,
     cache_desc,
+    check_library,
     copy_blocks,
     fp8_cache_desc,
     library,

@@ -14,6 +14,7 @@ import torch
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libpkv.so")
+CHECK_LIB_PATH = os.path.join(PKG_DIR, "libpkv_check.so")
 
 # pkv_status
 OK = 0
@@ -21,11 +22,12 @@ STATUS_NAMES = {
     0: "PKV_OK", 1: "PKV_ERR_NULL_POINTER", 2: "PKV_ERR_BAD_DTYPE", 3: "PKV_ERR_BAD_SHAPE",
     4: "PKV_ERR_MISALIGNED", 5: "PKV_ERR_WORKSPACE", 6: "PKV_ERR_BAD_PARTITION",
     7: "PKV_ERR_TOO_LARGE", 8: "PKV_ERR_CUDA", 9: "PKV_ERR_DEVICE",
-    10: "PKV_ERR_NO_BLOCKS", 11: "PKV_ERR_BAD_SEQUENCE",
+    10: "PKV_ERR_NO_BLOCKS", 11: "PKV_ERR_BAD_SEQUENCE", 12: "PKV_ERR_ALIAS",
 }
 ERR_TOO_LARGE = 7
 ERR_NO_BLOCKS = 10
 ERR_BAD_SEQUENCE = 11
+ERR_ALIAS = 12
 # device-side flags
 DEV_BAD_BLOCK = 0x1
 DEV_BAD_SLOT = 0x2
@@ -103,9 +105,11 @@ SIGNATURES = {
     "pkv_bm_block_tables": (ctypes.c_int, [_c_void_p, _c_void_p, _i32, _c_void_p, _i32, _c_void_p]),
     "pkv_bm_free_list": (ctypes.c_int, [_c_void_p, _c_void_p, _i32, ctypes.POINTER(_i32)]),
     "pkv_version": (_i32, []),
+    "pkv_check_build": (_i32, []),
 }
 
 _lib = None
+_check_lib = None
 
 
 class PkvError(RuntimeError):
@@ -116,20 +120,38 @@ class PkvError(RuntimeError):
         super().__init__(f"{where}: {name} ({text})")
 
 
+def load(path: str) -> ctypes.CDLL:
+    """Open one build of the library and give every entry point its C
+    signature.  Raises if the file is missing."""
+    if not os.path.exists(path):
+        flag = " --check" if path == CHECK_LIB_PATH else ""
+        raise RuntimeError(f"{path} is missing: build it with `python -m paged_kv_cache_407_b200.build{flag}`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def library() -> ctypes.CDLL:
-    """Load libpkv.so (once).  Raises if it has not been built."""
+    """Load libpkv.so (once), or its check build libpkv_check.so when the
+    environment sets PKV_CHECK=1 (the cache write and the block copy then
+    verify that no slot / copy destination repeats, synchronising the
+    stream; see include/pkv.h).  Raises if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_407_b200.build`")
-        lib = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(lib, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = lib
+        _lib = load(CHECK_LIB_PATH if os.environ.get("PKV_CHECK", "0") == "1" else LIB_PATH)
     return _lib
+
+
+def check_library() -> ctypes.CDLL:
+    """The check build, loaded (once) beside whichever build library()
+    serves; its calls take the same C arguments."""
+    global _check_lib
+    if _check_lib is None:
+        _check_lib = load(CHECK_LIB_PATH)
+    return _check_lib
 
 
 def _check(status: int, where: str) -> None:

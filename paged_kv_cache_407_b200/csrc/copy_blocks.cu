@@ -5,6 +5,7 @@
 // request diverges inside a shared block, that block is copied first.  Each
 // (src, dst) pair makes block dst of both pools a bit copy of block src.
 #include "pkv_device.cuh"
+#include "alias_check.h"
 #include "pkv_host.h"
 
 namespace pkv {
@@ -58,6 +59,11 @@ extern "C" pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, pkv_cache_de
     return PKV_ERR_MISALIGNED;
   if (num_pairs > 2147483647 / 2) return PKV_ERR_TOO_LARGE;
   if ((st = check_device()) != PKV_OK) return st;
+#ifdef PKV_CHECK
+  if ((st = check_copy_pairs(block_pairs, num_pairs, cache.num_blocks, reinterpret_cast<cudaStream_t>(stream))) !=
+      PKV_OK)
+    return st;
+#endif
   const int64_t block_vecs = static_cast<int64_t>(cache.num_kv_heads) * cache.block_size *
                              cache.head_dim * elem_bytes(cache.dtype) / 16;
   const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyUnroll;

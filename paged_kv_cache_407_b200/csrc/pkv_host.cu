@@ -174,6 +174,7 @@ extern "C" const char *pkv_status_string(pkv_status s) {
     case PKV_ERR_DEVICE: return "current device is not compute capability 10.0 (B200, sm_100a)";
     case PKV_ERR_NO_BLOCKS: return "the free block pool cannot supply the blocks asked for";
     case PKV_ERR_BAD_SEQUENCE: return "unknown, repeated or already present sequence id";
+    case PKV_ERR_ALIAS: return "a slot repeats in one cache write, or a copy destination repeats or is also a source";
   }
   return "unknown pkv_status";
 }

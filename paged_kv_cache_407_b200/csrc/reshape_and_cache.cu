@@ -10,6 +10,7 @@
 #include <cuda_fp8.h>
 
 #include "pkv_device.cuh"
+#include "alias_check.h"
 #include "pkv_host.h"
 
 namespace pkv {
@@ -179,6 +180,10 @@ extern "C" pkv_status pkv_reshape_and_cache_fp8(const void *key, const void *val
       !aligned(key, 2) || !aligned(value, 2))
     return PKV_ERR_MISALIGNED;
   if ((st = check_device()) != PKV_OK) return st;
+#ifdef PKV_CHECK
+  if ((st = check_unique_slots(slot_mapping, num_tokens, reinterpret_cast<cudaStream_t>(stream))) != PKV_OK)
+    return st;
+#endif
   const int64_t num_slots = static_cast<int64_t>(cache.num_blocks) * cache.block_size;
   const int threads = 256;
   const int64_t items = static_cast<int64_t>(num_tokens) * cache.num_kv_heads * (cache.head_dim / 4);
@@ -229,6 +234,10 @@ extern "C" pkv_status pkv_reshape_and_cache(const void *key, const void *value,
       !aligned(key, 2) || !aligned(value, 2))
     return PKV_ERR_MISALIGNED;
   if ((st = check_device()) != PKV_OK) return st;
+#ifdef PKV_CHECK
+  if ((st = check_unique_slots(slot_mapping, num_tokens, reinterpret_cast<cudaStream_t>(stream))) != PKV_OK)
+    return st;
+#endif
 
   const int64_t num_slots = static_cast<int64_t>(cache.num_blocks) * cache.block_size;
   const bool vec = aligned(key, 16) && aligned(value, 16) && key_token_stride % 8 == 0 &&

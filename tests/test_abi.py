@@ -52,10 +52,41 @@ def test_only_declared_symbols_are_exported():
 
 
 def test_status_strings_and_version(lib):
-    for code in range(12):
-        assert lib.pkv_status_string(code)
+    for code in range(13):
+        assert lib.pkv_status_string(code) != b"unknown pkv_status"
     assert lib.pkv_status_string(0) == b"ok"
     assert bd.version() >= 100
+
+
+@pytest.fixture(scope="module")
+def check_lib():
+    from paged_kv_cache_407_b200.build import build_check
+    build_check()
+    return bd.check_library()
+
+
+def test_check_build_exports_the_same_abi(lib, check_lib):
+    """libpkv_check.so (PKV_CHECK) declares and exports exactly what
+    libpkv.so does, and says which build it is."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", bd.CHECK_LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if l.split()[-2:-1] == ["T"]}
+    assert {s for s in exported if s.startswith("pkv_")} == set(declared_functions())
+    assert check_lib.pkv_check_build() == 1 and lib.pkv_check_build() == 0
+    assert check_lib.pkv_status_string(bd.ERR_ALIAS) == lib.pkv_status_string(bd.ERR_ALIAS)
+
+
+def test_check_build_validates_arguments_before_its_alias_checks(check_lib):
+    """The host-side argument checks come first and are the regular build's;
+    calls with nothing to write or copy return at once, touching no device."""
+    null = None
+    d = bd.CacheDesc(16, 16, 4, 64, 0)
+    assert check_lib.pkv_reshape_and_cache(null, null, 0, 0, null, null, d, null, 1, null, null) == 1
+    assert check_lib.pkv_reshape_and_cache(null, null, 0, 0, null, null, d, null, 0, null, null) == 0
+    assert check_lib.pkv_copy_blocks(null, null, d, null, 0, null, null) == 0
+    assert check_lib.pkv_copy_blocks(null, null, d, null, 2, null, null) == 1
+    assert check_lib.pkv_copy_blocks(null, null, bd.CacheDesc(16, 12, 4, 64, 0), null, 2, null, null) == 3
 
 
 def _desc(N=16, B=16, H=4, D=64, dt=0):
