@@ -242,3 +242,15 @@ def test_withheld_load_entry_validates_on_the_host(lib):
     assert call(wait_us=0) == 3 and call(wait_us=2_000_000) == 3
     assert call(block=-1) == 3
     assert call(block=32) == 6                                   # past the first 512-token partition
+
+
+def test_environment_selects_the_check_build(check_lib):
+    """With PKV_CHECK=1 the binding's library() serves libpkv_check.so."""
+    import subprocess
+    import sys
+    code = ("from paged_kv_cache_407_b200 import binding as bd; "
+            "assert bd.library().pkv_check_build() == 1; "
+            "assert bd.library()._name == bd.CHECK_LIB_PATH; print('ok')")
+    env = dict(os.environ, PKV_CHECK="1")
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", res.stderr
