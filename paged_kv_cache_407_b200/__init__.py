@@ -30,6 +30,7 @@ from .binding import (  # noqa: F401
     reshape_and_cache_fp8,
     state_buffer,
     state_views,
+    use_check_build,
     version,
     workspace_size,
 )

@@ -135,23 +135,33 @@ def load(path: str) -> ctypes.CDLL:
 
 
 def library() -> ctypes.CDLL:
-    """Load libpkv.so (once), or its check build libpkv_check.so when the
-    environment sets PKV_CHECK=1 (the cache write and the block copy then
-    verify that no slot / copy destination repeats, synchronising the
-    stream; see include/pkv.h).  Raises if it has not been built."""
+    """The build every binding call goes through: libpkv.so, loaded on first
+    use, unless use_check_build() chose the check build first.  Raises if it
+    has not been built."""
     global _lib
     if _lib is None:
-        _lib = load(CHECK_LIB_PATH if os.environ.get("PKV_CHECK", "0") == "1" else LIB_PATH)
+        _lib = load(LIB_PATH)
     return _lib
 
 
 def check_library() -> ctypes.CDLL:
-    """The check build, loaded (once) beside whichever build library()
-    serves; its calls take the same C arguments."""
+    """The check build libpkv_check.so (PKV_CHECK: the cache write and the
+    block copy also verify that no slot / copy destination repeats,
+    synchronising the stream; see include/pkv.h), loaded once, beside
+    whichever build library() serves.  Its calls take the same C arguments."""
     global _check_lib
     if _check_lib is None:
         _check_lib = load(CHECK_LIB_PATH)
     return _check_lib
+
+
+def use_check_build() -> None:
+    """Route every later binding call to the check build.  Call it before the
+    first library call of the process; raises if libpkv.so is already in use."""
+    global _lib
+    if _lib is not None and _lib is not check_library():
+        raise RuntimeError("libpkv.so is already in use: call use_check_build() before the first library call")
+    _lib = check_library()
 
 
 def _check(status: int, where: str) -> None:

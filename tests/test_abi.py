@@ -244,13 +244,17 @@ def test_withheld_load_entry_validates_on_the_host(lib):
     assert call(block=32) == 6                                   # past the first 512-token partition
 
 
-def test_environment_selects_the_check_build(check_lib):
-    """With PKV_CHECK=1 the binding's library() serves libpkv_check.so."""
+def test_binding_can_route_every_call_to_the_check_build(check_lib):
+    """use_check_build() before the first call makes library() serve
+    libpkv_check.so; after the regular build is in use it refuses."""
     import subprocess
     import sys
-    code = ("from paged_kv_cache_407_b200 import binding as bd; "
-            "assert bd.library().pkv_check_build() == 1; "
-            "assert bd.library()._name == bd.CHECK_LIB_PATH; print('ok')")
-    env = dict(os.environ, PKV_CHECK="1")
-    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True)
+    code = ("from paged_kv_cache_407_b200 import binding as bd; bd.use_check_build(); "
+            "assert bd.library().pkv_check_build() == 1; assert bd.library()._name == bd.CHECK_LIB_PATH; "
+            "print('ok')")
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
     assert res.returncode == 0 and res.stdout.strip() == "ok", res.stderr
+    code = ("from paged_kv_cache_407_b200 import binding as bd; bd.library()\n"
+            "try:\n    bd.use_check_build()\nexcept RuntimeError:\n    print('refused')")
+    res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
+    assert res.returncode == 0 and res.stdout.strip() == "refused", res.stderr
