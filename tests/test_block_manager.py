@@ -135,3 +135,28 @@ def test_host_arrays_feed_the_device_calls():
     assert copies.dtype == np.int64 and copies.shape == (0, 2)
     assert tables.dtype == np.int32 and tables.shape == (5, 10) and (tables[:, 8:] == -1).all()
     assert lens.dtype == np.int32 and lens.tolist() == [11 + 7 * s for s in range(5)]
+
+
+
+def test_concurrent_native_threads_keep_one_manager_consistent(tmp_path):
+    """Calls on one manager are serialised by its lock.  tests/native/
+    bm_threads.cpp, built against libpkv.so, runs eight host threads that
+    add, fork, extend and free their own requests on one shared pool (which
+    runs dry, so steps are refused too) and then checks the lengths, the
+    reference counts and the free pool against what the threads did.  Built
+    from the same source with the lock taken out, that program crashes or
+    reports inconsistencies."""
+    import os
+    import shutil
+    import subprocess
+    from paged_kv_cache_407_b200.build import INCLUDE, LIB_PATH
+    cxx = os.environ.get("CXX") or shutil.which("g++") or shutil.which("c++")
+    assert cxx, "a host C++ compiler is needed"
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "native", "bm_threads.cpp")
+    exe = str(tmp_path / "bm_threads")
+    libdir = os.path.dirname(LIB_PATH)
+    subprocess.run([cxx, "-O2", "-std=c++17", "-pthread", "-I", INCLUDE, src, "-L", libdir, "-lpkv",
+                    f"-Wl,-rpath,{libdir}", "-o", exe], check=True, capture_output=True, text=True)
+    for threads, steps in ((8, 4000), (16, 2000)):
+        res = subprocess.run([exe, str(threads), str(steps)], capture_output=True, text=True, timeout=120)
+        assert res.returncode == 0 and "inconsistencies 0" in res.stdout, (res.returncode, res.stdout, res.stderr)
