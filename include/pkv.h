@@ -46,8 +46,9 @@
  *     copy destination repeats or is also a source.  Those calls then copy
  *     the index array to the host and synchronise the stream before queuing
  *     anything, so a check build cannot be captured in a CUDA graph (the call
- *     returns PKV_ERR_CUDA while its stream is capturing).  pkv_check_build()
- *     tells the two builds apart.
+ *     returns PKV_ERR_CUDA while its stream is capturing, PKV_ERR_TOO_LARGE
+ *     when the host copy cannot be allocated).  pkv_check_build() tells the
+ *     two builds apart.
  *
  * Cache layout ("HND"): k_cache and v_cache are separate pools, each
  *   [num_blocks][num_kv_heads][block_size][head_dim] row-major, element type

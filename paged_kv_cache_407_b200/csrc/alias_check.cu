@@ -6,6 +6,7 @@
 // private block from a block that is only read).  The regular build leaves
 // both unchecked (the kernels would race; the result is unspecified).
 #include <algorithm>
+#include <new>
 #include <vector>
 
 #include "alias_check.h"
@@ -40,7 +41,7 @@ bool has_repeat(std::vector<int64_t> &v) {
 
 }  // namespace
 
-pkv_status check_unique_slots(const int64_t *slot_mapping, int32_t num_tokens, cudaStream_t stream) {
+pkv_status check_unique_slots(const int64_t *slot_mapping, int32_t num_tokens, cudaStream_t stream) try {
   if (num_tokens <= 0) return PKV_OK;
   std::vector<int64_t> h;
   pkv_status st = fetch(h, slot_mapping, static_cast<size_t>(num_tokens), stream);
@@ -50,10 +51,12 @@ pkv_status check_unique_slots(const int64_t *slot_mapping, int32_t num_tokens, c
   for (const int64_t p : h)
     if (p >= 0) used.push_back(p);  // negative slots are padding: they write nothing
   return has_repeat(used) ? PKV_ERR_ALIAS : PKV_OK;
+} catch (const std::bad_alloc &) {
+  return PKV_ERR_TOO_LARGE;  // no host memory for the copy: nothing was queued
 }
 
 pkv_status check_copy_pairs(const int64_t *block_pairs, int32_t num_pairs, int64_t num_blocks,
-                            cudaStream_t stream) {
+                            cudaStream_t stream) try {
   if (num_pairs <= 0) return PKV_OK;
   std::vector<int64_t> h;
   pkv_status st = fetch(h, block_pairs, 2 * static_cast<size_t>(num_pairs), stream);
@@ -70,6 +73,8 @@ pkv_status check_copy_pairs(const int64_t *block_pairs, int32_t num_pairs, int64
   for (const int64_t d : dsts)
     if (std::binary_search(srcs.begin(), srcs.end(), d)) return PKV_ERR_ALIAS;
   return PKV_OK;
+} catch (const std::bad_alloc &) {
+  return PKV_ERR_TOO_LARGE;
 }
 
 }  // namespace pkv

@@ -11,6 +11,8 @@ namespace pkv {
 
 // PKV_ERR_ALIAS if a non-negative slot occurs twice among the num_tokens
 // device-resident slots (copied to the host; the stream is synchronised).
+// PKV_ERR_CUDA if the copy fails or the stream is capturing;
+// PKV_ERR_TOO_LARGE if the host copy cannot be allocated.
 pkv_status check_unique_slots(const int64_t *slot_mapping, int32_t num_tokens, cudaStream_t stream);
 
 // PKV_ERR_ALIAS if, among the (src, dst) pairs with both ids in
