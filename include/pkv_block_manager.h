@@ -32,7 +32,9 @@
  * Ownership and threading: a manager is created and destroyed by the caller;
  * all pointers passed in are host memory owned by the caller; calls on one
  * manager are serialised by an internal lock.  Sequence ids are any int64.
- * On an error the manager is unchanged.  No call touches the GPU.
+ * On an error the manager is unchanged.  A call that runs out of host memory
+ * returns PKV_ERR_TOO_LARGE (pkv_bm_blocks_needed: -1), also with the manager
+ * unchanged; no C++ exception leaves these calls.  No call touches the GPU.
  */
 #ifndef PKV_BLOCK_MANAGER_H_
 #define PKV_BLOCK_MANAGER_H_

@@ -113,17 +113,20 @@ struct pkv_block_manager {
   }
 };
 
+// No C++ exception leaves the C ABI: the calls that allocate host memory
+// return PKV_ERR_TOO_LARGE when it runs out, and they allocate before they
+// change anything, so the manager is then unchanged.
 extern "C" {
 
 pkv_status pkv_bm_create(int32_t num_blocks, int32_t block_size, int32_t max_blocks_per_seq,
-                         pkv_block_manager **out) {
+                         pkv_block_manager **out) try {
   if (out == nullptr) return PKV_ERR_NULL_POINTER;
   *out = nullptr;
   if (num_blocks < 1 || block_size < 1 || max_blocks_per_seq < 1) return PKV_ERR_BAD_SHAPE;
-  auto *bm = new (std::nothrow) pkv_block_manager(num_blocks, block_size, max_blocks_per_seq);
-  if (bm == nullptr) return PKV_ERR_TOO_LARGE;
-  *out = bm;
+  *out = new pkv_block_manager(num_blocks, block_size, max_blocks_per_seq);
   return PKV_OK;
+} catch (const std::bad_alloc &) {
+  return PKV_ERR_TOO_LARGE;
 }
 
 void pkv_bm_destroy(pkv_block_manager *bm) { delete bm; }
@@ -154,7 +157,7 @@ int32_t pkv_bm_context_len(const pkv_block_manager *bm, int64_t seq_id) {
 }
 
 pkv_status pkv_bm_add_sequence(pkv_block_manager *bm, int64_t seq_id, int32_t num_tokens,
-                               int64_t *slot_mapping) {
+                               int64_t *slot_mapping) try {
   if (bm == nullptr) return PKV_ERR_NULL_POINTER;
   if (num_tokens < 0) return PKV_ERR_BAD_SHAPE;
   std::lock_guard<std::mutex> g(bm->mu);
@@ -165,24 +168,29 @@ pkv_status pkv_bm_add_sequence(pkv_block_manager *bm, int64_t seq_id, int32_t nu
   if (nb > bm->pool.size()) return PKV_ERR_NO_BLOCKS;
   Sequence q;
   q.table.reserve(static_cast<size_t>(nb));
+  Sequence &dst = bm->seqs.emplace(seq_id, Sequence{}).first->second;  // the last allocation
   for (int64_t j = 0; j < nb; ++j) q.table.push_back(bm->take());
   q.len = num_tokens;
   if (slot_mapping != nullptr)
     for (int64_t t = 0; t < num_tokens; ++t)
       slot_mapping[t] = static_cast<int64_t>(q.table[static_cast<size_t>(t / B)]) * B + t % B;
-  bm->seqs.emplace(seq_id, std::move(q));
+  dst = std::move(q);
   return PKV_OK;
+} catch (const std::bad_alloc &) {
+  return PKV_ERR_TOO_LARGE;
 }
 
-pkv_status pkv_bm_fork(pkv_block_manager *bm, int64_t parent_id, int64_t child_id) {
+pkv_status pkv_bm_fork(pkv_block_manager *bm, int64_t parent_id, int64_t child_id) try {
   if (bm == nullptr) return PKV_ERR_NULL_POINTER;
   std::lock_guard<std::mutex> g(bm->mu);
   auto it = bm->seqs.find(parent_id);
   if (it == bm->seqs.end() || bm->seqs.count(child_id)) return PKV_ERR_BAD_SEQUENCE;
   Sequence child = it->second;
-  for (int32_t b : child.table) ++bm->ref[static_cast<size_t>(b)];
-  bm->seqs.emplace(child_id, std::move(child));
+  const Sequence &added = bm->seqs.emplace(child_id, std::move(child)).first->second;
+  for (int32_t b : added.table) ++bm->ref[static_cast<size_t>(b)];
   return PKV_OK;
+} catch (const std::bad_alloc &) {
+  return PKV_ERR_TOO_LARGE;
 }
 
 pkv_status pkv_bm_free_sequence(pkv_block_manager *bm, int64_t seq_id) {
@@ -195,17 +203,19 @@ pkv_status pkv_bm_free_sequence(pkv_block_manager *bm, int64_t seq_id) {
   return PKV_OK;
 }
 
-int32_t pkv_bm_blocks_needed(const pkv_block_manager *cbm, const int64_t *seq_ids, int32_t n) {
+int32_t pkv_bm_blocks_needed(const pkv_block_manager *cbm, const int64_t *seq_ids, int32_t n) try {
   if (cbm == nullptr || n < 0 || (n > 0 && seq_ids == nullptr)) return -1;
   auto *bm = const_cast<pkv_block_manager *>(cbm);  // only the scratch vectors change
   std::lock_guard<std::mutex> g(bm->mu);
   if (!bm->resolve(seq_ids, n)) return -1;
   return static_cast<int32_t>(bm->needed());
+} catch (const std::bad_alloc &) {
+  return -1;
 }
 
 pkv_status pkv_bm_append(pkv_block_manager *bm, const int64_t *seq_ids, int32_t n,
                          int64_t *slot_mapping, int64_t *copy_pairs, int32_t copy_capacity,
-                         int32_t *num_copies) {
+                         int32_t *num_copies) try {
   if (bm == nullptr) return PKV_ERR_NULL_POINTER;
   if (n < 0 || copy_capacity < n) return PKV_ERR_BAD_SHAPE;
   if (n > 0 && (seq_ids == nullptr || slot_mapping == nullptr || copy_pairs == nullptr))
@@ -219,6 +229,8 @@ pkv_status pkv_bm_append(pkv_block_manager *bm, const int64_t *seq_ids, int32_t 
     if (q->len % B == 0 && static_cast<int64_t>(q->table.size()) + 1 > bm->max_blocks)
       return PKV_ERR_TOO_LARGE;
   if (bm->needed() > bm->pool.size()) return PKV_ERR_NO_BLOCKS;
+  for (Sequence *q : bm->batch)  // the step's only allocations, before anything changes
+    if (q->len % B == 0) q->table.reserve(q->table.size() + 1);
   int32_t copies = 0;
   for (int32_t i = 0; i < n; ++i) {
     Sequence *q = bm->batch[static_cast<size_t>(i)];
@@ -238,6 +250,8 @@ pkv_status pkv_bm_append(pkv_block_manager *bm, const int64_t *seq_ids, int32_t 
   }
   *num_copies = copies;
   return PKV_OK;
+} catch (const std::bad_alloc &) {
+  return PKV_ERR_TOO_LARGE;
 }
 
 pkv_status pkv_bm_block_tables(const pkv_block_manager *cbm, const int64_t *seq_ids, int32_t n,
