@@ -258,3 +258,22 @@ def test_binding_can_route_every_call_to_the_check_build(check_lib):
             "try:\n    bd.use_check_build()\nexcept RuntimeError:\n    print('refused')")
     res = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True)
     assert res.returncode == 0 and res.stdout.strip() == "refused", res.stderr
+
+
+def test_headers_are_plain_c_and_usable_from_c(lib, tmp_path):
+    """tests/native/c_client.c includes both headers as strict C99 (no
+    warning with -pedantic), links libpkv.so and checks the calls that need
+    no GPU: status text, version, host-side argument checks, and the block
+    manager through a prompt, a fork, a copy-on-write step and a free."""
+    import shutil
+    import subprocess
+    from paged_kv_cache_407_b200.build import INCLUDE, LIB_PATH
+    cc = os.environ.get("CC") or shutil.which("gcc") or shutil.which("cc")
+    assert cc, "a host C compiler is needed"
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "native", "c_client.c")
+    exe = str(tmp_path / "c_client")
+    libdir = os.path.dirname(LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", INCLUDE, src, "-L", libdir,
+                    "-lpkv", f"-Wl,-rpath,{libdir}", "-o", exe], check=True, capture_output=True, text=True)
+    res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0 and res.stdout.strip() == "c client ok", (res.stdout, res.stderr)
